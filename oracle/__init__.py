@@ -1,0 +1,179 @@
+"""fp64 CPU oracle of the sparse-MoE FFN layer forward -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference leg of
+``bench.py`` may import this package.  The product path (``sparse_mixture_experts_16_b200``)
+never does, and shares no code with it.
+
+The arithmetic lives in ``moe_oracle.cpp`` (plain C++ loops in fp64 over exact bf16 inputs);
+this module only compiles it with g++ and marshals numpy arrays.  Pins that tie it to the
+pages and to mathematics (not to itself) are in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.cpp")
+_LIB = os.path.join(_HERE, "libmoe_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    if os.path.exists(_LIB) and not force and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    subprocess.run(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
+                    "-o", _LIB + ".tmp", _SRC], check=True)
+    os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int
+        L.oracle_router.argtypes = [P, P, P, i64, i64, i32, i32, P, P, P, i32]
+        L.oracle_topk_exhaustive.argtypes = [P, i64, i32, i32, P]
+        L.oracle_permute.argtypes = [P, i64, i32, i32, P, P, P, P, P]
+        L.oracle_expert_ffn.argtypes = [P, P, P, i64, i64, P]
+        L.oracle_expert_ffn.restype = None
+        L.oracle_layer.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, P, P, P, i32]
+        L.oracle_layer_eager.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, P]
+        _lib = L
+    return _lib
+
+
+def _nthreads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def router(x, wg, bias, k, return_logits=False, nthreads=None):
+    """idx[T,k] int32 (score-descending), p[T,k] float64 (and logits[T,E] float64)."""
+    x, wg = _u16(x), _u16(wg)
+    T, D = x.shape
+    E = wg.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    idx = np.empty((T, k), np.int32)
+    p = np.empty((T, k), np.float64)
+    lg = np.empty((T, E), np.float64) if return_logits else None
+    rc = _L().oracle_router(x.ctypes.data, wg.ctypes.data, _ptr(b), T, D, E, k, _ptr(lg), idx.ctypes.data,
+                            p.ctypes.data, nthreads or _nthreads())
+    if rc != 0:
+        raise ValueError(f"oracle_router rc={rc}")
+    return (idx, p, lg) if return_logits else (idx, p)
+
+
+def topk_exhaustive(scores, k):
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    T, E = s.shape
+    idx = np.empty((T, k), np.int32)
+    rc = _L().oracle_topk_exhaustive(s.ctypes.data, T, E, k, idx.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_topk_exhaustive rc={rc}")
+    return idx
+
+
+def permute(idx, E):
+    """counts[E], offsets[E+1], perm_token[T*k], perm_slot[T*k], inv_perm[T*k] (all int32)."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, k = idx.shape
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    pt = np.empty(T * k, np.int32)
+    ps = np.empty(T * k, np.int32)
+    inv = np.empty(T * k, np.int32)
+    rc = _L().oracle_permute(idx.ctypes.data, T, E, k, counts.ctypes.data, offsets.ctypes.data,
+                             pt.ctypes.data, ps.ctypes.data, inv.ctypes.data)
+    if rc != 0:
+        raise ValueError("expert id out of range")
+    return counts, offsets, pt, ps, inv
+
+
+def expert_ffn(x_row, gate_up_e, down_e):
+    x_row, gu, dn = _u16(x_row), _u16(gate_up_e), _u16(down_e)
+    D = x_row.shape[-1]
+    F = dn.shape[1]
+    assert gu.shape == (2 * F, D) and dn.shape == (D, F)
+    out = np.empty(D, np.float64)
+    _L().oracle_expert_ffn(x_row.ctypes.data, gu.ctypes.data, dn.ctypes.data, D, F, out.ctypes.data)
+    return out
+
+
+def layer(x, wg, bias, gate_up, down, k, shared_gate_up=None, shared_down=None, nthreads=None,
+          F=None):
+    """y[T,D] float64 plus (idx, p).
+
+    gate_up / down are either packed arrays [E,2F,D] / [E,D,F] or dicts {expert: array} holding
+    only the experts that the tokens of ``x`` route to (for sampled checks at full size).
+    """
+    x, wg = _u16(x), _u16(wg)
+    T, D = x.shape
+    E = wg.shape[0]
+    keep = []
+    if isinstance(gate_up, dict):
+        gu_ptrs = (ctypes.c_void_p * E)()
+        dn_ptrs = (ctypes.c_void_p * E)()
+        for e, a in gate_up.items():
+            a = _u16(a)
+            keep.append(a)
+            gu_ptrs[e] = a.ctypes.data
+            F = a.shape[0] // 2
+        for e, a in down.items():
+            a = _u16(a)
+            keep.append(a)
+            dn_ptrs[e] = a.ctypes.data
+    else:
+        gate_up, down = _u16(gate_up), _u16(down)
+        keep += [gate_up, down]
+        F = gate_up.shape[1] // 2
+        gu_ptrs = (ctypes.c_void_p * E)(*[gate_up.ctypes.data + e * gate_up[0].nbytes for e in range(E)])
+        dn_ptrs = (ctypes.c_void_p * E)(*[down.ctypes.data + e * down[0].nbytes for e in range(E)])
+    sgu = None if shared_gate_up is None else _u16(shared_gate_up)
+    sdn = None if shared_down is None else _u16(shared_down)
+    Fs = 0 if sgu is None else sgu.shape[0] // 2
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    y = np.empty((T, D), np.float64)
+    idx = np.empty((T, k), np.int32)
+    p = np.empty((T, k), np.float64)
+    rc = _L().oracle_layer(x.ctypes.data, wg.ctypes.data, _ptr(b), gu_ptrs, dn_ptrs, _ptr(sgu), _ptr(sdn),
+                           T, D, E, k, F, Fs, y.ctypes.data, idx.ctypes.data, p.ctypes.data,
+                           nthreads or _nthreads())
+    if rc != 0:
+        raise ValueError(f"oracle_layer rc={rc}")
+    return y, idx, p
+
+
+def layer_eager(x, wg, bias, gate_up, down, k, shared_gate_up=None, shared_down=None):
+    x, wg, gate_up, down = _u16(x), _u16(wg), _u16(gate_up), _u16(down)
+    T, D = x.shape
+    E = wg.shape[0]
+    F = gate_up.shape[1] // 2
+    sgu = None if shared_gate_up is None else _u16(shared_gate_up)
+    sdn = None if shared_down is None else _u16(shared_down)
+    Fs = 0 if sgu is None else sgu.shape[0] // 2
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    y = np.empty((T, D), np.float64)
+    rc = _L().oracle_layer_eager(x.ctypes.data, wg.ctypes.data, _ptr(b), gate_up.ctypes.data,
+                                 down.ctypes.data, _ptr(sgu), _ptr(sdn), T, D, E, k, F, Fs, y.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle_layer_eager rc={rc}")
+    return y

@@ -1,0 +1,263 @@
+// moe_oracle.cpp -- plain fp64 CPU oracle of the sparse Mixture-of-Experts FFN layer forward.
+//
+// TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's CPU-baseline
+// leg load this code.  It shares no source with the CUDA path.  Every function is the plain
+// definition, written for a reader to check against the pages by eye:
+//
+//   * josueisai.com, "Mixture of experts: por que un modelo enorme apenas usa sus parametros",
+//     section "El router: la pieza que de verdad decide": the router is a linear projection
+//     followed by a softmax; the k best experts are kept, the softmax is normalised only over
+//     the chosen k, and the chosen experts' outputs are summed weighted by those scores; the
+//     eager per-expert loop printed there is the procedural form (oracle_layer_eager below).
+//   * gotburnout.io glossary "MoE (Mixture of Experts)", section 2 (layer diagram):
+//     p = Softmax(TopK(W_g x)), y = sum_i p_i Expert_i(x) (+ residual, which the caller adds),
+//     shared experts always active; section 3 step 3: the SwiGLU expert FFN.
+//   * dev.smart-guide.co.kr deep-dive, section "La Solucion: WeightConverter": the packed
+//     gate_up_proj tensor is the per-expert w1 and w3 matrices merged along a new expert dim 0
+//     and concatenated along dim 1 (w1 first), so gate_up[e] = [w1_e ; w3_e], shape [2F, D].
+//
+// Readings taken where the pages are silent or garbled (each is repeated in the design notes):
+//   - SiLU goes on rows [0, F) of gate_up[e] (w1, "gate"); rows [F, 2F) (w3, "up") multiply.
+//   - The optional per-expert bias (aux-loss-free balancing) enters the selection only; the
+//     weights p use the unbiased logits.
+//   - top-k order: score descending, ties to the lower expert id.
+//   - expert-contiguous order: experts ascending, tokens ascending within an expert.
+//   - the shared expert is added with coefficient 1.
+//   - no intermediate rounding: bf16 inputs are read as exact doubles and everything after is fp64.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+#include <algorithm>
+
+namespace {
+
+inline double bf16_value(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+template <class Fn>
+void for_tokens(int64_t T, int nthreads, Fn fn) {
+  if (nthreads <= 1 || T < 2) {
+    for (int64_t t = 0; t < T; ++t) fn(t);
+    return;
+  }
+  std::vector<std::thread> pool;
+  int n = (int)std::min<int64_t>(nthreads, T);
+  for (int w = 0; w < n; ++w)
+    pool.emplace_back([=] {
+      for (int64_t t = w; t < T; t += n) fn(t);
+    });
+  for (auto& th : pool) th.join();
+}
+
+// logits l[e] = sum_d x[d] * W_g[e, d] for one token (the router's linear projection)
+void router_logits(const uint16_t* x_row, const uint16_t* wg, int64_t D, int E, double* l) {
+  for (int e = 0; e < E; ++e) {
+    double acc = 0.0;
+    const uint16_t* w = wg + (int64_t)e * D;
+    for (int64_t d = 0; d < D; ++d) acc += bf16_value(x_row[d]) * bf16_value(w[d]);
+    l[e] = acc;
+  }
+}
+
+// Top-k selection on s = l + bias, then p = softmax over the chosen k of the unbiased l.
+void select_and_weight(const double* l, const float* bias, int E, int k, int32_t* idx, double* p) {
+  std::vector<double> s(E);
+  std::vector<char> taken(E, 0);
+  for (int e = 0; e < E; ++e) s[e] = l[e] + (bias ? (double)bias[e] : 0.0);
+  for (int j = 0; j < k; ++j) {
+    int best = -1;
+    for (int e = 0; e < E; ++e)
+      if (!taken[e] && (best < 0 || s[e] > s[best])) best = e;  // strict '>' keeps the lower id on ties
+    taken[best] = 1;
+    idx[j] = best;
+  }
+  double m = l[idx[0]];
+  for (int j = 1; j < k; ++j) m = std::max(m, l[idx[j]]);
+  double z = 0.0;
+  for (int j = 0; j < k; ++j) z += std::exp(l[idx[j]] - m);
+  for (int j = 0; j < k; ++j) p[j] = std::exp(l[idx[j]] - m) / z;
+}
+
+// One SwiGLU expert on one token: a = silu(G x) * (U x), out = Down a.
+// G = gate_up[0:F, :], U = gate_up[F:2F, :], Down = down[D, F]; silu(z) = z / (1 + e^-z).
+void expert_ffn(const uint16_t* x_row, const uint16_t* gate_up, const uint16_t* down, int64_t D,
+                int64_t F, double* out) {
+  std::vector<double> a(F);
+  for (int64_t n = 0; n < F; ++n) {
+    const uint16_t* grow = gate_up + n * D;
+    const uint16_t* urow = gate_up + (F + n) * D;
+    double g = 0.0, u = 0.0;
+    for (int64_t d = 0; d < D; ++d) {
+      double xv = bf16_value(x_row[d]);
+      g += bf16_value(grow[d]) * xv;
+      u += bf16_value(urow[d]) * xv;
+    }
+    a[n] = g / (1.0 + std::exp(-g)) * u;
+  }
+  for (int64_t d = 0; d < D; ++d) {
+    const uint16_t* drow = down + d * F;
+    double acc = 0.0;
+    for (int64_t n = 0; n < F; ++n) acc += bf16_value(drow[n]) * a[n];
+    out[d] = acc;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+// Router: idx[T, k] (score-descending) and p[T, k]; logits[T, E] if non-NULL.
+// Returns 0, or -1 on invalid sizes.
+int oracle_router(const uint16_t* x, const uint16_t* wg, const float* bias, int64_t T, int64_t D,
+                  int E, int k, double* logits, int32_t* idx, double* p, int nthreads) {
+  if (T < 0 || D < 1 || E < 1 || k < 1 || k > E) return -1;
+  for_tokens(T, nthreads, [&](int64_t t) {
+    std::vector<double> l(E);
+    router_logits(x + t * D, wg, D, E, l.data());
+    if (logits) std::copy(l.begin(), l.end(), logits + t * E);
+    select_and_weight(l.data(), bias, E, k, idx + t * k, p + t * k);
+  });
+  return 0;
+}
+
+// Top-k by exhaustive search over all k-subsets: the chosen set is the one with the largest
+// total score (with distinct scores this is exactly the set of the k largest), listed by
+// score descending.  Independent of the selection loop above; for small E only.
+int oracle_topk_exhaustive(const double* s, int64_t T, int E, int k, int32_t* idx) {
+  if (E > 20 || k < 1 || k > E) return -1;
+  for (int64_t t = 0; t < T; ++t) {
+    const double* st = s + t * E;
+    double best_sum = -INFINITY;
+    uint32_t best_mask = 0;
+    for (uint32_t mask = 0; mask < (1u << E); ++mask) {
+      if (__builtin_popcount(mask) != k) continue;
+      double sum = 0.0;
+      for (int e = 0; e < E; ++e)
+        if (mask >> e & 1u) sum += st[e];
+      if (sum > best_sum) best_sum = sum, best_mask = mask;
+    }
+    std::vector<int> chosen;
+    for (int e = 0; e < E; ++e)
+      if (best_mask >> e & 1u) chosen.push_back(e);
+    std::stable_sort(chosen.begin(), chosen.end(), [&](int a, int b) { return st[a] > st[b]; });
+    for (int j = 0; j < k; ++j) idx[t * k + j] = chosen[j];
+  }
+  return 0;
+}
+
+// Dispatch metadata: counts[E], offsets[E+1] (exclusive prefix sum), and the expert-contiguous
+// order (experts ascending, tokens ascending within an expert): row r holds the assignment
+// (perm_token[r], perm_slot[r]) and inv_perm[t*k + j] = r.  Returns -1 on an expert id
+// outside [0, E).
+int oracle_permute(const int32_t* idx, int64_t T, int E, int k, int32_t* counts, int32_t* offsets,
+                   int32_t* perm_token, int32_t* perm_slot, int32_t* inv_perm) {
+  for (int64_t i = 0; i < T * k; ++i)
+    if (idx[i] < 0 || idx[i] >= E) return -1;
+  for (int e = 0; e < E; ++e) counts[e] = 0;
+  for (int64_t i = 0; i < T * k; ++i) counts[idx[i]]++;
+  offsets[0] = 0;
+  for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+  int64_t r = 0;
+  for (int e = 0; e < E; ++e)
+    for (int64_t t = 0; t < T; ++t)
+      for (int j = 0; j < k; ++j)
+        if (idx[t * k + j] == e) {
+          perm_token[r] = (int32_t)t;
+          perm_slot[r] = j;
+          inv_perm[t * k + j] = (int32_t)r;
+          ++r;
+        }
+  return 0;
+}
+
+// One expert FFN on one token row (exposed for per-assignment checks).
+void oracle_expert_ffn(const uint16_t* x_row, const uint16_t* gate_up, const uint16_t* down, int64_t D,
+                       int64_t F, double* out) {
+  expert_ffn(x_row, gate_up, down, D, F, out);
+}
+
+// Layer forward: y[t] = sum_j p[t,j] * Expert_{idx[t,j]}(x_t) + SharedExpert(x_t).
+// gate_up_ptrs[e] -> [2F, D] and down_ptrs[e] -> [D, F] for each expert e (an entry may be NULL
+// when no token routes to e).  shared_gate_up [2Fs, D], shared_down [D, Fs] may be NULL (Fs = 0).
+// idx_out / p_out (optional) receive the routing.  Returns 0, -1 bad sizes, -2 missing expert.
+int oracle_layer(const uint16_t* x, const uint16_t* wg, const float* bias,
+                 const uint16_t* const* gate_up_ptrs, const uint16_t* const* down_ptrs,
+                 const uint16_t* shared_gate_up, const uint16_t* shared_down, int64_t T, int64_t D,
+                 int E, int k, int64_t F, int64_t Fs, double* y, int32_t* idx_out, double* p_out,
+                 int nthreads) {
+  if (T < 0 || D < 1 || E < 1 || k < 1 || k > E || F < 1 || Fs < 0) return -1;
+  std::vector<int> missing(T, 0);
+  for_tokens(T, nthreads, [&](int64_t t) {
+    std::vector<double> l(E), p(k), o(D), yt(D, 0.0);
+    std::vector<int32_t> idx(k);
+    router_logits(x + t * D, wg, D, E, l.data());
+    select_and_weight(l.data(), bias, E, k, idx.data(), p.data());
+    for (int j = 0; j < k; ++j) {
+      int e = idx[j];
+      if (!gate_up_ptrs[e] || !down_ptrs[e]) { missing[t] = 1; return; }
+      expert_ffn(x + t * D, gate_up_ptrs[e], down_ptrs[e], D, F, o.data());
+      for (int64_t d = 0; d < D; ++d) yt[d] += p[j] * o[d];
+    }
+    if (Fs > 0 && shared_gate_up && shared_down) {
+      expert_ffn(x + t * D, shared_gate_up, shared_down, D, Fs, o.data());
+      for (int64_t d = 0; d < D; ++d) yt[d] += o[d];
+    }
+    std::copy(yt.begin(), yt.end(), y + t * D);
+    if (idx_out) std::copy(idx.begin(), idx.end(), idx_out + t * k);
+    if (p_out) std::copy(p.begin(), p.end(), p_out + t * k);
+  });
+  for (int64_t t = 0; t < T; ++t)
+    if (missing[t]) return -2;
+  return 0;
+}
+
+// The eager form of the same layer: route every token, then for each top-k slot j and each
+// expert e, run expert e on exactly the tokens whose j-th choice is e and accumulate
+// p[t, j] * Expert_e(x_t) into their output rows; finally add the shared expert.  The top-k here
+// sorts all E experts by score (ties to the lower id) instead of the selection loop.
+int oracle_layer_eager(const uint16_t* x, const uint16_t* wg, const float* bias,
+                       const uint16_t* gate_up, const uint16_t* down, const uint16_t* shared_gate_up,
+                       const uint16_t* shared_down, int64_t T, int64_t D, int E, int k, int64_t F,
+                       int64_t Fs, double* y) {
+  if (T < 0 || D < 1 || E < 1 || k < 1 || k > E) return -1;
+  std::vector<double> l(T * E), p(T * k);
+  std::vector<int32_t> idx(T * k);
+  for (int64_t t = 0; t < T; ++t) {
+    router_logits(x + t * D, wg, D, E, &l[t * E]);
+    std::vector<int> order(E);
+    for (int e = 0; e < E; ++e) order[e] = e;
+    auto score = [&](int e) { return l[t * E + e] + (bias ? (double)bias[e] : 0.0); };
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return score(a) > score(b); });
+    double z = 0.0, m = -INFINITY;
+    for (int j = 0; j < k; ++j) m = std::max(m, l[t * E + order[j]]);
+    for (int j = 0; j < k; ++j) z += std::exp(l[t * E + order[j]] - m);
+    for (int j = 0; j < k; ++j) {
+      idx[t * k + j] = order[j];
+      p[t * k + j] = std::exp(l[t * E + order[j]] - m) / z;
+    }
+  }
+  std::fill(y, y + T * D, 0.0);
+  std::vector<double> o(D);
+  for (int j = 0; j < k; ++j)
+    for (int e = 0; e < E; ++e)
+      for (int64_t t = 0; t < T; ++t) {
+        if (idx[t * k + j] != e) continue;
+        expert_ffn(x + t * D, gate_up + (int64_t)e * 2 * F * D, down + (int64_t)e * D * F, D, F, o.data());
+        for (int64_t d = 0; d < D; ++d) y[t * D + d] += p[t * k + j] * o[d];
+      }
+  if (Fs > 0 && shared_gate_up && shared_down)
+    for (int64_t t = 0; t < T; ++t) {
+      expert_ffn(x + t * D, shared_gate_up, shared_down, D, Fs, o.data());
+      for (int64_t d = 0; d < D; ++d) y[t * D + d] += o[d];
+    }
+  return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,268 @@
+"""Pins of the fp64 oracle to things other than itself (CPU only).
+
+Each test ties one part of the oracle to a fact fixed by the pages' definition or by
+mathematics -- an exhaustive search, a closed form, an invariance, a textbook reduction --
+chosen so that a plausible slip in the oracle (dropped term, wrong sign, wrong index,
+transposed operand, SiLU on the wrong half, bias in the weights) fails at least one of them.
+
+Definition (gotburnout.io glossary "MoE", section 2; josueisai.com "Mixture of experts",
+section "El router"): p = Softmax(TopK(W_g x)) normalised over the chosen k only,
+y = sum_i p_i Expert_i(x) + shared experts, Expert(x) = (silu(x G^T) * (x U^T)) Down^T.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import moe_inputs as mi
+import oracle
+
+f64 = mi.bf16_to_f64
+
+
+def _bf16(a):
+    """float64 array -> bf16 bit patterns (round to nearest even)."""
+    u = np.asarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def _rand_layer(rng, T, D, E, F, Fs=0, wscale=0.05):
+    x = _bf16(rng.standard_normal((T, D)))
+    wg = _bf16(rng.standard_normal((E, D)) * 0.3)
+    gu = _bf16(rng.standard_normal((E, 2 * F, D)) * wscale)
+    dn = _bf16(rng.standard_normal((E, D, F)) * wscale)
+    sgu = _bf16(rng.standard_normal((2 * Fs, D)) * wscale) if Fs else None
+    sdn = _bf16(rng.standard_normal((D, Fs)) * wscale) if Fs else None
+    return x, wg, gu, dn, sgu, sdn
+
+
+def _dense_swiglu(x, gu, dn):
+    """Textbook dense SwiGLU FFN with numpy matmuls: (silu(x G^T) * (x U^T)) Down^T."""
+    X, GU, DN = f64(x), f64(gu), f64(dn)
+    F = DN.shape[1]
+    g = X @ GU[:F].T
+    u = X @ GU[F:].T
+    a = g / (1.0 + np.exp(-g)) * u
+    return a @ DN.T
+
+
+# ----------------------------------------------------------------------------- router
+@pytest.mark.parametrize("E,k", [(8, 1), (8, 2), (8, 3), (8, 8), (5, 3), (12, 4)])
+def test_topk_equals_exhaustive_subset_search(E, k):
+    rng = np.random.default_rng(E * 31 + k)
+    x, wg, *_ = _rand_layer(rng, 64, 32, E, 8)
+    bias = (rng.standard_normal(E) * 0.5).astype(np.float32)
+    idx, p, lg = oracle.router(x, wg, bias, k, return_logits=True)
+    s = lg + bias.astype(np.float64)
+    assert (idx == oracle.topk_exhaustive(s, k)).all()
+
+
+def test_logits_equal_library_matmul():
+    rng = np.random.default_rng(1)
+    x, wg, *_ = _rand_layer(rng, 40, 96, 7, 8)
+    _, _, lg = oracle.router(x, wg, None, 2, return_logits=True)
+    ref = f64(x) @ f64(wg).T
+    np.testing.assert_allclose(lg, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_weights_sum_to_one_and_are_descending():
+    rng = np.random.default_rng(2)
+    x, wg, *_ = _rand_layer(rng, 200, 64, 16, 8)
+    idx, p = oracle.router(x, wg, None, 4)
+    assert np.abs(p.sum(1) - 1.0).max() <= 1e-12
+    assert (np.diff(p, axis=1) <= 0).all()  # without bias, score order = weight order
+    assert (p > 0).all()
+
+
+def test_k1_weight_is_one():
+    rng = np.random.default_rng(3)
+    x, wg, *_ = _rand_layer(rng, 50, 32, 6, 8)
+    _, p = oracle.router(x, wg, None, 1)
+    assert (p == 1.0).all()
+
+
+def test_k2_weights_are_logistic_of_logit_gap():
+    """softmax over two chosen logits = logistic sigmoid of their difference (closed form)."""
+    rng = np.random.default_rng(4)
+    x, wg, *_ = _rand_layer(rng, 64, 48, 8, 8)
+    idx, p, lg = oracle.router(x, wg, None, 2, return_logits=True)
+    l0 = lg[np.arange(64), idx[:, 0]]
+    l1 = lg[np.arange(64), idx[:, 1]]
+    ref = np.array([1.0 / (1.0 + math.exp(b - a)) for a, b in zip(l0, l1)])
+    np.testing.assert_allclose(p[:, 0], ref, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(p[:, 1], 1.0 - ref, rtol=0, atol=1e-14)
+
+
+def test_shifting_every_logit_or_every_bias_changes_nothing():
+    rng = np.random.default_rng(5)
+    x, wg, *_ = _rand_layer(rng, 80, 32, 8, 8)
+    bias = (rng.standard_normal(8) * 0.5).astype(np.float32)
+    idx, p = oracle.router(x, wg, bias, 3)
+    # append an all-ones feature whose router weight is 2.0 for every expert: logits + 2
+    x2 = np.concatenate([x, np.full((80, 1), _bf16([1.0])[0], np.uint16)], axis=1)
+    wg2 = np.concatenate([wg, np.full((8, 1), _bf16([2.0])[0], np.uint16)], axis=1)
+    idx2, p2 = oracle.router(x2, wg2, bias, 3)
+    assert (idx2 == idx).all()
+    np.testing.assert_allclose(p2, p, rtol=0, atol=1e-13)
+    idx3, p3 = oracle.router(x, wg, bias + np.float32(0.75), 3)
+    assert (idx3 == idx).all()
+    assert (p3 == p).all()
+
+
+def test_bias_steers_selection_but_not_weights():
+    rng = np.random.default_rng(6)
+    x, wg, *_ = _rand_layer(rng, 30, 32, 8, 8)
+    bias = np.zeros(8, np.float32)
+    bias[5] = 1000.0
+    idx, p, lg = oracle.router(x, wg, bias, 2, return_logits=True)
+    assert (idx[:, 0] == 5).all()
+    for t in range(30):
+        l = lg[t, idx[t]]
+        ref = np.exp(l - l.max()) / np.exp(l - l.max()).sum()
+        np.testing.assert_allclose(p[t], ref, rtol=0, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- dispatch
+def test_permute_is_stable_sort_by_expert():
+    rng = np.random.default_rng(7)
+    T, E, k = 300, 13, 3
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    counts, offsets, pt, ps, inv = oracle.permute(idx, E)
+    flat = idx.reshape(-1)
+    assert (counts == np.bincount(flat, minlength=E)).all()
+    assert offsets[0] == 0 and (offsets[1:] == np.cumsum(counts)).all()
+    order = np.argsort(flat, kind="stable")  # library stable sort of the (t, j) slots
+    assert (pt == order // k).all() and (ps == order % k).all()
+    assert (inv[order] == np.arange(T * k)).all()  # inv_perm o perm = identity
+    assert sorted(inv.tolist()) == list(range(T * k))  # bijection
+    for e in range(E):
+        seg = pt[offsets[e]:offsets[e + 1]]
+        assert (np.diff(seg) > 0).all()
+        assert (flat[order[offsets[e]:offsets[e + 1]]] == e).all()
+
+
+def test_permute_counts_equal_router_histogram():
+    rng = np.random.default_rng(8)
+    x, wg, *_ = _rand_layer(rng, 257, 64, 9, 8)
+    idx, _ = oracle.router(x, wg, None, 2)
+    counts, offsets, *_ = oracle.permute(idx, 9)
+    for e in range(9):
+        assert counts[e] == int((idx == e).sum())
+    assert offsets[-1] == 257 * 2
+
+
+def test_permute_rejects_out_of_range_ids():
+    with pytest.raises(ValueError):
+        oracle.permute(np.array([[0, 5]], np.int32), 4)
+
+
+# ----------------------------------------------------------------------------- experts
+def test_single_expert_reduces_to_dense_swiglu():
+    rng = np.random.default_rng(9)
+    x, wg, gu, dn, _, _ = _rand_layer(rng, 33, 64, 1, 48)
+    y, idx, p = oracle.layer(x, wg, None, gu, dn, 1)
+    assert (idx == 0).all() and (p == 1).all()
+    np.testing.assert_allclose(y, _dense_swiglu(x, gu[0], dn[0]), rtol=1e-12, atol=1e-14)
+
+
+def test_scalar_closed_form():
+    """D = F = 1: y = c * silu(a x) * (b x), with a the gate (first-half) weight."""
+    for (xv, a, b, c) in [(1.5, 0.75, -2.0, 0.5), (-3.0, 1.25, 0.5, -1.0), (0.25, -4.0, 3.0, 2.0)]:
+        x = _bf16([[xv]])
+        wg = _bf16([[1.0]])
+        gu = _bf16([[[a], [b]]])
+        dn = _bf16([[[c]]])
+        y, _, _ = oracle.layer(x, wg, None, gu, dn, 1)
+        g = a * xv
+        ref = c * (g / (1.0 + math.exp(-g))) * (b * xv)
+        assert abs(y[0, 0] - ref) <= 1e-15 * max(1.0, abs(ref))
+
+
+def test_identical_experts_with_k_equal_E_give_dense_ffn():
+    rng = np.random.default_rng(10)
+    T, D, E, F = 20, 32, 4, 24
+    x, wg, gu, dn, _, _ = _rand_layer(rng, T, D, E, F)
+    gu[:] = gu[0]
+    dn[:] = dn[0]
+    y, _, _ = oracle.layer(x, wg, None, gu, dn, E)
+    np.testing.assert_allclose(y, _dense_swiglu(x, gu[0], dn[0]), rtol=1e-12, atol=1e-14)
+
+
+def test_scaling_down_proj_scales_output():
+    rng = np.random.default_rng(11)
+    x, wg, gu, dn, _, _ = _rand_layer(rng, 25, 32, 6, 16)
+    y1, _, _ = oracle.layer(x, wg, None, gu, dn, 2)
+    y2, _, _ = oracle.layer(x, wg, None, gu, _bf16(f64(dn) * 2.0), 2)
+    np.testing.assert_array_equal(y2, 2.0 * y1)
+
+
+def test_relabelling_experts_leaves_output_unchanged():
+    rng = np.random.default_rng(12)
+    E = 7
+    x, wg, gu, dn, _, _ = _rand_layer(rng, 40, 32, E, 16)
+    bias = (rng.standard_normal(E) * 0.3).astype(np.float32)
+    y1, idx1, _ = oracle.layer(x, wg, bias, gu, dn, 3)
+    perm = rng.permutation(E)
+    y2, idx2, _ = oracle.layer(x, wg[perm], bias[perm], gu[perm], dn[perm], 3)
+    assert (perm[idx2] == idx1).all()
+    np.testing.assert_array_equal(y2, y1)
+
+
+def test_permuting_tokens_permutes_output():
+    rng = np.random.default_rng(13)
+    x, wg, gu, dn, sgu, sdn = _rand_layer(rng, 37, 32, 5, 16, Fs=8)
+    y1, _, _ = oracle.layer(x, wg, None, gu, dn, 2, sgu, sdn)
+    perm = rng.permutation(37)
+    y2, _, _ = oracle.layer(x[perm], wg, None, gu, dn, 2, sgu, sdn)
+    np.testing.assert_array_equal(y2, y1[perm])
+
+
+def test_shared_expert_adds_a_dense_ffn():
+    rng = np.random.default_rng(14)
+    x, wg, gu, dn, sgu, sdn = _rand_layer(rng, 30, 64, 6, 32, Fs=40)
+    y0, _, _ = oracle.layer(x, wg, None, gu, dn, 2)
+    y1, _, _ = oracle.layer(x, wg, None, gu, dn, 2, sgu, sdn)
+    np.testing.assert_allclose(y1 - y0, _dense_swiglu(x, sgu, sdn), rtol=1e-10, atol=1e-13)
+
+
+def test_routed_output_equals_weighted_sum_of_dense_experts():
+    """y_t = sum_j p_tj * DenseFFN_{idx_tj}(x_t), each expert evaluated with numpy matmuls."""
+    rng = np.random.default_rng(15)
+    T, E, k = 50, 6, 3
+    x, wg, gu, dn, _, _ = _rand_layer(rng, T, 48, E, 32)
+    y, idx, p = oracle.layer(x, wg, None, gu, dn, k)
+    dense = np.stack([_dense_swiglu(x, gu[e], dn[e]) for e in range(E)])  # [E, T, D]
+    ref = np.zeros_like(y)
+    for t in range(T):
+        for j in range(k):
+            ref[t] += p[t, j] * dense[idx[t, j], t]
+    np.testing.assert_allclose(y, ref, rtol=1e-11, atol=1e-14)
+
+
+def test_eager_loop_equals_layer():
+    rng = np.random.default_rng(16)
+    x, wg, gu, dn, sgu, sdn = _rand_layer(rng, 45, 32, 8, 16, Fs=16)
+    bias = (rng.standard_normal(8) * 0.4).astype(np.float32)
+    y, _, _ = oracle.layer(x, wg, bias, gu, dn, 2, sgu, sdn)
+    ye = oracle.layer_eager(x, wg, bias, gu, dn, 2, sgu, sdn)
+    np.testing.assert_allclose(ye, y, rtol=1e-13, atol=1e-15)
+
+
+def test_expert_ffn_matches_layer_for_single_assignment():
+    rng = np.random.default_rng(17)
+    x, wg, gu, dn, _, _ = _rand_layer(rng, 3, 64, 4, 32)
+    y, idx, p = oracle.layer(x, wg, None, gu, dn, 1)
+    for t in range(3):
+        np.testing.assert_array_equal(oracle.expert_ffn(x[t], gu[idx[t, 0]], dn[idx[t, 0]]), y[t])
+
+
+def test_sparse_expert_dict_matches_packed():
+    w = mi.WORKLOADS["tiny"]
+    inp = mi.host_inputs(w)
+    x = inp["x"][:16]
+    y1, idx, _ = oracle.layer(x, inp["wg"], None, inp["gate_up"], inp["down"], w.k)
+    used = sorted(set(idx.reshape(-1).tolist()))
+    y2, _, _ = oracle.layer(x, inp["wg"], None, {e: inp["gate_up"][e] for e in used},
+                            {e: inp["down"][e] for e in used}, w.k)
+    np.testing.assert_array_equal(y1, y2)
