@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse-MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one whole layer forward (router, dispatch, gate_up GEMM + SwiGLU, down GEMM with the
+router weight, combine) over one batch of synthetic tokens, inputs resident in HBM.  The timed
+steps replay a CUDA graph of the C-ABI call ``moe_layer_forward_timed`` (events around every
+stage, recorded on the launching stream).  ``e2e`` repeats the measurement through
+``moe_layer_forward_host`` with pinned host buffers (x in, y out, copies inside the timed region).
+With N > 1 (torchrun) every rank runs an independent replica (weak scaling); the only
+collectives are the barrier and the max-over-ranks of the elapsed time.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE layer tokens/s at 1 B200; prefill TFLOP/s and decode active-weight GB/s vs peak"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------------- accounting
+def gateup_flops(w: mi.Workload) -> float:
+    """Algorithmic FLOPs of the gate_up launch: 2*D*2F per routed row, 2*D*2Fs per token."""
+    return float(w.T) * (w.k * 4.0 * w.D * w.F + 4.0 * w.D * w.Fs)
+
+
+def down_flops(w: mi.Workload) -> float:
+    return float(w.T) * (w.k * 2.0 * w.D * w.F + 2.0 * w.D * w.Fs)
+
+
+def active_weight_bytes(w: mi.Workload, n_active: int, part: str = "all") -> float:
+    """Bytes of weights that must be streamed: distinct active experts (+ shared expert)."""
+    gu = 2.0 * w.F * w.D * 2 * n_active + 2.0 * w.Fs * w.D * 2
+    dn = 1.0 * w.D * w.F * 2 * n_active + 1.0 * w.D * w.Fs * 2
+    return {"gate_up": gu, "down": dn, "all": gu + dn}[part]
+
+
+def decode_tokens_per_s_bound(bandwidth_bytes_per_s: float, active_params: float, bytes_per_param: float) -> float:
+    """The pages' decode model: tokens/s = memory bandwidth / bytes of active parameters per token
+    (keryc.com, "Por que MoEs importan": gpt-oss-20b, ~3.6e9 active params, bf16, ~800 GB/s)."""
+    return bandwidth_bytes_per_s / (active_params * bytes_per_param)
+
+
+# ---------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", self.gpu_id, "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), sm_max=float(f[2]), power=float(f[3]), hw=f[5], hwt=f[6], swt=f[7],
+                                 pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        loaded = [r for r in rows if r["power"] > 300] or rows
+        reasons = set()
+        for r in loaded:
+            if r["hw"] == "Active":
+                reasons.add("hw_slowdown")
+            if r["hwt"] == "Active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active":
+                reasons.add("sw_thermal_slowdown")
+            if r["pcap"] == "Active":
+                reasons.add("sw_power_cap")
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["sm_max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------------------------- CPU oracle
+def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, max_experts: int = 40):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload's tokens (all host
+    cores).  Returns (tokens/s, cores, description)."""
+    import oracle
+
+    cores = host_cores()
+    x_all_rows = np.arange(w.T)
+    wg = mi.host_wg(w)
+    bias = mi.bias_f32(w)
+    # route a prefix of tokens to know which experts the sample needs (outside the timed region)
+    probe = x_all_rows[: min(w.T, 256)]
+    xp = mi.host_x(w, rows=probe)
+    idx, _ = oracle.router(xp, wg, bias, w.k)
+    chosen, experts = [], set()
+    for i, t in enumerate(probe):
+        e = set(idx[i].tolist())
+        if len(experts | e) > max_experts and chosen:
+            continue
+        experts |= e
+        chosen.append(i)
+    experts = sorted(experts)
+    gu = dict(zip(experts, mi.host_gate_up(w, experts)))
+    dn = dict(zip(experts, mi.host_down(w, experts)))
+    sgu, sdn = mi.host_shared(w)
+    chosen = np.array(chosen)
+    # time a growing number of tokens until the budget is reached
+    n, done, elapsed = min(len(chosen), cores), 0, 0.0
+    while True:
+        rows = chosen[np.arange(done, done + n) % len(chosen)]
+        x = xp[rows]
+        t0 = time.perf_counter()
+        oracle.layer(x, wg, bias, gu, dn, w.k, sgu, sdn, nthreads=cores)
+        dt = time.perf_counter() - t0
+        done += n
+        elapsed += dt
+        if elapsed >= budget_s or done >= 64 * cores:
+            break
+        n = max(1, int(n * min(4.0, max(1.5, (budget_s - elapsed) / max(dt, 1e-3)))))
+    desc = (f"{done} tokens of workload {w.name} (full layer: routing over all E experts, top-{w.k} SwiGLU experts"
+            f"{', shared expert' if w.Fs else ''}) through the fp64 oracle on {cores} threads; tokens/s = "
+            f"{done} / {elapsed:.2f} s")
+    return done / elapsed, cores, desc
+
+
+# ---------------------------------------------------------------------------------- GPU arm
+def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
+    import ctypes
+
+    import torch
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_16_b200 as moe
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    pk, pk_kind = peaks()
+    with torch.cuda.stream(stream):
+        inp = mi.device_inputs(w, device=dev)
+        layer = moe.MoELayer(inp["wg"], inp["gate_up"], inp["down"], w.k, bias=inp["bias"],
+                             shared_gate_up=inp["shared_gate_up"], shared_down=inp["shared_down"])
+        x = inp["x"]
+        y = torch.empty_like(x)
+        ws = layer.workspace(w.T)
+        n_kernels = layer.kernel_count(w.T)
+        weight_bytes = sum(t.numel() * t.element_size() for t in (inp["gate_up"], inp["down"], inp["wg"]))
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if weight_bytes < 8 * L2_BYTES else None
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        for e in evs:
+            e.record(stream)
+        for _ in range(max(args.warmup, 3)):
+            layer.forward(x, y, stream=stream)
+        stream.synchronize()
+        if layer.device_error(stream) != 0:
+            raise RuntimeError("device error during warm-up")
+        # the timed step: a CUDA graph of moe_layer_forward_timed (stage events inside the graph)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            layer.forward_timed(x, y, evs, stream=stream)
+        for _ in range(3):
+            graph.replay()
+        stream.synchronize()
+        # active experts (for the decode byte count)
+        idx, _ = moe.moe_router_topk(x, inp["wg"], inp["bias"], w.k, stream=stream)
+        n_active = int(torch.unique(idx).numel())
+        stream.synchronize()
+
+    gpu_id = str(local_rank)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+
+    step_ms, stage_ms = [], [[] for _ in range(5)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clk, torch.cuda.stream(stream):
+        t_begin = time.perf_counter()
+        for s in range(args.steps):
+            if flush is not None:
+                flush.fill_(s)  # evict the weights from L2 (outside the stage events)
+            graph.replay()
+            stream.synchronize()
+            step_ms.append(evs[0].elapsed_time(evs[5]))
+            for j in range(5):
+                stage_ms[j].append(evs[j].elapsed_time(evs[j + 1]))
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - t_begin
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    ms_per_step = total_ms / len(step_ms)
+    value = world * w.T * len(step_ms) / (total_ms / 1e3)
+
+    # ---- end to end through the public API with pinned host buffers
+    x_h = x.cpu().pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            layer.forward_host(x_h, y_h, stream=stream)
+        stream.synchronize()
+        e2e_steps = max(5, min(args.steps, 50))
+        e2e_ms = 0.0
+        for _ in range(e2e_steps):
+            if flush is not None:
+                flush.fill_(1)
+            e0.record(stream)
+            layer.forward_host(x_h, y_h, stream=stream)
+            e1.record(stream)
+            stream.synchronize()
+            e2e_ms += e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * w.T * e2e_steps / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant kernel (gate_up grouped GEMM: ~2/3 of the FLOPs / weight bytes)
+    gate_ms = statistics.mean(stage_ms[2])
+    down_ms = statistics.mean(stage_ms[3])
+    decode = w.T <= 64
+    if decode:
+        bytes_gu = active_weight_bytes(w, n_active, "gate_up") + w.T * w.k * w.D * 2.0 + w.T * (w.k * w.F + w.Fs) * 2.0
+        achieved = bytes_gu / (gate_ms / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"kernel": "grouped_gemm_kernel<gate_up, stream>", "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)"}
+    else:
+        achieved = gateup_flops(w) / (gate_ms / 1e3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        roof = {"kernel": "grouped_gemm_kernel<gate_up, tiled>", "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
+                "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4)}
+    layer_tflops = w.flops / (ms_per_step / 1e3) / 1e12 * world
+    layer_gbs = active_weight_bytes(w, n_active) / (ms_per_step / 1e3) / 1e9
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": len(step_ms),
+        "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init weights)",
+        "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": ("L2 flushed (256 MB write) before every timed step" if flush is not None
+                          else f"inputs larger than L2 (weights {weight_bytes / 1e9:.2f} GB), no flush"),
+                   "timing": "CUDA-graph replay of moe_layer_forward_timed; events on the launching stream"},
+        "roofline": roof,
+        "layer": {"tflops": round(layer_tflops, 1), "active_experts": n_active,
+                  "active_weight_gbs": round(layer_gbs, 1),
+                  "frac_tensor_sustained": round(layer_tflops / world / pk["bf16_tflops_sustained"], 4),
+                  "frac_hbm": round(layer_gbs / pk["hbm_gbs"], 4)},
+        "stages_ms": {n: round(statistics.mean(v), 4) for n, v in
+                      zip(("router", "dispatch", "gate_up_gemm", "down_gemm", "combine"), stage_ms)},
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": w.T * w.D * 2,
+                "d2h_bytes_per_step": w.T * w.D * 2, "api": "moe_layer_forward_host (pinned host x, y)"},
+        "gpu_launches": n_kernels * len(step_ms),
+        "clocks": clk.summary(),
+        "wall_s_timed_region": round(wall, 3),
+    }
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            v, cores, desc = cpu_oracle_rate(w)
+            result["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                      "sample": desc}
+        print(json.dumps(result), flush=True)
+    del graph
+
+
+def run_reference(args, w: mi.Workload, rank: int, world: int):
+    if rank != 0:
+        return
+    steps = []
+    cores = host_cores()
+    desc = None
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for s in range(args.warmup + args.steps):
+        v, cores, desc = cpu_oracle_rate(w, budget_s=budget)
+        if s >= args.warmup:
+            steps.append(v)
+    value = statistics.mean(steps)
+    ms = w.T / value * 1e3
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; random-init weights)",
+        "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="mixtral", choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = mi.WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=__import__("torch").device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,187 @@
+/*
+ * moe_b200.h -- C ABI of the sparse Mixture-of-Experts FFN layer forward on one B200 (sm_100a).
+ *
+ * The layer (gotburnout.io glossary "MoE (Mixture of Experts)", section 2, layer diagram and
+ * section 3, token pipeline; josueisai.com "Mixture of experts", section "El router"):
+ *
+ *     logits = W_g x                       router projection, fp32 accumulation
+ *     S      = the k experts with the largest (logits + bias)   (bias: optional, selection only)
+ *     p_j    = softmax over the chosen k of the unbiased logits
+ *     y      = sum_j p_j * Expert_{S_j}(x) + SharedExpert(x)
+ *     Expert_e(x) = down[e] (silu(G_e x) * (U_e x)),   G_e = gate_up[e][0:F], U_e = gate_up[e][F:2F]
+ *
+ * The residual add of the diagram is the caller's: y excludes it.
+ *
+ * Packed weights (dev.smart-guide.co.kr deep-dive, section "La Solucion: WeightConverter": the
+ * per-expert w1 / w3 matrices merged on a new expert dim 0 and concatenated on dim 1):
+ *     gate_up [E, 2F, D]  row-major, rows [0,F) = w1 ("gate", through SiLU), [F,2F) = w3 ("up")
+ *     down    [E, D, F]   row-major
+ *
+ * Conventions for every entry point:
+ *   - bf16 tensors are passed as moe_bf16_t (the raw bf16 bit pattern), row-major, contiguous.
+ *   - All tensor pointers are DEVICE pointers owned by the caller, except the two host
+ *     buffers of moe_layer_forward_host.  The library never allocates, frees or keeps them.
+ *   - Tensor pointers must be 16-byte aligned; workspaces 256-byte aligned.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  No entry point synchronises except moe_get_device_error.
+ *   - Arguments are validated on the host before anything is launched; on an error status
+ *     nothing has been enqueued.  A failed launch returns MOE_ERR_CUDA.
+ *   - Errors found by kernels (an expert id outside [0,E) reaching moe_permute, a device-side
+ *     wait that gave up) are OR-ed into a sticky error word in the first 256 bytes of the
+ *     workspace; read it with moe_get_device_error.
+ *   - Shapes: D, F, Fs multiples of 64; 1 <= E <= 1024; 1 <= k <= min(E, 32); T >= 0 (T = 0 is a
+ *     no-op); T*k < 2^31.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t; /* bf16 bit pattern */
+typedef void* moe_stream_t;  /* cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,         /* null pointer, k > E, negative size, ...          */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,   /* D/F/Fs not a multiple of 64, E > 1024, k > 32     */
+  MOE_ERR_ALIGNMENT = 3,           /* a pointer is not 16-byte (workspace: 256-byte) aligned */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below the matching *_workspace_size()     */
+  MOE_ERR_CUDA = 5,                /* a CUDA runtime call or kernel launch failed         */
+  MOE_ERR_DEVICE_INDEX = 6,        /* (device) an expert id outside [0, E) was seen       */
+  MOE_ERR_TIMEOUT = 7,             /* (device) a bounded wait inside a kernel gave up     */
+  MOE_ERR_NO_DEVICE = 8            /* no current CUDA device of compute capability 10.x   */
+} moe_status_t;
+
+/* ----------------------------------------------------------------------------------------
+ * Step 1: router projection + top-k + renormalised softmax (one fused kernel).
+ * josueisai.com "Mixture of experts", section "El router"; gotburnout.io glossary, section 2
+ * (p = Softmax(TopK(W_g x))) and section 2 item 4 (aux-loss-free balancing bias).
+ *
+ *   x        [T, D]  bf16      w_gate [E, D] bf16      bias [E] fp32 or NULL
+ *   topk_idx [T, k]  int32     out: expert ids, by (logit + bias) descending, ties -> lower id
+ *   topk_w   [T, k]  fp32      out: exp(l_j - m) / sum_i exp(l_i - m) over the chosen k, with
+ *                              the UNBIASED fp32 logits l (the bias only steers the selection)
+ * ---------------------------------------------------------------------------------------- */
+moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, const float* bias, int T,
+                             int D, int E, int k, int32_t* topk_idx, float* topk_w,
+                             moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Step 2: dispatch -- histogram, exclusive prefix sum and permutation into expert-contiguous
+ * order (keryc.com "Mixture of Experts optimiza Transformers y LLMs", section "Ejecucion
+ * eficiente: backends de expertos": the grouped backend sorts tokens by expert id).
+ * Order: experts ascending, tokens ascending within an expert (a stable counting sort of the
+ * T*k slots by expert id).  M = T*k rows.
+ *
+ *   topk_idx [T, k] int32, topk_w [T, k] fp32, x [T, D] bf16 (NULL: metadata only)
+ *   counts   [E]    int32  out: slots routed to each expert
+ *   offsets  [E+1]  int32  out: offsets[0] = 0, offsets[e+1] = offsets[e] + counts[e]
+ *   perm_token [M]  int32  out: token of row r
+ *   inv_perm [T*k]  int32  out: row of slot t*k + j
+ *   p_perm   [M]    fp32   out: topk_w of row r
+ *   x_perm   [M, D] bf16   out (if x != NULL): x_perm[r] = x[perm_token[r]]
+ *   ws: >= moe_permute_workspace_size(T, E, k) bytes of device memory (contents need not be
+ *       initialised); its first 256 bytes are the device error word.
+ * An id outside [0, E) sets MOE_ERR_DEVICE_INDEX in the error word; that slot is dropped.
+ * ---------------------------------------------------------------------------------------- */
+size_t moe_permute_workspace_size(int T, int E, int k);
+moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_bf16_t* x, int T,
+                         int D, int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm_token,
+                         int32_t* inv_perm, float* p_perm, moe_bf16_t* x_perm, void* ws,
+                         size_t ws_bytes, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Step 3: the routed experts as grouped GEMMs over expert-contiguous rows (tcgen05 / TMEM /
+ * TMA).  gotburnout.io glossary, section 3 step 3 (the SwiGLU expert) and step 4 (outputs
+ * multiplied by the router weights).
+ *
+ *   x_perm   [M, D] bf16       rows of segment e are [offsets[e], offsets[e+1])
+ *   offsets  [E+1]  int32      device; offsets[E] <= M
+ *   row_scale [M]   fp32 or NULL (1.0): multiplies output row r (pass p_perm)
+ *   max_seg:  an upper bound on any segment length (pass M if unknown).  max_seg <= 64
+ *             selects the weight-streaming (decode) kernels, otherwise the tiled kernels.
+ *   gate_up  [E, 2F, D] bf16, down [E, D, F] bf16
+ *   out_perm [M, D] bf16 out:   out_perm[r] = row_scale[r] * Expert_e(x_perm[r]) (bf16)
+ *   ws: >= moe_grouped_swiglu_ffn_workspace_size(M, F) bytes (holds h = silu(G x) * (U x),
+ *       [M, F] bf16); first 256 bytes: the device error word.
+ * ---------------------------------------------------------------------------------------- */
+size_t moe_grouped_swiglu_ffn_workspace_size(int M, int F);
+moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* offsets,
+                                    const float* row_scale, int M, int max_seg, int E, int D, int F,
+                                    const moe_bf16_t* gate_up, const moe_bf16_t* down,
+                                    moe_bf16_t* out_perm, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Step 4: weighted combine back to token order (gotburnout.io glossary, section 2 "Weighted
+ * Aggregation", section 3 step 4).  out_perm rows are already scaled by their router weight.
+ *
+ *   y[t] = sum_{j=0..k-1} out_perm[inv_perm[t*k + j]] + shared_out[t]     (fp32 sum, j order)
+ *   out_perm [T*k, D] bf16, inv_perm [T*k] int32, shared_out [T, D] bf16 or NULL, y [T, D] bf16
+ * ---------------------------------------------------------------------------------------- */
+moe_status_t moe_combine(const moe_bf16_t* out_perm, const int32_t* inv_perm,
+                         const moe_bf16_t* shared_out, int T, int D, int k, moe_bf16_t* y,
+                         moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * The whole layer (steps 1-4, plus the always-on shared expert of gotburnout.io glossary,
+ * section 2 item 3 "Shared Experts", added with weight 1).
+ * T <= 64 runs the weight-streaming (decode) kernels, larger T the tiled (prefill) kernels;
+ * `flags` can force either for testing.
+ * ---------------------------------------------------------------------------------------- */
+#define MOE_FLAG_FORCE_PREFILL 1
+#define MOE_FLAG_FORCE_DECODE 2 /* only valid for T <= 64 */
+
+typedef struct {
+  int32_t T, D, E, k, F, Fs;       /* Fs = 0: no shared expert                              */
+  const moe_bf16_t* w_gate;        /* [E, D]                                                */
+  const float* bias;               /* [E] selection bias or NULL                            */
+  const moe_bf16_t* gate_up;       /* [E, 2F, D]                                            */
+  const moe_bf16_t* down;          /* [E, D, F]                                             */
+  const moe_bf16_t* shared_gate_up;/* [2Fs, D] or NULL                                      */
+  const moe_bf16_t* shared_down;   /* [D, Fs] or NULL                                       */
+  int32_t flags;                   /* 0 or MOE_FLAG_*                                       */
+} moe_layer_desc_t;
+
+/* Device workspace bytes for moe_layer_forward / moe_layer_forward_host (0 if desc invalid). */
+size_t moe_layer_workspace_size(const moe_layer_desc_t* desc);
+
+/* x [T, D] bf16 (device) -> y [T, D] bf16 (device).  Clears the workspace's error word first. */
+moe_status_t moe_layer_forward(const moe_layer_desc_t* desc, const moe_bf16_t* x, moe_bf16_t* y,
+                               void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Same with HOST buffers (pinned memory for asynchronous copies): copies x_host into the
+ * workspace, runs the layer, copies y back to y_host, all on `stream`.  The caller
+ * synchronises the stream before reading y_host. */
+moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16_t* x_host,
+                                    moe_bf16_t* y_host, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream);
+
+/* moe_layer_forward that also records events[0..n_events) (cudaEvent_t handles created by the
+ * caller) on `stream` around its stages: events[0] before the router, then one event after
+ * each of: router, dispatch, gate_up GEMM (+SwiGLU), down GEMM, combine (6 events in all;
+ * n_events must be >= 6).  Used to time each stage on the launching stream. */
+moe_status_t moe_layer_forward_timed(const moe_layer_desc_t* desc, const moe_bf16_t* x,
+                                     moe_bf16_t* y, void* ws, size_t ws_bytes, moe_stream_t stream,
+                                     void* const* events, int n_events);
+
+/* Number of kernels one moe_layer_forward launches for this descriptor (0 if invalid). */
+int moe_layer_kernel_count(const moe_layer_desc_t* desc);
+
+/* Synchronises `stream`, returns the status held in the workspace's error word (MOE_OK,
+ * MOE_ERR_DEVICE_INDEX or MOE_ERR_TIMEOUT) and clears it. */
+moe_status_t moe_get_device_error(void* ws, moe_stream_t stream);
+
+/* Static, human-readable name of a status. */
+const char* moe_status_string(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

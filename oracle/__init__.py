@@ -177,3 +177,46 @@ def layer_eager(x, wg, bias, gate_up, down, k, shared_gate_up=None, shared_down=
     if rc != 0:
         raise ValueError(f"oracle_layer_eager rc={rc}")
     return y
+
+
+# ----------------------------------------------------------------------------- gap-enforced inputs
+# Router scores must be separated by at least GAP among each token's top k+1 experts (fp64
+# scores on the bf16 inputs), so fp32 accumulation on a GPU (error ~1e-4 at D = 7168) cannot
+# reorder them and top-k indices can be compared bit for bit.
+GAP = 1e-2
+
+
+def scores(x_rows, wg, bias, k):
+    """Selection scores l + bias in fp64 for the given token rows."""
+    _, _, lg = router(x_rows, wg, bias, k, return_logits=True)
+    return lg + (0.0 if bias is None else np.asarray(bias, np.float64))
+
+
+def gap_violations(s, k, delta=GAP):
+    """Rows whose top-(k+1) scores have a consecutive gap below delta."""
+    E = s.shape[1]
+    m = min(k + 1, E)
+    if m < 2:
+        return np.zeros(s.shape[0], bool)
+    top = -np.sort(-s, axis=1)[:, :m]
+    return (np.diff(-top, axis=1) < delta).any(axis=1)
+
+
+def gap_redraw(w, delta=GAP, max_rounds=50):
+    """Per-token substream index for workload ``w`` (a moe_inputs.Workload) such that every
+    token's router scores keep the minimum gap; a violating token row is redrawn from the next
+    substream of x, deterministically."""
+    import moe_inputs as mi
+
+    wg = mi.host_wg(w)
+    bias = mi.bias_f32(w)
+    redraw = np.zeros(w.T, np.uint32)
+    todo = np.arange(w.T)
+    for _ in range(max_rounds):
+        x = mi.host_x(w, rows=todo, redraw=redraw[todo])
+        bad = gap_violations(scores(x, wg, bias, w.k), w.k, delta)
+        if not bad.any():
+            return redraw
+        todo = todo[bad]
+        redraw[todo] += 1
+    raise RuntimeError("gap enforcement did not converge")

@@ -1,0 +1,72 @@
+// moe_common.cuh -- shared definitions of the CUDA path (kernels and host launchers).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+// ---- device error word (first 256 bytes of every workspace) -------------------------------
+constexpr int kErrBadIndex = 1;  // an expert id outside [0, E)
+constexpr int kErrTimeout = 2;   // a bounded device-side wait gave up
+constexpr size_t kWsHeader = 256;
+
+// wall-time limit of every spin-wait inside a kernel
+constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+
+__device__ __forceinline__ void set_error(int* err, int bits) {
+  if (err) atomicOr(err, bits);
+}
+
+// ---- bf16 helpers -----------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// two fp32 -> packed bf16x2 (round to nearest even), low half = a
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---- host launchers (defined in the .cu files) ---------------------------------------------
+cudaError_t launch_router_topk(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int D, int E,
+                               int k, int32_t* idx, float* w, int* err_to_clear, cudaStream_t s);
+
+size_t permute_scratch_bytes(int T, int E);
+cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16_t* x, int T, int D, int E,
+                           int k, int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,
+                           float* p_perm, uint16_t* x_perm, int32_t* scratch, int* err, cudaStream_t s,
+                           int* n_launches);
+
+cudaError_t launch_combine(const uint16_t* out_perm, const int32_t* inv_perm, const uint16_t* shared_out, int T,
+                           int D, int k, uint16_t* y, cudaStream_t s);
+
+// One "set" of a grouped GEMM launch: either the routed experts (groups = segments of the
+// expert-contiguous rows given by offsets) or the shared expert (one group of m_rows rows).
+struct GemmSetHost {
+  int K;                    // reduction length (multiple of 64)
+  const uint16_t* a;        // activations [a_rows, K]
+  int64_t a_rows;           // rows of the activation tensor (tensor-map extent)
+  const uint16_t* w;        // weights [n_groups * w_rows_per_group, K]
+  int n_groups;             // E (routed) or 1 (shared)
+  const int32_t* offsets;   // routed: device offsets[E+1]; shared: NULL
+  int m_rows;               // shared: rows of its single group
+  int n_out;                // output columns (F for gate_up -> h, D for down)
+  uint16_t* out;            // [rows, n_out] bf16
+  const float* row_scale;   // per-row factor (down) or NULL
+};
+
+enum GemmKind { kGateUp = 0, kDown = 1 };
+
+// Launch one grouped GEMM (gate_up + SwiGLU, or down + row scale) over up to two sets.
+// decode_nt > 0 selects the weight-streaming
+// kernels with a token tile of decode_nt (16/32/48/64); 0 selects the tiled kernels.
+cudaError_t launch_grouped_gemm(GemmKind kind, const GemmSetHost* sets, int n_sets, int decode_nt, int* err,
+                                cudaStream_t s);
+
+}  // namespace moe

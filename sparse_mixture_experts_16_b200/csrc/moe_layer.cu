@@ -1,0 +1,346 @@
+// moe_layer.cu -- the C ABI (include/moe_b200.h): argument validation, workspace layout and the
+// chaining of the layer's kernels on one stream.  Host code only; the kernels live in
+// router_topk.cu, permute.cu, grouped_gemm_sm100.cu and combine.cu.
+#include <cstdint>
+#include <cstring>
+
+#include "moe_common.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kDecodeTMax = 64;  // T <= this runs the weight-streaming kernels
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status_t check_device() {
+  static int verdict[64];  // 0 unknown, 1 ok, 2 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  if (dev < 64 && verdict[dev] == 1) return MOE_OK;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  if (dev < 64) verdict[dev] = major == 10 ? 1 : 2;
+  return major == 10 ? MOE_OK : MOE_ERR_NO_DEVICE;
+}
+
+moe_status_t shape_status(long long T, long long D, long long E, long long k) {
+  if (T < 0 || D <= 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (D % 64 != 0 || E > 1024 || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (T * k >= (1LL << 31) || T * D >= (1LL << 40)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+struct LayerWs {
+  size_t topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
+      out_sh, x_stage, y_stage, total;
+};
+
+LayerWs layer_ws(const moe_layer_desc_t& d) {
+  LayerWs w;
+  size_t o = kWsHeader;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  const size_t T = d.T, D = d.D, E = d.E, k = d.k, F = d.F, Fs = d.Fs, M = T * k;
+  w.topk_idx = take(M * 4);
+  w.topk_w = take(M * 4);
+  w.scratch = take(permute_scratch_bytes(d.T, d.E));
+  w.counts = take(E * 4);
+  w.offsets = take((E + 1) * 4);
+  w.perm_token = take(M * 4);
+  w.inv_perm = take(M * 4);
+  w.p_perm = take(M * 4);
+  w.x_perm = take(M * D * 2);
+  w.h = take(M * F * 2);
+  w.h_sh = take(T * Fs * 2);
+  w.out_perm = take(M * D * 2);
+  w.out_sh = take(T * D * 2);
+  w.x_stage = take(T * D * 2);
+  w.y_stage = take(T * D * 2);
+  w.total = o;
+  return w;
+}
+
+moe_status_t validate_desc(const moe_layer_desc_t* d) {
+  if (d == nullptr) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = shape_status(d->T, d->D, d->E, d->k);
+  if (st != MOE_OK) return st;
+  if (d->F <= 0 || d->Fs < 0) return MOE_ERR_INVALID_ARG;
+  if (d->F % 64 != 0 || d->Fs % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)d->E * 2 * d->F >= (1LL << 31) || (long long)d->T * d->k * d->F >= (1LL << 40))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!d->w_gate || !d->gate_up || !d->down) return MOE_ERR_INVALID_ARG;
+  if ((d->Fs > 0) != (d->shared_gate_up != nullptr) || (d->Fs > 0) != (d->shared_down != nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if ((d->flags & ~(MOE_FLAG_FORCE_PREFILL | MOE_FLAG_FORCE_DECODE)) != 0) return MOE_ERR_INVALID_ARG;
+  if ((d->flags & MOE_FLAG_FORCE_PREFILL) && (d->flags & MOE_FLAG_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
+  if ((d->flags & MOE_FLAG_FORCE_DECODE) && d->T > kDecodeTMax) return MOE_ERR_INVALID_ARG;
+  if (!aligned(d->w_gate, 16) || !aligned(d->gate_up, 16) || !aligned(d->down, 16) ||
+      !aligned(d->shared_gate_up, 16) || !aligned(d->shared_down, 16) || !aligned(d->bias, 4))
+    return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+bool use_decode(const moe_layer_desc_t& d) {
+  if (d.flags & MOE_FLAG_FORCE_DECODE) return true;
+  if (d.flags & MOE_FLAG_FORCE_PREFILL) return false;
+  return d.T <= kDecodeTMax;
+}
+
+int decode_tile(int max_seg) { return ((max_seg + 15) / 16) * 16; }
+
+#define MOE_CUDA_TRY(expr)                 \
+  do {                                     \
+    if ((expr) != cudaSuccess) {           \
+      cudaGetLastError();                  \
+      return MOE_ERR_CUDA;                 \
+    }                                      \
+  } while (0)
+
+moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float* row_scale, int M, int E, int D,
+                     int F, const uint16_t* gate_up, const uint16_t* down, uint16_t* h, uint16_t* out_perm,
+                     // optional shared expert over x[T, D]
+                     const uint16_t* x, int T, int Fs, const uint16_t* sgu, const uint16_t* sdn, uint16_t* h_sh,
+                     uint16_t* out_sh, int decode_nt, int* err, cudaStream_t s, cudaEvent_t ev_mid,
+                     unsigned ev_flags) {
+  GemmSetHost g[2];
+  memset(g, 0, sizeof(g));
+  g[0].K = D, g[0].a = x_perm, g[0].a_rows = M, g[0].w = gate_up, g[0].n_groups = E, g[0].offsets = offsets;
+  g[0].n_out = F, g[0].out = h;
+  int n_sets = 1;
+  if (Fs > 0) {
+    g[1].K = D, g[1].a = x, g[1].a_rows = T, g[1].w = sgu, g[1].n_groups = 1, g[1].m_rows = T;
+    g[1].n_out = Fs, g[1].out = h_sh;
+    n_sets = 2;
+  }
+  MOE_CUDA_TRY(launch_grouped_gemm(kGateUp, g, n_sets, decode_nt, err, s));
+  if (ev_mid) MOE_CUDA_TRY(cudaEventRecordWithFlags(ev_mid, s, ev_flags));
+  GemmSetHost dn[2];
+  memset(dn, 0, sizeof(dn));
+  dn[0].K = F, dn[0].a = h, dn[0].a_rows = M, dn[0].w = down, dn[0].n_groups = E, dn[0].offsets = offsets;
+  dn[0].n_out = D, dn[0].out = out_perm, dn[0].row_scale = row_scale;
+  if (Fs > 0) {
+    dn[1].K = Fs, dn[1].a = h_sh, dn[1].a_rows = T, dn[1].w = sdn, dn[1].n_groups = 1, dn[1].m_rows = T;
+    dn[1].n_out = D, dn[1].out = out_sh;
+  }
+  MOE_CUDA_TRY(launch_grouped_gemm(kDown, dn, n_sets, decode_nt, err, s));
+  return MOE_OK;
+}
+
+moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_t* y, void* ws, size_t ws_bytes,
+                           cudaStream_t s, cudaEvent_t const* ev) {
+  moe_status_t st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if (!x || !y || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  const LayerWs w = layer_ws(*d);
+  if (ws_bytes < w.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = check_device()) != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
+
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  int* err = reinterpret_cast<int*>(b);
+  auto I = [&](size_t off) { return reinterpret_cast<int32_t*>(b + off); };
+  auto Fp = [&](size_t off) { return reinterpret_cast<float*>(b + off); };
+  auto H = [&](size_t off) { return reinterpret_cast<uint16_t*>(b + off); };
+  const int T = d->T, D = d->D, E = d->E, k = d->k, F = d->F, Fs = d->Fs, M = T * k;
+
+  // Under stream capture, stage events become event-record nodes of the graph (so they can
+  // time each replay); otherwise they are plain records on the stream.
+  unsigned rec_flags = cudaEventRecordDefault;
+  if (ev) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    MOE_CUDA_TRY(cudaStreamIsCapturing(s, &cs));
+    if (cs == cudaStreamCaptureStatusActive) rec_flags = cudaEventRecordExternal;
+  }
+  auto record = [&](cudaEvent_t e) { return cudaEventRecordWithFlags(e, s, rec_flags); };
+
+  if (ev) MOE_CUDA_TRY(record(ev[0]));
+  MOE_CUDA_TRY(launch_router_topk(x, d->w_gate, d->bias, T, D, E, k, I(w.topk_idx), Fp(w.topk_w), err, s));
+  if (ev) MOE_CUDA_TRY(record(ev[1]));
+  MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), x, T, D, E, k, I(w.counts), I(w.offsets),
+                              I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), H(w.x_perm), I(w.scratch), err, s,
+                              nullptr));
+  if (ev) MOE_CUDA_TRY(record(ev[2]));
+  const int nt = use_decode(*d) ? decode_tile(T) : 0;
+  st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), H(w.out_perm), x,
+               T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), H(w.out_sh), nt, err, s, ev ? ev[3] : nullptr,
+               rec_flags);
+  if (st != MOE_OK) return st;
+  if (ev) MOE_CUDA_TRY(record(ev[4]));
+  MOE_CUDA_TRY(launch_combine(H(w.out_perm), I(w.inv_perm), Fs > 0 ? H(w.out_sh) : nullptr, T, D, k, y, s));
+  if (ev) MOE_CUDA_TRY(record(ev[5]));
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_INDEX: return "MOE_ERR_DEVICE_INDEX";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_NO_DEVICE: return "MOE_ERR_NO_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, const float* bias, int T, int D, int E,
+                             int k, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  moe_status_t st = shape_status(T, D, E, k);
+  if (st != MOE_OK) return st;
+  if (!x || !w_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_gate, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+    return MOE_ERR_ALIGNMENT;
+  if ((st = check_device()) != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  MOE_CUDA_TRY(launch_router_topk(x, w_gate, bias, T, D, E, k, topk_idx, topk_w, nullptr, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+size_t moe_permute_workspace_size(int T, int E, int k) {
+  if (shape_status(T, 64, E, k) != MOE_OK) return 0;
+  return kWsHeader + permute_scratch_bytes(T, E);
+}
+
+moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, const moe_bf16_t* x, int T, int D, int E, int k,
+                         int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* inv_perm, float* p_perm,
+                         moe_bf16_t* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = shape_status(T, D, E, k);
+  if (st != MOE_OK) return st;
+  if (!topk_idx || !topk_w || !counts || !offsets || !perm_token || !inv_perm || !p_perm || !ws)
+    return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(ws, 256) || !aligned(topk_idx, 4) ||
+      !aligned(topk_w, 4) || !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(perm_token, 4) ||
+      !aligned(inv_perm, 4) || !aligned(p_perm, 4))
+    return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < moe_permute_workspace_size(T, E, k)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = check_device()) != MOE_OK) return st;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  MOE_CUDA_TRY(launch_permute(topk_idx, topk_w, x, T, D, E, k, counts, offsets, perm_token, inv_perm, p_perm, x_perm,
+                              reinterpret_cast<int32_t*>(b + kWsHeader), reinterpret_cast<int*>(b),
+                              (cudaStream_t)stream, nullptr));
+  return MOE_OK;
+}
+
+size_t moe_grouped_swiglu_ffn_workspace_size(int M, int F) {
+  if (M < 0 || F <= 0 || F % 64 != 0) return 0;
+  return kWsHeader + align_up((size_t)M * F * 2, 256);
+}
+
+moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const float* row_scale, int M,
+                                    int max_seg, int E, int D, int F, const moe_bf16_t* gate_up,
+                                    const moe_bf16_t* down, moe_bf16_t* out_perm, void* ws, size_t ws_bytes,
+                                    moe_stream_t stream) {
+  if (M < 0 || E <= 0 || D <= 0 || F <= 0 || max_seg < 0 || max_seg > M) return MOE_ERR_INVALID_ARG;
+  if (D % 64 != 0 || F % 64 != 0 || E > 1024) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!x_perm || !offsets || !gate_up || !down || !out_perm || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x_perm, 16) || !aligned(gate_up, 16) || !aligned(down, 16) || !aligned(out_perm, 16) ||
+      !aligned(ws, 256) || !aligned(offsets, 4) || !aligned(row_scale, 4))
+    return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < moe_grouped_swiglu_ffn_workspace_size(M, F)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const int nt = max_seg <= kDecodeTMax ? decode_tile(max_seg < 1 ? 1 : max_seg) : 0;
+  return run_ffn(x_perm, offsets, row_scale, M, E, D, F, gate_up, down, reinterpret_cast<uint16_t*>(b + kWsHeader),
+                 out_perm, nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr, nt, reinterpret_cast<int*>(b),
+                 (cudaStream_t)stream, nullptr, cudaEventRecordDefault);
+}
+
+moe_status_t moe_combine(const moe_bf16_t* out_perm, const int32_t* inv_perm, const moe_bf16_t* shared_out, int T,
+                         int D, int k, moe_bf16_t* y, moe_stream_t stream) {
+  if (T < 0 || D <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+  if (D % 64 != 0 || k > 32 || (long long)T * k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!out_perm || !inv_perm || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned(out_perm, 16) || !aligned(shared_out, 16) || !aligned(y, 16) || !aligned(inv_perm, 4))
+    return MOE_ERR_ALIGNMENT;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  MOE_CUDA_TRY(launch_combine(out_perm, inv_perm, shared_out, T, D, k, y, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+size_t moe_layer_workspace_size(const moe_layer_desc_t* desc) {
+  if (validate_desc(desc) != MOE_OK) return 0;
+  return layer_ws(*desc).total;
+}
+
+moe_status_t moe_layer_forward(const moe_layer_desc_t* desc, const moe_bf16_t* x, moe_bf16_t* y, void* ws,
+                               size_t ws_bytes, moe_stream_t stream) {
+  return layer_forward(desc, x, y, ws, ws_bytes, (cudaStream_t)stream, nullptr);
+}
+
+moe_status_t moe_layer_forward_timed(const moe_layer_desc_t* desc, const moe_bf16_t* x, moe_bf16_t* y, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream, void* const* events, int n_events) {
+  if (events == nullptr || n_events < 6) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (events[i] == nullptr) return MOE_ERR_INVALID_ARG;
+  return layer_forward(desc, x, y, ws, ws_bytes, (cudaStream_t)stream,
+                       reinterpret_cast<cudaEvent_t const*>(events));
+}
+
+moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16_t* x_host, moe_bf16_t* y_host,
+                                    void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = validate_desc(desc);
+  if (st != MOE_OK) return st;
+  if (!x_host || !y_host || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  const LayerWs w = layer_ws(*desc);
+  if (ws_bytes < w.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = check_device()) != MOE_OK) return st;
+  if (desc->T == 0) return MOE_OK;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const size_t bytes = (size_t)desc->T * desc->D * 2;
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_CUDA_TRY(cudaMemcpyAsync(b + w.x_stage, x_host, bytes, cudaMemcpyHostToDevice, s));
+  st = layer_forward(desc, reinterpret_cast<uint16_t*>(b + w.x_stage), reinterpret_cast<uint16_t*>(b + w.y_stage),
+                     ws, ws_bytes, s, nullptr);
+  if (st != MOE_OK) return st;
+  MOE_CUDA_TRY(cudaMemcpyAsync(y_host, b + w.y_stage, bytes, cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
+}
+
+int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
+  if (validate_desc(desc) != MOE_OK || desc->T == 0) return 0;
+  return 1 /*router*/ + 4 /*hist, scan, scatter, gather*/ + 2 /*grouped GEMMs*/ + 1 /*combine*/;
+}
+
+moe_status_t moe_get_device_error(void* ws, moe_stream_t stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  int h = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_CUDA_TRY(cudaMemcpyAsync(&h, ws, sizeof(int), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA_TRY(cudaStreamSynchronize(s));
+  if (h != 0) {
+    MOE_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), s));
+    MOE_CUDA_TRY(cudaStreamSynchronize(s));
+  }
+  if (h & kErrTimeout) return MOE_ERR_TIMEOUT;
+  if (h & kErrBadIndex) return MOE_ERR_DEVICE_INDEX;
+  return MOE_OK;
+}
+
+}  // extern "C"

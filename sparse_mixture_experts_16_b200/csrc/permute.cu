@@ -1,0 +1,169 @@
+// permute.cu -- step 2 of the layer: dispatch tokens into expert-contiguous order.
+//
+// keryc.com "Mixture of Experts optimiza Transformers y LLMs", section "Ejecucion eficiente:
+// backends de expertos": the grouped backend sorts the tokens by expert id before the grouped
+// GEMMs and puts the results back in the original order afterwards.
+//
+// A deterministic, stable counting sort of the T*k (token, slot) pairs by expert id:
+//   1. hist    : per block of 256 tokens, per-expert counts with shared-memory atomics
+//   2. scan    : per expert, exclusive scan over blocks; then exclusive scan over experts
+//   3. scatter : per block, one warp walks the block's slots in (token, slot) order; ranks of
+//                equal experts inside each 32-slot step come from __match_any_sync + popc, and
+//                a shared running counter per expert carries them across steps
+//   4. gather  : x_perm[r] = x[perm_token[r]], one warp per row, 16-byte vector moves
+// Within an expert, rows are therefore ordered by token id (a token picks an expert at most once).
+#include "moe_common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTokPerBlock = 256;
+
+__global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                                                   int32_t* __restrict__ block_counts, int* err) {
+  extern __shared__ int cnt[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kTokPerBlock;
+  const int n_items = min(T - t0, kTokPerBlock) * k;
+  const int32_t* base = idx + (size_t)t0 * k;
+  for (int i = threadIdx.x; i < n_items; i += blockDim.x) {
+    const int e = base[i];
+    if ((unsigned)e < (unsigned)E)
+      atomicAdd(&cnt[e], 1);
+    else
+      set_error(err, kErrBadIndex);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) block_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// One block of 1024 threads.  block_counts[b][e] becomes the exclusive prefix over blocks.
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_counts, int nb, int E,
+                                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ int32_t warp_tot[32];
+  const int e = threadIdx.x;  // E <= 1024
+  int total = 0;
+  if (e < E) {
+    for (int b = 0; b < nb; ++b) {
+      const int v = block_counts[(size_t)b * E + e];
+      block_counts[(size_t)b * E + e] = total;
+      total += v;
+    }
+    counts[e] = total;
+  }
+  // block-wide inclusive scan of total over e
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = total;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += v;
+    }
+    warp_tot[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  if (warp > 0) incl += warp_tot[warp - 1];
+  if (e < E) offsets[e + 1] = incl;
+  if (e == 0) offsets[0] = 0;
+}
+
+// One warp per block of 256 tokens; order-preserving ranks.
+__global__ void __launch_bounds__(32) scatter_kernel(const int32_t* __restrict__ idx, const float* __restrict__ w,
+                                                     int T, int E, int k, const int32_t* __restrict__ block_off,
+                                                     const int32_t* __restrict__ offsets,
+                                                     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm,
+                                                     float* __restrict__ p_perm) {
+  extern __shared__ int run[];  // next free row per expert
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) run[e] = offsets[e] + block_off[(size_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int t0 = blockIdx.x * kTokPerBlock;
+  const int n_items = min(T - t0, kTokPerBlock) * k;
+  const size_t base = (size_t)t0 * k;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int i0 = 0; i0 < n_items; i0 += 32) {
+    const int i = i0 + lane;
+    int e = -1;
+    if (i < n_items) {
+      e = idx[base + i];
+      if ((unsigned)e >= (unsigned)E) {
+        inv_perm[base + i] = -1;  // dropped slot (error already recorded by hist_kernel)
+        e = -1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int r = run[e] + __popc(peers & lt_mask);
+      const size_t slot = base + i;
+      perm_token[r] = (int32_t)(slot / k);
+      inv_perm[slot] = r;
+      p_perm[r] = w[slot];
+    }
+    __syncwarp();
+    if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// x_perm[r] = x[perm_token[r]] for r < offsets[E]; one warp per row, 16-byte moves.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
+                                                          const int32_t* __restrict__ perm_token,
+                                                          const int32_t* __restrict__ offsets, int E, int T,
+                                                          int D, uint16_t* __restrict__ x_perm) {
+  const int n_rows = offsets[E];
+  const int lane = threadIdx.x & 31;
+  const int nv = D / 8;
+  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n_rows; r += (gridDim.x * blockDim.x) >> 5) {
+    const int t = perm_token[r];
+    if ((unsigned)t >= (unsigned)T) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * D);
+    for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+}  // namespace
+
+size_t permute_scratch_bytes(int T, int E) {
+  const size_t nb = (size_t)(T + kTokPerBlock - 1) / kTokPerBlock;
+  return align_up(nb * (size_t)E * sizeof(int32_t), 256);
+}
+
+cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16_t* x, int T, int D, int E, int k,
+                           int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* inv_perm, float* p_perm,
+                           uint16_t* x_perm, int32_t* scratch, int* err, cudaStream_t s, int* n_launches) {
+  const int nb = (T + kTokPerBlock - 1) / kTokPerBlock;
+  int launches = 0;
+  if (nb > 0) {
+    hist_kernel<<<nb, 256, E * sizeof(int), s>>>(idx, T, E, k, scratch, err);
+    ++launches;
+  }
+  scan_kernel<<<1, 1024, 0, s>>>(scratch, nb, E, counts, offsets);
+  ++launches;
+  if (nb > 0) {
+    scatter_kernel<<<nb, 32, E * sizeof(int), s>>>(idx, topk_w, T, E, k, scratch, offsets, perm_token, inv_perm,
+                                                 p_perm);
+    ++launches;
+  }
+  if (x != nullptr && x_perm != nullptr && T > 0) {
+    const long long rows = (long long)T * k;
+    long long blocks = (rows + 7) / 8;
+    if (blocks > 148LL * 16) blocks = 148LL * 16;
+    gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, perm_token, offsets, E, T, D, x_perm);
+    ++launches;
+  }
+  if (n_launches) *n_launches = launches;
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,133 @@
+"""The C-ABI library on the host (no GPU needed): it loads, exports every symbol the header
+declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sparse_mixture_experts_16_b200 as moe
+from sparse_mixture_experts_16_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    moe_build.build()
+    return moe.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert sorted(_declared()) == sorted(moe.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\bT (moe_\w+)", out.stdout))
+    missing = [s for s in _declared() if s not in exported]
+    assert not missing, missing
+    for s in _declared():
+        assert getattr(L, s) is not None
+
+
+def test_status_strings(L):
+    for code, name in moe.STATUS.items():
+        assert moe.moe_status_string(code) == name
+    assert moe.moe_status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+def _desc(**kw):
+    base = dict(T=16, D=128, E=8, k=2, F=128, Fs=0, w_gate=0x1000, bias=None, gate_up=0x2000, down=0x3000,
+                shared_gate_up=None, shared_down=None, flags=0)
+    base.update(kw)
+    return moe.LayerDesc(*[base[n] for n, _ in moe.LayerDesc._fields_])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=9), 1),               # k > E
+    (dict(k=0), 1),
+    (dict(T=-1), 1),
+    (dict(D=96), 2),              # not a multiple of 64
+    (dict(F=100), 2),
+    (dict(E=1025, k=2), 2),
+    (dict(E=64, k=33), 2),        # k > 32
+    (dict(Fs=64), 1),             # shared size without shared weights
+    (dict(w_gate=None), 1),
+    (dict(w_gate=0x1008), 3),     # misaligned
+    (dict(flags=3), 1),           # both force flags
+    (dict(flags=2, T=65), 1),     # decode forced above the decode range
+])
+def test_layer_forward_rejects_bad_descriptors(L, kw, status):
+    d = _desc(**kw)
+    assert L.moe_layer_workspace_size(ctypes.byref(d)) == 0
+    st = L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, 1 << 30, None)
+    assert st == status, moe.STATUS.get(st)
+
+
+def test_layer_workspace_size_and_small_workspace(L):
+    d = _desc()
+    need = L.moe_layer_workspace_size(ctypes.byref(d))
+    assert need > 256 and need % 256 == 0
+    assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, need - 1, None) == 4
+    assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100010, need, None) == 3  # ws not 256-aligned
+    assert L.moe_layer_forward(ctypes.byref(d), 0x4008, 0x5000, 0x100000, need, None) == 3
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 8
+    assert L.moe_layer_kernel_count(ctypes.byref(_desc(k=9))) == 0
+    # shared expert grows the workspace
+    d2 = _desc(Fs=256, shared_gate_up=0x6000, shared_down=0x7000)
+    assert L.moe_layer_workspace_size(ctypes.byref(d2)) > need
+
+
+def test_step_entry_points_validate_on_host(L):
+    # router: k > E, D not multiple of 64, misaligned x
+    assert L.moe_router_topk(0x1000, 0x2000, None, 4, 128, 4, 5, 0x3000, 0x4000, None) == 1
+    assert L.moe_router_topk(0x1000, 0x2000, None, 4, 100, 4, 2, 0x3000, 0x4000, None) == 2
+    assert L.moe_router_topk(0x1001, 0x2000, None, 4, 128, 4, 2, 0x3000, 0x4000, None) == 3
+    assert L.moe_router_topk(None, 0x2000, None, 4, 128, 4, 2, 0x3000, 0x4000, None) == 1
+    # permute: workspace too small, x without x_perm
+    need = L.moe_permute_workspace_size(300, 8, 2)
+    assert need >= 256 + 2 * 8 * 4
+    args = [0x1000, 0x2000, 0x3000, 300, 128, 8, 2, 0x4000, 0x5000, 0x6000, 0x7000, 0x8000, 0x9000]
+    assert L.moe_permute(*args, 0x100000, need - 1, None) == 4
+    args_bad = list(args)
+    args_bad[-1] = None  # x given, x_perm missing
+    assert L.moe_permute(*args_bad, 0x100000, need, None) == 1
+    # grouped ffn: max_seg > M, F not multiple of 64
+    assert L.moe_grouped_swiglu_ffn(0x1000, 0x2000, None, 10, 11, 4, 128, 128, 0x3000, 0x4000, 0x5000, 0x100000,
+                                    1 << 20, None) == 1
+    assert L.moe_grouped_swiglu_ffn(0x1000, 0x2000, None, 10, 10, 4, 128, 100, 0x3000, 0x4000, 0x5000, 0x100000,
+                                    1 << 20, None) == 2
+    assert L.moe_grouped_swiglu_ffn_workspace_size(10, 128) == 256 + 2560 + (256 - 2560 % 256) % 256
+    # combine: k > 32, misaligned y
+    assert L.moe_combine(0x1000, 0x2000, None, 4, 128, 33, 0x3000, None) == 2
+    assert L.moe_combine(0x1000, 0x2000, None, 4, 128, 2, 0x3004, None) == 3
+    # timed forward needs 6 events
+    d = _desc()
+    assert L.moe_layer_forward_timed(ctypes.byref(d), 0x4000, 0x5000, 0x100000, 1 << 30, None, None, 0) == 1
+
+
+def test_valid_call_without_a_gpu_reports_no_device(L):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    d = _desc()
+    need = L.moe_layer_workspace_size(ctypes.byref(d))
+    assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, need, None) == 8
+    assert L.moe_get_device_error(0x100000, None) == 8
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(moe, "_lib", None)
+    monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(ImportError):
+        moe.lib()
