@@ -106,7 +106,8 @@ moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, const moe
  *   max_seg:  an upper bound on any segment length (pass M if unknown).  max_seg <= 64
  *             selects the weight-streaming (decode) kernels, otherwise the tiled kernels.
  *   gate_up  [E, 2F, D] bf16, down [E, D, F] bf16
- *   out_perm [M, D] bf16 out:   out_perm[r] = row_scale[r] * Expert_e(x_perm[r]) (bf16)
+ *   out_perm [M, D] fp32 out:   out_perm[r] = row_scale[r] * Expert_e(x_perm[r])
+ *            (kept in fp32 so that y is rounded to bf16 once, in the combine)
  *   ws: >= moe_grouped_swiglu_ffn_workspace_size(M, F) bytes (holds h = silu(G x) * (U x),
  *       [M, F] bf16); first 256 bytes: the device error word.
  * ---------------------------------------------------------------------------------------- */
@@ -114,19 +115,18 @@ size_t moe_grouped_swiglu_ffn_workspace_size(int M, int F);
 moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* offsets,
                                     const float* row_scale, int M, int max_seg, int E, int D, int F,
                                     const moe_bf16_t* gate_up, const moe_bf16_t* down,
-                                    moe_bf16_t* out_perm, void* ws, size_t ws_bytes,
-                                    moe_stream_t stream);
+                                    float* out_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
  * Step 4: weighted combine back to token order (gotburnout.io glossary, section 2 "Weighted
  * Aggregation", section 3 step 4).  out_perm rows are already scaled by their router weight.
  *
- *   y[t] = sum_{j=0..k-1} out_perm[inv_perm[t*k + j]] + shared_out[t]     (fp32 sum, j order)
- *   out_perm [T*k, D] bf16, inv_perm [T*k] int32, shared_out [T, D] bf16 or NULL, y [T, D] bf16
+ *   y[t] = bf16( sum_{j=0..k-1} out_perm[inv_perm[t*k + j]] + shared_out[t] )  (fp32 sum, j order)
+ *   out_perm [T*k, D] fp32, inv_perm [T*k] int32 (entries < 0 are skipped), shared_out [T, D]
+ *   fp32 or NULL, y [T, D] bf16
  * ---------------------------------------------------------------------------------------- */
-moe_status_t moe_combine(const moe_bf16_t* out_perm, const int32_t* inv_perm,
-                         const moe_bf16_t* shared_out, int T, int D, int k, moe_bf16_t* y,
-                         moe_stream_t stream);
+moe_status_t moe_combine(const float* out_perm, const int32_t* inv_perm, const float* shared_out,
+                         int T, int D, int k, moe_bf16_t* y, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
  * The whole layer (steps 1-4, plus the always-on shared expert of gotburnout.io glossary,

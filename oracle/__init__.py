@@ -202,7 +202,7 @@ def gap_violations(s, k, delta=GAP):
     return (np.diff(-top, axis=1) < delta).any(axis=1)
 
 
-def gap_redraw(w, delta=GAP, max_rounds=50):
+def gap_redraw(w, delta=GAP, max_rounds=200):
     """Per-token substream index for workload ``w`` (a moe_inputs.Workload) such that every
     token's router scores keep the minimum gap; a violating token row is redrawn from the next
     substream of x, deterministically."""

@@ -165,7 +165,7 @@ def moe_grouped_swiglu_ffn(x_perm, offsets, row_scale, gate_up, down, max_seg=No
     F = twoF // 2
     assert D2 == D and tuple(down.shape) == (E, D, F)
     if out_perm is None:
-        out_perm = torch.empty(M, D, dtype=torch.bfloat16, device=x_perm.device)
+        out_perm = torch.empty(M, D, dtype=torch.float32, device=x_perm.device)
     need = lib().moe_grouped_swiglu_ffn_workspace_size(M, F)
     if ws is None or ws.numel() < need:
         ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x_perm.device)

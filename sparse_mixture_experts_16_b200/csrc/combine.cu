@@ -2,19 +2,26 @@
 //
 // gotburnout.io glossary "MoE", section 2 ("Weighted Aggregation: y = Sum(p_i * Expert_i(x))")
 // and section 3 step 4: the selected experts' outputs, already multiplied by their normalised
-// router weights in the down-projection epilogue, are summed per token; the always-on shared
-// expert's output is added with weight 1.
+// router weights in the down-projection epilogue (kept in fp32), are summed per token; the
+// always-on shared expert's output is added with weight 1; y is rounded once to bf16.
 //
 // One warp per token row: the k row indices are loaded once and broadcast with shuffles, then
-// every lane sums 8 bf16 columns at a time (16-byte loads) in fp32, in slot order j = 0..k-1.
+// every lane sums 8 fp32 columns at a time (two 16-byte loads per row) in slot order j = 0..k-1.
 #include "moe_common.cuh"
 
 namespace moe {
 namespace {
 
-__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ out_perm,
+__device__ __forceinline__ void add8(float (&acc)[8], const float* src) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  acc[0] += a.x, acc[1] += a.y, acc[2] += a.z, acc[3] += a.w;
+  acc[4] += b.x, acc[5] += b.y, acc[6] += b.z, acc[7] += b.w;
+}
+
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ out_perm,
                                                       const int32_t* __restrict__ inv_perm,
-                                                      const uint16_t* __restrict__ shared_out, int T, int D, int k,
+                                                      const float* __restrict__ shared_out, int T, int D, int k,
                                                       uint16_t* __restrict__ y) {
   const int lane = threadIdx.x & 31;
   const int nv = D / 8;
@@ -26,15 +33,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
       for (int j = 0; j < k; ++j) {
         const int r = __shfl_sync(0xffffffffu, my_row, j);
         if (r < 0 || r >= M) continue;
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(out_perm + (size_t)r * D) + v);
-        acc[0] += bf16_lo(q.x), acc[1] += bf16_hi(q.x), acc[2] += bf16_lo(q.y), acc[3] += bf16_hi(q.y);
-        acc[4] += bf16_lo(q.z), acc[5] += bf16_hi(q.z), acc[6] += bf16_lo(q.w), acc[7] += bf16_hi(q.w);
+        add8(acc, out_perm + (size_t)r * D + 8 * v);
       }
-      if (shared_out != nullptr) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(shared_out + (size_t)t * D) + v);
-        acc[0] += bf16_lo(q.x), acc[1] += bf16_hi(q.x), acc[2] += bf16_lo(q.y), acc[3] += bf16_hi(q.y);
-        acc[4] += bf16_lo(q.z), acc[5] += bf16_hi(q.z), acc[6] += bf16_lo(q.w), acc[7] += bf16_hi(q.w);
-      }
+      if (shared_out != nullptr) add8(acc, shared_out + (size_t)t * D + 8 * v);
       uint4 o;
       o.x = pack_bf16x2(acc[0], acc[1]);
       o.y = pack_bf16x2(acc[2], acc[3]);
@@ -47,8 +48,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 
 }  // namespace
 
-cudaError_t launch_combine(const uint16_t* out_perm, const int32_t* inv_perm, const uint16_t* shared_out, int T,
-                           int D, int k, uint16_t* y, cudaStream_t s) {
+cudaError_t launch_combine(const float* out_perm, const int32_t* inv_perm, const float* shared_out, int T, int D,
+                           int k, uint16_t* y, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   long long blocks = ((long long)T + 7) / 8;
   if (blocks > 148LL * 16) blocks = 148LL * 16;

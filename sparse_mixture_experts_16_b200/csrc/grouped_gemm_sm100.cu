@@ -12,7 +12,7 @@
 //
 // One kernel template, two GEMMs, two regimes:
 //   kGateUp : h[r, :]   = silu(A[r] G_e^T) * (A[r] U_e^T)             (SwiGLU in the epilogue)
-//   kDown   : out[r, :] = row_scale[r] * (h[r] Down_e^T)                (router weight in epilogue)
+//   kDown   : out[r, :] = row_scale[r] * (h[r] Down_e^T)  in fp32       (router weight in epilogue)
 //   tiled (prefill, NT = 0): a tile is 128 activation rows of one expert segment x 256 MMA
 //       columns (gate_up: 128 gate + 128 up weight rows, so both halves of a SwiGLU output land
 //       in the same TMEM lane; down: 256 weight rows).  MMA M=128, N=256, K=16.
@@ -48,7 +48,7 @@ struct alignas(64) GemmParams {
   CUtensorMap a_map[2];  // activations per set (box rows: 128 tiled / NT streaming)
   CUtensorMap w_map[2];  // weights per set (box rows: 128, or 256 for tiled kDown)
   const int32_t* offsets[2];
-  uint16_t* out[2];
+  void* out[2];  // kGateUp: bf16 h [rows, F]; kDown: fp32 [rows, D]
   const float* row_scale[2];
   int n_groups[2];
   int m_rows[2];
@@ -311,7 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
       const Tile ti = decode_tile<KIND, NT>(p, tile_start, G, t);
       const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * C::kAccCols;
       const int n_out = p.n_out[ti.set];
-      uint16_t* out = p.out[ti.set];
+      uint16_t* out_h = static_cast<uint16_t*>(p.out[ti.set]);
+      float* out_f = static_cast<float*>(p.out[ti.set]);
       if constexpr (C::kTiled) {
         const int r_local = ti.m * kBM + q * 32 + lane;
         const bool row_ok = r_local < ti.rows;
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
               for (int i = 0; i < 16; ++i)
                 pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
                                     silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
-              uint4* dst = reinterpret_cast<uint4*>(out + grow * n_out + col);
+              uint4* dst = reinterpret_cast<uint4*>(out_h + grow * n_out + col);
 #pragma unroll
               for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
             }
@@ -346,13 +347,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             tmem_ld_32x32b_x32(tacc + c0, a);
             tmem_ld_wait();
             if (row_ok) {
-              uint32_t pk[16];
+              float4* dst = reinterpret_cast<float4*>(out_f + grow * n_out + col);
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(__uint_as_float(a[2 * i]) * sc, __uint_as_float(a[2 * i + 1]) * sc);
-              uint4* dst = reinterpret_cast<uint4*>(out + grow * n_out + col);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(a[4 * v]) * sc, __uint_as_float(a[4 * v + 1]) * sc,
+                                     __uint_as_float(a[4 * v + 2]) * sc, __uint_as_float(a[4 * v + 3]) * sc);
             }
           }
         }
@@ -373,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
               const int j = j0 + jj;
               if (j < ti.rows && col_ok) {
                 const float h = silu_mul(__uint_as_float(g[jj]), __uint_as_float(u[jj]));
-                out[(size_t)(ti.row0 + j) * n_out + col] = (uint16_t)(pack_bf16x2(h, 0.f) & 0xFFFFu);
+                out_h[(size_t)(ti.row0 + j) * n_out + col] = (uint16_t)(pack_bf16x2(h, 0.f) & 0xFFFFu);
               }
             }
           } else {
@@ -386,8 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
               const int j = j0 + jj;
               if (j < ti.rows && col_ok) {
                 const float sc = rs != nullptr ? rs[ti.row0 + j] : 1.0f;
-                out[(size_t)(ti.row0 + j) * n_out + col] =
-                    (uint16_t)(pack_bf16x2(__uint_as_float(a[jj]) * sc, 0.f) & 0xFFFFu);
+                out_f[(size_t)(ti.row0 + j) * n_out + col] = __uint_as_float(a[jj]) * sc;
               }
             }
           }

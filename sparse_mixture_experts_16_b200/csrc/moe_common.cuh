@@ -43,8 +43,8 @@ cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16
                            float* p_perm, uint16_t* x_perm, int32_t* scratch, int* err, cudaStream_t s,
                            int* n_launches);
 
-cudaError_t launch_combine(const uint16_t* out_perm, const int32_t* inv_perm, const uint16_t* shared_out, int T,
-                           int D, int k, uint16_t* y, cudaStream_t s);
+cudaError_t launch_combine(const float* out_perm, const int32_t* inv_perm, const float* shared_out, int T, int D,
+                           int k, uint16_t* y, cudaStream_t s);
 
 // One "set" of a grouped GEMM launch: either the routed experts (groups = segments of the
 // expert-contiguous rows given by offsets) or the shared expert (one group of m_rows rows).
@@ -57,7 +57,7 @@ struct GemmSetHost {
   const int32_t* offsets;   // routed: device offsets[E+1]; shared: NULL
   int m_rows;               // shared: rows of its single group
   int n_out;                // output columns (F for gate_up -> h, D for down)
-  uint16_t* out;            // [rows, n_out] bf16
+  void* out;                // [rows, n_out]: bf16 (gate_up -> h) or fp32 (down)
   const float* row_scale;   // per-row factor (down) or NULL
 };
 

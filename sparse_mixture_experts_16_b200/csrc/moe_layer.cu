@@ -63,8 +63,8 @@ LayerWs layer_ws(const moe_layer_desc_t& d) {
   w.x_perm = take(M * D * 2);
   w.h = take(M * F * 2);
   w.h_sh = take(T * Fs * 2);
-  w.out_perm = take(M * D * 2);
-  w.out_sh = take(T * D * 2);
+  w.out_perm = take(M * D * 4);
+  w.out_sh = take(T * D * 4);
   w.x_stage = take(T * D * 2);
   w.y_stage = take(T * D * 2);
   w.total = o;
@@ -108,10 +108,10 @@ int decode_tile(int max_seg) { return ((max_seg + 15) / 16) * 16; }
   } while (0)
 
 moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float* row_scale, int M, int E, int D,
-                     int F, const uint16_t* gate_up, const uint16_t* down, uint16_t* h, uint16_t* out_perm,
+                     int F, const uint16_t* gate_up, const uint16_t* down, uint16_t* h, float* out_perm,
                      // optional shared expert over x[T, D]
                      const uint16_t* x, int T, int Fs, const uint16_t* sgu, const uint16_t* sdn, uint16_t* h_sh,
-                     uint16_t* out_sh, int decode_nt, int* err, cudaStream_t s, cudaEvent_t ev_mid,
+                     float* out_sh, int decode_nt, int* err, cudaStream_t s, cudaEvent_t ev_mid,
                      unsigned ev_flags) {
   GemmSetHost g[2];
   memset(g, 0, sizeof(g));
@@ -173,12 +173,12 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
                               nullptr));
   if (ev) MOE_CUDA_TRY(record(ev[2]));
   const int nt = use_decode(*d) ? decode_tile(T) : 0;
-  st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), H(w.out_perm), x,
-               T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), H(w.out_sh), nt, err, s, ev ? ev[3] : nullptr,
+  st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), Fp(w.out_perm), x,
+               T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, err, s, ev ? ev[3] : nullptr,
                rec_flags);
   if (st != MOE_OK) return st;
   if (ev) MOE_CUDA_TRY(record(ev[4]));
-  MOE_CUDA_TRY(launch_combine(H(w.out_perm), I(w.inv_perm), Fs > 0 ? H(w.out_sh) : nullptr, T, D, k, y, s));
+  MOE_CUDA_TRY(launch_combine(Fp(w.out_perm), I(w.inv_perm), Fs > 0 ? Fp(w.out_sh) : nullptr, T, D, k, y, s));
   if (ev) MOE_CUDA_TRY(record(ev[5]));
   return MOE_OK;
 }
@@ -248,7 +248,7 @@ size_t moe_grouped_swiglu_ffn_workspace_size(int M, int F) {
 
 moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const float* row_scale, int M,
                                     int max_seg, int E, int D, int F, const moe_bf16_t* gate_up,
-                                    const moe_bf16_t* down, moe_bf16_t* out_perm, void* ws, size_t ws_bytes,
+                                    const moe_bf16_t* down, float* out_perm, void* ws, size_t ws_bytes,
                                     moe_stream_t stream) {
   if (M < 0 || E <= 0 || D <= 0 || F <= 0 || max_seg < 0 || max_seg > M) return MOE_ERR_INVALID_ARG;
   if (D % 64 != 0 || F % 64 != 0 || E > 1024) return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -267,8 +267,8 @@ moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* off
                  (cudaStream_t)stream, nullptr, cudaEventRecordDefault);
 }
 
-moe_status_t moe_combine(const moe_bf16_t* out_perm, const int32_t* inv_perm, const moe_bf16_t* shared_out, int T,
-                         int D, int k, moe_bf16_t* y, moe_stream_t stream) {
+moe_status_t moe_combine(const float* out_perm, const int32_t* inv_perm, const float* shared_out, int T, int D,
+                         int k, moe_bf16_t* y, moe_stream_t stream) {
   if (T < 0 || D <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
   if (D % 64 != 0 || k > 32 || (long long)T * k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!out_perm || !inv_perm || !y) return MOE_ERR_INVALID_ARG;

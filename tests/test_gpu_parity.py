@@ -30,8 +30,8 @@ def W(T, D, E, k, F, Fs=0, bias="none", seed=0):
     return mi.Workload(f"T{T}D{D}E{E}k{k}F{F}Fs{Fs}", T=T, D=D, E=E, k=k, F=F, Fs=Fs, bias=bias, seed=seed)
 
 
-def host_case(w):
-    rd = gap_redraw(w)
+def host_case(w, delta=None):
+    rd = gap_redraw(w) if delta is None else gap_redraw(w, delta)
     return mi.host_inputs(w, redraw=rd), rd
 
 
@@ -95,7 +95,9 @@ ROUTER_CASES = [
 
 @pytest.mark.parametrize("w", ROUTER_CASES, ids=lambda w: w.name)
 def test_router_topk_parity(w):
-    inp, _ = host_case(w)
+    # with k = 32 of E = 1024 the 33 top scores are dense; at D = 128 the fp32 logit error is
+    # ~1e-6, so a 2e-4 gap is still far above it
+    inp, _ = host_case(w, delta=2e-4 if w.k >= 32 else None)
     d = device_from_host(inp)
     idx, wts = moe.moe_router_topk(d["x"], d["wg"], d["bias"], w.k)
     o_idx, o_p = oracle.router(inp["x"], inp["wg"], inp["bias"], w.k)
@@ -167,18 +169,17 @@ def test_combine_bit_exact(T, k, D, shared):
 
     rng = np.random.default_rng(T + k)
     M = T * k
-    outp = mi.rows_bf16(mi.STREAM_DOWN, np.arange(M), D, 0.5)
+    outp = rng.standard_normal((M, D)).astype(np.float32)
     inv = rng.permutation(M).astype(np.int32)
-    sh = mi.rows_bf16(mi.STREAM_SH_DOWN, np.arange(T), D, 0.5) if shared else None
-    y = moe.moe_combine(to_torch_bf16(outp), torch.from_numpy(inv).cuda(),
-                        to_torch_bf16(sh) if shared else None, T, k)
+    sh = rng.standard_normal((T, D)).astype(np.float32) if shared else None
+    y = moe.moe_combine(torch.from_numpy(outp).cuda(), torch.from_numpy(inv).cuda(),
+                        torch.from_numpy(sh).cuda() if shared else None, T, k)
     # definition: fp32 sum over j = 0..k-1 in order, then the shared row, rounded to bf16
-    vals = bf16_np_to_f64(outp).astype(np.float32)
     acc = np.zeros((T, D), np.float32)
     for j in range(k):
-        acc += vals[inv.reshape(T, k)[:, j]]
+        acc += outp[inv.reshape(T, k)[:, j]]
     if shared:
-        acc += bf16_np_to_f64(sh).astype(np.float32)
+        acc += sh
     u = acc.view(np.uint32).astype(np.uint64)
     ref = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
     assert (to_np_bf16(y) == ref).all()
@@ -198,8 +199,9 @@ def test_grouped_ffn_rows_match_oracle_expert_ffn(max_seg_mode):
     scale = p.reshape(-1)[pt * k + ps].astype(np.float32)
     out, _ = moe.moe_grouped_swiglu_ffn(to_torch_bf16(xp), torch.from_numpy(offsets).cuda(),
                                         torch.from_numpy(scale).cuda(), to_torch_bf16(inp["gate_up"]),
-                                        to_torch_bf16(inp["down"]), max_seg=int(counts.max()))
-    got = bf16_np_to_f64(to_np_bf16(out))
+                                        to_torch_bf16(inp["down"]),
+                                        max_seg=int(counts.max()) if max_seg_mode == "stream" else None)
+    got = out.cpu().numpy().astype(np.float64)
     ref = np.stack([scale[r] * oracle.expert_ffn(xp[r], inp["gate_up"][e], inp["down"][e])
                     for e in range(E) for r in range(offsets[e], offsets[e + 1])])
     assert rel_rms_err(got, ref) <= REL_RMS_TOL
