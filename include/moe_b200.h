@@ -96,6 +96,31 @@ moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, const moe
                          size_t ws_bytes, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
+ * moe_permute without a workspace.  The pages have no counterpart to this entry point: it
+ * exists for callers that cannot allocate device memory -- their GPU memory is owned by
+ * someone else (an inference engine that reserves the device's memory for its own pools up
+ * front, a plugin whose host program does not share its allocator) -- and so cannot hand
+ * moe_permute a workspace.  It allocates nothing.
+ *
+ * Arguments, results and row order are those of moe_permute, without ws / ws_bytes.  The
+ * scratch (per-block expert counts) is a fixed 512 KiB array inside the library, held by every
+ * GPU that loads the library until the process exits; it fits ceil(T/256) * E <= 131072
+ * (e.g. T <= 32768 with E = 1024).  Larger sizes return MOE_ERR_WORKSPACE_TOO_SMALL and
+ * launch nothing.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture.
+ * All calls share the one array: calls whose kernels overlap on the GPU (e.g. on two streams
+ * with no ordering between them) race and give wrong results.  Each call writes every scratch
+ * entry it reads, so contents left by an earlier call do no harm.
+ * Out-of-range expert ids are dropped as in moe_permute (inv_perm entry -1) but, with no
+ * workspace, there is no error word that reports them.
+ * ---------------------------------------------------------------------------------------- */
+moe_status_t moe_permute_noalloc(const int32_t* topk_idx, const float* topk_w, const moe_bf16_t* x,
+                                 int T, int D, int E, int k, int32_t* counts, int32_t* offsets,
+                                 int32_t* perm_token, int32_t* inv_perm, float* p_perm,
+                                 moe_bf16_t* x_perm, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
  * Step 3: the routed experts as grouped GEMMs over expert-contiguous rows (tcgen05 / TMEM /
  * TMA).  gotburnout.io glossary, section 3 step 3 (the SwiGLU expert) and step 4 (outputs
  * multiplied by the router weights).

@@ -26,7 +26,8 @@ STATUS = {
 
 # every symbol include/moe_b200.h declares
 EXPORTS = (
-    "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_grouped_swiglu_ffn_workspace_size",
+    "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
+    "moe_grouped_swiglu_ffn_workspace_size",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_layer_workspace_size", "moe_layer_forward",
     "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_get_device_error",
     "moe_status_string",
@@ -64,6 +65,7 @@ def lib():
             "moe_router_topk": ([P, P, P, I, I, I, I, P, P, P], I),
             "moe_permute_workspace_size": ([I, I, I], Z),
             "moe_permute": ([P, P, P, I, I, I, I, P, P, P, P, P, P, P, Z, P], I),
+            "moe_permute_noalloc": ([P, P, P, I, I, I, I, P, P, P, P, P, P, P], I),
             "moe_grouped_swiglu_ffn_workspace_size": ([I, I], Z),
             "moe_grouped_swiglu_ffn": ([P, P, P, I, I, I, I, I, P, P, P, P, Z, P], I),
             "moe_combine": ([P, P, P, I, I, I, P, P], I),
@@ -152,6 +154,32 @@ def moe_permute(topk_idx, topk_w, x, E, stream=None, ws=None):
                              out["counts"].data_ptr(), out["offsets"].data_ptr(), out["perm_token"].data_ptr(),
                              out["inv_perm"].data_ptr(), out["p_perm"].data_ptr(), _ptr(out["x_perm"]),
                              ws.data_ptr(), ws.numel(), _stream(stream)), "moe_permute")
+    return out
+
+
+def moe_permute_noalloc(topk_idx, topk_w, x, E, out=None, stream=None):
+    """moe_permute for callers that cannot allocate device memory: the library keeps the
+    scratch in a fixed internal array.  ``out`` (optional) holds caller-provided output tensors
+    (keys as moe_permute's result); missing ones are created here by torch, not by the library."""
+    import torch
+
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    D = x.shape[1] if x is not None else 64
+    M = T * k
+    out = dict(out or {})
+    out.setdefault("counts", torch.empty(E, dtype=torch.int32, device=dev))
+    out.setdefault("offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    out.setdefault("perm_token", torch.empty(M, dtype=torch.int32, device=dev))
+    out.setdefault("inv_perm", torch.empty(M, dtype=torch.int32, device=dev))
+    out.setdefault("p_perm", torch.empty(M, dtype=torch.float32, device=dev))
+    if x is not None:
+        out.setdefault("x_perm", torch.empty(M, D, dtype=torch.bfloat16, device=dev))
+    _check(lib().moe_permute_noalloc(topk_idx.data_ptr(), topk_w.data_ptr(), _ptr(x), T, D, E, k,
+                                     out["counts"].data_ptr(), out["offsets"].data_ptr(),
+                                     out["perm_token"].data_ptr(), out["inv_perm"].data_ptr(),
+                                     out["p_perm"].data_ptr(), _ptr(out.get("x_perm")), _stream(stream)),
+           "moe_permute_noalloc")
     return out
 
 
