@@ -58,18 +58,23 @@ typedef enum {
 } moe_status_t;
 
 /* ----------------------------------------------------------------------------------------
- * Step 1: router projection + top-k + renormalised softmax (one fused kernel).
+ * Step 1: router projection + top-k + renormalised softmax.
  * josueisai.com "Mixture of experts", section "El router"; gotburnout.io glossary, section 2
  * (p = Softmax(TopK(W_g x))) and section 2 item 4 (aux-loss-free balancing bias).
  *
  *   x        [T, D]  bf16      w_gate [E, D] bf16      bias [E] fp32 or NULL
  *   topk_idx [T, k]  int32     out: expert ids, by (logit + bias) descending, ties -> lower id
  *   topk_w   [T, k]  fp32      out: exp(l_j - m) / sum_i exp(l_i - m) over the chosen k, with
- *                              the UNBIASED fp32 logits l (the bias only steers the selection)
+ *                              the UNBIASED logits l (the bias only steers the selection)
+ * The logits are bf16 x bf16 products accumulated in fp32 on the tensor cores (split over K in
+ * a fixed number of partial sums that the top-k kernel adds in a fixed order).
+ *   ws: >= moe_router_topk_workspace_size(T, D, E) bytes of device memory (first 256 bytes:
+ *       the device error word; the rest holds the partial logits).
  * ---------------------------------------------------------------------------------------- */
+size_t moe_router_topk_workspace_size(int T, int D, int E);
 moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, const float* bias, int T,
-                             int D, int E, int k, int32_t* topk_idx, float* topk_w,
-                             moe_stream_t stream);
+                             int D, int E, int k, int32_t* topk_idx, float* topk_w, void* ws,
+                             size_t ws_bytes, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
  * Step 2: dispatch -- histogram, exclusive prefix sum and permutation into expert-contiguous

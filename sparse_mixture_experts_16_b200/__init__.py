@@ -26,7 +26,7 @@ STATUS = {
 
 # every symbol include/moe_b200.h declares
 EXPORTS = (
-    "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
+    "moe_router_topk_workspace_size", "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
     "moe_grouped_swiglu_ffn_workspace_size",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_layer_workspace_size", "moe_layer_forward",
     "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_get_device_error",
@@ -62,7 +62,8 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         sig = {
-            "moe_router_topk": ([P, P, P, I, I, I, I, P, P, P], I),
+            "moe_router_topk_workspace_size": ([I, I, I], Z),
+            "moe_router_topk": ([P, P, P, I, I, I, I, P, P, P, Z, P], I),
             "moe_permute_workspace_size": ([I, I, I], Z),
             "moe_permute": ([P, P, P, I, I, I, I, P, P, P, P, P, P, P, Z, P], I),
             "moe_permute_noalloc": ([P, P, P, I, I, I, I, P, P, P, P, P, P, P], I),
@@ -109,7 +110,7 @@ def _need(t, dtype, shape, name):
 
 
 # ------------------------------------------------------------------------------ steps
-def moe_router_topk(x, w_gate, bias, k, topk_idx=None, topk_w=None, stream=None):
+def moe_router_topk(x, w_gate, bias, k, topk_idx=None, topk_w=None, ws=None, stream=None):
     """Router projection + top-k + softmax over the chosen k -> (topk_idx[T,k] int32, topk_w[T,k] fp32)."""
     import torch
 
@@ -123,8 +124,11 @@ def moe_router_topk(x, w_gate, bias, k, topk_idx=None, topk_w=None, stream=None)
         topk_idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    need = lib().moe_router_topk_workspace_size(T, D, E)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
     _check(lib().moe_router_topk(x.data_ptr(), w_gate.data_ptr(), _ptr(bias), T, D, E, k, topk_idx.data_ptr(),
-                                 topk_w.data_ptr(), _stream(stream)), "moe_router_topk")
+                                 topk_w.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)), "moe_router_topk")
     return topk_idx, topk_w
 
 

@@ -13,6 +13,8 @@
 // One kernel template, two GEMMs, two regimes:
 //   kGateUp : h[r, :]   = silu(A[r] G_e^T) * (A[r] U_e^T)             (SwiGLU in the epilogue)
 //   kDown   : out[r, :] = row_scale[r] * (h[r] Down_e^T)  in fp32       (router weight in epilogue)
+//   kRouter : logits[r, :] = x[r] W_g^T in fp32 (one group; split-K partial sums, reduced by the
+//             top-k kernel in a fixed order)
 //   tiled (prefill, NT = 0): a tile is 128 activation rows of one expert segment x 256 MMA
 //       columns (gate_up: 128 gate + 128 up weight rows, so both halves of a SwiGLU output land
 //       in the same TMEM lane; down: 256 weight rows).  MMA M=128, N=256, K=16.
@@ -55,6 +57,8 @@ struct alignas(64) GemmParams {
   int n_out[2];
   int w_rows[2];  // weight rows per group: 2F (gate_up) or D (down)
   int k_blocks[2];  // K / 64 per set (down: F routed, Fs shared)
+  int ld_out[2];    // row stride of the output (elements)
+  int k_splits;     // kRouter: K is split into this many contiguous k-block ranges
   int n_sets;
   int* err;
 };
@@ -63,6 +67,7 @@ template <int KIND, int NT>
 struct Cfg {
   static constexpr bool kTiled = (NT == 0);
   // shared-memory stage: [A (16 KB) | B ...]
+  // (kRouter is laid out like kDown: one weight operand)
   static constexpr int kStageBytes = kTiled ? (kTileBytesA + 256 * kBK * 2)
                                             : (KIND == kGateUp ? 2 * kTileBytesA + NT * kBK * 2
                                                                : kTileBytesA + NT * kBK * 2);
@@ -80,6 +85,7 @@ struct Cfg {
 
 struct Tile {
   int set, gl, row0, rows, m, n;
+  int ks, kb0, kb1;  // split index and k-block range [kb0, kb1)
 };
 
 __device__ __forceinline__ void group_rows(const GemmParams& p, int s, int gl, int& row0, int& rows) {
@@ -97,8 +103,9 @@ __device__ __forceinline__ int group_tiles(const GemmParams& p, int s, int rows)
   using C = Cfg<KIND, NT>;
   const int nt = (p.n_out[s] + C::kOutPerTile - 1) / C::kOutPerTile;
   if (rows <= 0) return 0;
-  if constexpr (C::kTiled) return ((rows + kBM - 1) / kBM) * nt;
-  return nt;
+  const int splits = KIND == kRouter ? p.k_splits : 1;
+  if constexpr (C::kTiled) return ((rows + kBM - 1) / kBM) * nt * splits;
+  return nt * splits;
 }
 
 template <int KIND, int NT>
@@ -112,7 +119,16 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, const int* tile
   ti.set = lo < p.n_groups[0] ? 0 : 1;
   ti.gl = ti.set == 0 ? lo : lo - p.n_groups[0];
   group_rows(p, ti.set, ti.gl, ti.row0, ti.rows);
-  const int local = t - tile_start[lo];
+  int local = t - tile_start[lo];
+  const int kbs = p.k_blocks[ti.set];
+  ti.ks = 0, ti.kb0 = 0, ti.kb1 = kbs;
+  if constexpr (KIND == kRouter) {
+    const int per = (kbs + p.k_splits - 1) / p.k_splits;
+    ti.ks = local % p.k_splits;
+    local /= p.k_splits;
+    ti.kb0 = ti.ks * per;
+    ti.kb1 = min(kbs, ti.kb0 + per);
+  }
   if constexpr (NT == 0) {
     const int mt = (ti.rows + kBM - 1) / kBM;
     ti.n = local / mt;
@@ -207,8 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const CUtensorMap* amap = &p.a_map[ti.set];
         const CUtensorMap* wmap = &p.w_map[ti.set];
         const int wbase = ti.gl * p.w_rows[ti.set];
-        const int kbs = p.k_blocks[ti.set];
-        for (int kb = 0; kb < kbs; ++kb, ++it) {
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++it) {
           const int stage = it % C::kStages;
           if (!mbar_wait(&empty[stage], ((it / C::kStages) & 1) ^ 1, kWaitLimitNs)) {
             ok = false;
@@ -261,8 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         }
         tc_fence_after();
         const uint32_t d = tmem_base + buf * C::kAccCols;
-        const int kbs = p.k_blocks[decode_tile<KIND, NT>(p, tile_start, G, t).set];
-        for (int kb = 0; kb < kbs; ++kb, ++it) {
+        const Tile ti = decode_tile<KIND, NT>(p, tile_start, G, t);
+        for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++it) {
           const int stage = it % C::kStages;
           if (!mbar_wait(&full[stage], (it / C::kStages) & 1, kWaitLimitNs)) {
             ok = false;
@@ -272,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
           const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint32_t acc = (kb | kk) != 0;
+            const uint32_t acc = (kb > ti.kb0 || kk > 0) ? 1u : 0u;
             if constexpr (C::kTiled) {
               umma_bf16(d, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sa + kTileBytesA + kk * 32),
                         C::kIdesc, acc);
@@ -337,6 +352,25 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
               for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
             }
           }
+        } else if constexpr (KIND == kRouter) {
+          // partial logits of split ks: out[ks][row][col], row stride ld (a multiple of 32)
+          const int ld = p.ld_out[ti.set];
+          float* orow = out_f + ((size_t)ti.ks * p.m_rows[ti.set] + grow) * ld;
+#pragma unroll 1
+          for (int c0 = 0; c0 < 256; c0 += 32) {
+            const int col = ti.n * 256 + c0;
+            if (col >= n_out) break;
+            uint32_t a[32];
+            tmem_ld_32x32b_x32(tacc + c0, a);
+            tmem_ld_wait();
+            if (row_ok) {
+              float4* dst = reinterpret_cast<float4*>(orow + col);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
+                                     __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
+            }
+          }
         } else {
           const float sc = (row_ok && p.row_scale[ti.set] != nullptr) ? p.row_scale[ti.set][grow] : 1.0f;
 #pragma unroll 1
@@ -374,6 +408,17 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                 const float h = silu_mul(__uint_as_float(g[jj]), __uint_as_float(u[jj]));
                 out_h[(size_t)(ti.row0 + j) * n_out + col] = (uint16_t)(pack_bf16x2(h, 0.f) & 0xFFFFu);
               }
+            }
+          } else if constexpr (KIND == kRouter) {
+            uint32_t a[16];
+            tmem_ld_32x32b_x16(tacc + j0, a);
+            tmem_ld_wait();
+            const int ld = p.ld_out[ti.set];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = j0 + jj;
+              if (j < ti.rows && col_ok)
+                out_f[((size_t)ti.ks * p.m_rows[ti.set] + ti.row0 + j) * ld + col] = __uint_as_float(a[jj]);
             }
           } else {
             uint32_t a[16];
@@ -447,14 +492,15 @@ int num_sms() {
 }
 
 template <int KIND, int NT>
-cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int* err, cudaStream_t s) {
+cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int* err, cudaStream_t s) {
   using C = Cfg<KIND, NT>;
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.n_sets = n_sets;
+  p.k_splits = k_splits;
   p.err = err;
   const uint32_t a_box = C::kTiled ? kBM : NT;
-  const uint32_t w_box = (C::kTiled && KIND == kDown) ? 256 : 128;
+  const uint32_t w_box = (C::kTiled && KIND != kGateUp) ? 256 : 128;
   for (int i = 0; i < n_sets; ++i) {
     const GemmSetHost& st = sets[i];
     const int K = st.K;
@@ -466,6 +512,7 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int* err, cudaStr
     p.offsets[i] = st.offsets;
     p.out[i] = st.out;
     p.row_scale[i] = st.row_scale;
+    p.ld_out[i] = st.ld_out > 0 ? st.ld_out : st.n_out;
     p.n_groups[i] = st.n_groups;
     p.m_rows[i] = st.m_rows;
     p.n_out[i] = st.n_out;
@@ -494,22 +541,50 @@ cudaError_t launch_grouped_gemm(GemmKind kind, const GemmSetHost* sets, int n_se
   if (groups > kMaxGroups) return cudaErrorInvalidValue;
   if (kind == kGateUp) {
     switch (decode_nt) {
-      case 0: return launch_kernel<kGateUp, 0>(sets, n_sets, err, s);
-      case 16: return launch_kernel<kGateUp, 16>(sets, n_sets, err, s);
-      case 32: return launch_kernel<kGateUp, 32>(sets, n_sets, err, s);
-      case 48: return launch_kernel<kGateUp, 48>(sets, n_sets, err, s);
-      case 64: return launch_kernel<kGateUp, 64>(sets, n_sets, err, s);
+      case 0: return launch_kernel<kGateUp, 0>(sets, n_sets, 1, err, s);
+      case 16: return launch_kernel<kGateUp, 16>(sets, n_sets, 1, err, s);
+      case 32: return launch_kernel<kGateUp, 32>(sets, n_sets, 1, err, s);
+      case 48: return launch_kernel<kGateUp, 48>(sets, n_sets, 1, err, s);
+      case 64: return launch_kernel<kGateUp, 64>(sets, n_sets, 1, err, s);
     }
   } else {
     switch (decode_nt) {
-      case 0: return launch_kernel<kDown, 0>(sets, n_sets, err, s);
-      case 16: return launch_kernel<kDown, 16>(sets, n_sets, err, s);
-      case 32: return launch_kernel<kDown, 32>(sets, n_sets, err, s);
-      case 48: return launch_kernel<kDown, 48>(sets, n_sets, err, s);
-      case 64: return launch_kernel<kDown, 64>(sets, n_sets, err, s);
+      case 0: return launch_kernel<kDown, 0>(sets, n_sets, 1, err, s);
+      case 16: return launch_kernel<kDown, 16>(sets, n_sets, 1, err, s);
+      case 32: return launch_kernel<kDown, 32>(sets, n_sets, 1, err, s);
+      case 48: return launch_kernel<kDown, 48>(sets, n_sets, 1, err, s);
+      case 64: return launch_kernel<kDown, 64>(sets, n_sets, 1, err, s);
     }
   }
   return cudaErrorInvalidValue;
+}
+
+int router_k_splits(int T, int D, int E, int num_sm) {
+  const int kbs = D / kBK;
+  const long long base = T <= 64 ? (E + 127) / 128 : (long long)((T + kBM - 1) / kBM) * ((E + 255) / 256);
+  long long want = (num_sm + base - 1) / base;  // enough tiles to give every SM one
+  if (want < 1) want = 1;
+  if (want > kbs) want = kbs;
+  const int per = (int)((kbs + want - 1) / want);
+  return (kbs + per - 1) / per;  // every split non-empty
+}
+
+int router_k_splits(int T, int D, int E) { return router_k_splits(T, D, E, num_sms()); }
+
+cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wg, int T, int D, int E, float* partials, int ld,
+                               int k_splits, int* err, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  GemmSetHost st;
+  memset(&st, 0, sizeof(st));
+  st.K = D, st.a = x, st.a_rows = T, st.w = wg, st.n_groups = 1, st.offsets = nullptr, st.m_rows = T;
+  st.n_out = E, st.out = partials, st.row_scale = nullptr, st.ld_out = ld;
+  if (T > 64) return launch_kernel<kRouter, 0>(&st, 1, k_splits, err, s);
+  switch ((T + 15) / 16 * 16) {
+    case 16: return launch_kernel<kRouter, 16>(&st, 1, k_splits, err, s);
+    case 32: return launch_kernel<kRouter, 32>(&st, 1, k_splits, err, s);
+    case 48: return launch_kernel<kRouter, 48>(&st, 1, k_splits, err, s);
+    default: return launch_kernel<kRouter, 64>(&st, 1, k_splits, err, s);
+  }
 }
 
 }  // namespace moe

@@ -34,8 +34,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ---- host launchers (defined in the .cu files) ---------------------------------------------
-cudaError_t launch_router_topk(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int D, int E,
-                               int k, int32_t* idx, float* w, int* err_to_clear, cudaStream_t s);
+// Router: logits on the tensor cores (split-K partial sums, [k_splits][T][ld] fp32, ld = E rounded
+// up to 32), then a warp-level top-k + softmax kernel that reduces the splits in a fixed order.
+int router_k_splits(int T, int D, int E);
+inline int router_ld(int E) { return (E + 31) / 32 * 32; }
+inline size_t router_scratch_bytes(int T, int D, int E) {
+  return align_up((size_t)router_k_splits(T, D, E) * (size_t)T * router_ld(E) * sizeof(float), 256);
+}
+cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wg, int T, int D, int E, float* partials, int ld,
+                               int k_splits, int* err, cudaStream_t s);
+cudaError_t launch_router_select(const float* partials, int k_splits, int T, int ld, const float* bias, int E, int k,
+                                 int32_t* idx, float* w, cudaStream_t s);
 
 size_t permute_scratch_bytes(int T, int E);
 cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16_t* x, int T, int D, int E,
@@ -59,9 +68,10 @@ struct GemmSetHost {
   int n_out;                // output columns (F for gate_up -> h, D for down)
   void* out;                // [rows, n_out]: bf16 (gate_up -> h) or fp32 (down)
   const float* row_scale;   // per-row factor (down) or NULL
+  int ld_out;               // output row stride in elements (0: n_out)
 };
 
-enum GemmKind { kGateUp = 0, kDown = 1 };
+enum GemmKind { kGateUp = 0, kDown = 1, kRouter = 2 };
 
 // Launch one grouped GEMM (gate_up + SwiGLU, or down + row scale) over up to two sets.
 // decode_nt > 0 selects the weight-streaming

@@ -39,7 +39,7 @@ moe_status_t shape_status(long long T, long long D, long long E, long long k) {
 }
 
 struct LayerWs {
-  size_t topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
+  size_t router, topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
       out_sh, x_stage, y_stage, total;
 };
 
@@ -52,6 +52,7 @@ LayerWs layer_ws(const moe_layer_desc_t& d) {
     return at;
   };
   const size_t T = d.T, D = d.D, E = d.E, k = d.k, F = d.F, Fs = d.Fs, M = T * k;
+  w.router = take(router_scratch_bytes(d.T, d.D, d.E));
   w.topk_idx = take(M * 4);
   w.topk_w = take(M * 4);
   w.scratch = take(permute_scratch_bytes(d.T, d.E));
@@ -166,7 +167,11 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
   auto record = [&](cudaEvent_t e) { return cudaEventRecordWithFlags(e, s, rec_flags); };
 
   if (ev) MOE_CUDA_TRY(record(ev[0]));
-  MOE_CUDA_TRY(launch_router_topk(x, d->w_gate, d->bias, T, D, E, k, I(w.topk_idx), Fp(w.topk_w), err, s));
+  MOE_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));  // a fresh error word for this forward
+  const int splits = router_k_splits(T, D, E);
+  MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s));
+  MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
+                                    Fp(w.topk_w), s));
   if (ev) MOE_CUDA_TRY(record(ev[1]));
   MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), x, T, D, E, k, I(w.counts), I(w.offsets),
                               I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), H(w.x_perm), I(w.scratch), err, s,
@@ -202,16 +207,29 @@ const char* moe_status_string(moe_status_t status) {
   return "MOE_ERR_UNKNOWN";
 }
 
+size_t moe_router_topk_workspace_size(int T, int D, int E) {
+  if (shape_status(T, D, E, 1) != MOE_OK) return 0;
+  return kWsHeader + router_scratch_bytes(T, D, E);
+}
+
 moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, const float* bias, int T, int D, int E,
-                             int k, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+                             int k, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
   moe_status_t st = shape_status(T, D, E, k);
   if (st != MOE_OK) return st;
-  if (!x || !w_gate || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(w_gate, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+  if (!x || !w_gate || !topk_idx || !topk_w || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_gate, 16) || !aligned(bias, 4) || !aligned(topk_idx, 4) ||
+      !aligned(topk_w, 4) || !aligned(ws, 256))
     return MOE_ERR_ALIGNMENT;
+  if (ws_bytes < moe_router_topk_workspace_size(T, D, E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if ((st = check_device()) != MOE_OK) return st;
   if (T == 0) return MOE_OK;
-  MOE_CUDA_TRY(launch_router_topk(x, w_gate, bias, T, D, E, k, topk_idx, topk_w, nullptr, (cudaStream_t)stream));
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  float* part = reinterpret_cast<float*>(b + kWsHeader);
+  const int splits = router_k_splits(T, D, E);
+  cudaStream_t s = (cudaStream_t)stream;
+  MOE_CUDA_TRY(launch_router_gemm(x, w_gate, T, D, E, part, router_ld(E), splits, reinterpret_cast<int*>(b), s));
+  MOE_CUDA_TRY(launch_router_select(part, splits, T, router_ld(E), bias, E, k, topk_idx, topk_w, s));
   return MOE_OK;
 }
 
@@ -322,7 +340,7 @@ moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16
 
 int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  return 1 /*router*/ + 4 /*hist, scan, scatter, gather*/ + 2 /*grouped GEMMs*/ + 1 /*combine*/;
+  return 2 /*router GEMM, top-k*/ + 4 /*hist, scan, scatter, gather*/ + 2 /*grouped GEMMs*/ + 1 /*combine*/;
 }
 
 moe_status_t moe_get_device_error(void* ws, moe_stream_t stream) {

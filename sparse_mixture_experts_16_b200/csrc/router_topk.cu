@@ -1,16 +1,15 @@
-// router_topk.cu -- step 1 of the layer: router projection, top-k, softmax over the chosen k.
+// router_topk.cu -- step 1 of the layer, second half: top-k and softmax over the chosen k.
 //
 // josueisai.com "Mixture of experts", section "El router": a linear projection gives one score
 // per expert, the k best are kept and the softmax is normalised over those k only.
 // gotburnout.io glossary "MoE", section 2 item 4: a per-expert bias (aux-loss-free balancing)
 // steers the selection; it is added to the scores for choosing, not to the weights.
 //
-// One fused kernel.  A block owns TT = 8*RT tokens and all E experts.  The D axis is walked in
-// chunks of 32: the chunk of W_g (E x 32) and of x (TT x 32) is converted to fp32 in shared
-// memory, W_g transposed so each lane reads its EJ consecutive experts with vector loads.  Each
-// warp owns RT tokens; lane l accumulates experts [l*EJ, l*EJ + EJ) in fp32 registers.  Top-k is
-// then a k-round warp arg-max over those registers (ties -> lower expert id), and the k chosen
-// unbiased logits are normalised with expf in fp32.
+// The projection itself (logits = x W_g^T, bf16 products accumulated in fp32) runs on the
+// tensor cores in grouped_gemm_sm100.cu and leaves k_splits partial sums [k_splits][T][ld].
+// Here one warp owns one token: lane l sums the partials of experts [l*EJ, l*EJ + EJ) in split
+// order (deterministic), then k rounds of a warp arg-max over (logit + bias) pick the experts
+// (ties -> lower expert id), and the chosen unbiased logits are normalised with expf in fp32.
 #include <cfloat>
 #include <climits>
 
@@ -19,94 +18,37 @@
 namespace moe {
 namespace {
 
-constexpr int kDC = 32;       // D chunk
-constexpr int kThreads = 256; // 8 warps
+constexpr int kThreads = 256;  // 8 tokens per block
 
 template <int EJ>
-__device__ __forceinline__ void load_row(const float* p, float (&w)[EJ]) {
-  if constexpr (EJ % 4 == 0) {
-#pragma unroll
-    for (int q = 0; q < EJ / 4; ++q) {
-      float4 v = reinterpret_cast<const float4*>(p)[q];
-      w[4 * q] = v.x, w[4 * q + 1] = v.y, w[4 * q + 2] = v.z, w[4 * q + 3] = v.w;
-    }
-  } else if constexpr (EJ == 2) {
-    float2 v = *reinterpret_cast<const float2*>(p);
-    w[0] = v.x, w[1] = v.y;
-  } else {
-    w[0] = p[0];
-  }
-}
-
-template <int EJ, int RT>
-__global__ void __launch_bounds__(kThreads) router_topk_kernel(const uint16_t* __restrict__ x,
-                                                               const uint16_t* __restrict__ wg,
-                                                               const float* __restrict__ bias, int T, int D,
-                                                               int E, int k, int32_t* __restrict__ idx_out,
-                                                               float* __restrict__ w_out, int* err_clear) {
-  constexpr int EP = 32 * EJ;  // padded expert count
-  constexpr int TT = 8 * RT;   // tokens per block
-  extern __shared__ __align__(16) float sm[];
-  float* ws = sm;              // [kDC][EP]   (W_g chunk, transposed)
-  float* xs = sm + kDC * EP;   // [TT][kDC]
-
-  if (err_clear != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_clear = 0;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * TT;
-
-  float acc[RT][EJ];
-#pragma unroll
-  for (int r = 0; r < RT; ++r)
-#pragma unroll
-    for (int j = 0; j < EJ; ++j) acc[r][j] = 0.f;
-
-  for (int d0 = 0; d0 < D; d0 += kDC) {
-    for (int v = threadIdx.x; v < EP * 4; v += kThreads) {
-      const int e = v >> 2, c = (v & 3) * 8;
-      uint4 q = make_uint4(0, 0, 0, 0);
-      if (e < E) q = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)e * D + d0 + c));
-      const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        ws[(c + 2 * i) * EP + e] = bf16_lo(w4[i]);
-        ws[(c + 2 * i + 1) * EP + e] = bf16_hi(w4[i]);
-      }
-    }
-    for (int v = threadIdx.x; v < TT * 4; v += kThreads) {
-      const int r = v >> 2, c = (v & 3) * 8, t = t0 + r;
-      uint4 q = make_uint4(0, 0, 0, 0);
-      if (t < T) q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * D + d0 + c));
-      float4* dst = reinterpret_cast<float4*>(xs + r * kDC + c);
-      dst[0] = make_float4(bf16_lo(q.x), bf16_hi(q.x), bf16_lo(q.y), bf16_hi(q.y));
-      dst[1] = make_float4(bf16_lo(q.z), bf16_hi(q.z), bf16_lo(q.w), bf16_hi(q.w));
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kDC; ++kk) {
-      float xv[RT], wv[EJ];
-#pragma unroll
-      for (int r = 0; r < RT; ++r) xv[r] = xs[(warp * RT + r) * kDC + kk];
-      load_row<EJ>(ws + kk * EP + lane * EJ, wv);
-#pragma unroll
-      for (int r = 0; r < RT; ++r)
-#pragma unroll
-        for (int j = 0; j < EJ; ++j) acc[r][j] = fmaf(xv[r], wv[j], acc[r][j]);
-    }
-    __syncthreads();
-  }
-
+__global__ void __launch_bounds__(kThreads) router_select_kernel(const float* __restrict__ part, int S, int T, int ld,
+                                                                 const float* __restrict__ bias, int E, int k,
+                                                                 int32_t* __restrict__ idx_out,
+                                                                 float* __restrict__ w_out) {
+  const int lane = threadIdx.x & 31;
+  const int e0 = lane * EJ;
   float bj[EJ];
 #pragma unroll
-  for (int j = 0; j < EJ; ++j) {
-    const int e = lane * EJ + j;
-    bj[j] = (bias != nullptr && e < E) ? bias[e] : 0.f;
-  }
+  for (int j = 0; j < EJ; ++j) bj[j] = (bias != nullptr && e0 + j < E) ? bias[e0 + j] : 0.f;
 
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += (gridDim.x * blockDim.x) >> 5) {
+    float l[EJ];
 #pragma unroll
-  for (int r = 0; r < RT; ++r) {
-    const int t = t0 + warp * RT + r;
-    if (t >= T) break;  // warp-uniform
+    for (int j = 0; j < EJ; ++j) l[j] = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float* row = part + ((size_t)s * T + t) * ld + e0;
+      if (EJ % 4 == 0 && e0 + EJ <= E) {
+#pragma unroll
+        for (int q = 0; q < EJ / 4; ++q) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(row) + q);
+          l[4 * q] += v.x, l[4 * q + 1] += v.y, l[4 * q + 2] += v.z, l[4 * q + 3] += v.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < EJ; ++j)
+          if (e0 + j < E) l[j] += __ldg(row + j);
+      }
+    }
     uint32_t taken = 0;
     int my_idx = -1;
     float my_l = 0.f;
@@ -116,9 +58,9 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(const uint16_t* _
       int be = INT_MAX;
 #pragma unroll
       for (int jj = 0; jj < EJ; ++jj) {
-        const int e = lane * EJ + jj;
-        const float sv = acc[r][jj] + bj[jj];
-        if (e < E && !((taken >> jj) & 1u) && (be == INT_MAX || sv > bv)) bv = sv, be = e, bl = acc[r][jj];
+        const int e = e0 + jj;
+        const float sv = l[jj] + bj[jj];
+        if (e < E && !((taken >> jj) & 1u) && (be == INT_MAX || sv > bv)) bv = sv, be = e, bl = l[jj];
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
@@ -144,37 +86,26 @@ __global__ void __launch_bounds__(kThreads) router_topk_kernel(const uint16_t* _
   }
 }
 
-template <int EJ, int RT>
-cudaError_t launch(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int D, int E, int k,
-                   int32_t* idx, float* w, int* err_clear, cudaStream_t s) {
-  constexpr int TT = 8 * RT;
-  const size_t smem = (size_t)(kDC * 32 * EJ + TT * kDC) * sizeof(float);
-  static bool configured = false;  // idempotent attribute set
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(router_topk_kernel<EJ, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  const int blocks = (T + TT - 1) / TT;
-  router_topk_kernel<EJ, RT><<<blocks, kThreads, smem, s>>>(x, wg, bias, T, D, E, k, idx, w, err_clear);
+template <int EJ>
+cudaError_t launch(const float* part, int S, int T, int ld, const float* bias, int E, int k, int32_t* idx, float* w,
+                   cudaStream_t s) {
+  long long blocks = ((long long)T + 7) / 8;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  router_select_kernel<EJ><<<(unsigned)blocks, kThreads, 0, s>>>(part, S, T, ld, bias, E, k, idx, w);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_router_topk(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int D, int E,
-                               int k, int32_t* idx, float* w, int* err_clear, cudaStream_t s) {
-  if (T == 0) {
-    if (err_clear) return cudaMemsetAsync(err_clear, 0, sizeof(int), s);
-    return cudaSuccess;
-  }
-  if (E <= 32) return launch<1, 4>(x, wg, bias, T, D, E, k, idx, w, err_clear, s);
-  if (E <= 64) return launch<2, 4>(x, wg, bias, T, D, E, k, idx, w, err_clear, s);
-  if (E <= 128) return launch<4, 4>(x, wg, bias, T, D, E, k, idx, w, err_clear, s);
-  if (E <= 256) return launch<8, 4>(x, wg, bias, T, D, E, k, idx, w, err_clear, s);
-  if (E <= 512) return launch<16, 2>(x, wg, bias, T, D, E, k, idx, w, err_clear, s);
-  return launch<32, 1>(x, wg, bias, T, D, E, k, idx, w, err_clear, s);
+cudaError_t launch_router_select(const float* partials, int k_splits, int T, int ld, const float* bias, int E, int k,
+                                 int32_t* idx, float* w, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  if (E <= 32) return launch<1>(partials, k_splits, T, ld, bias, E, k, idx, w, s);
+  if (E <= 64) return launch<2>(partials, k_splits, T, ld, bias, E, k, idx, w, s);
+  if (E <= 128) return launch<4>(partials, k_splits, T, ld, bias, E, k, idx, w, s);
+  if (E <= 256) return launch<8>(partials, k_splits, T, ld, bias, E, k, idx, w, s);
+  if (E <= 512) return launch<16>(partials, k_splits, T, ld, bias, E, k, idx, w, s);
+  return launch<32>(partials, k_splits, T, ld, bias, E, k, idx, w, s);
 }
 
 }  // namespace moe

@@ -80,7 +80,7 @@ def test_layer_workspace_size_and_small_workspace(L):
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, need - 1, None) == 4
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100010, need, None) == 3  # ws not 256-aligned
     assert L.moe_layer_forward(ctypes.byref(d), 0x4008, 0x5000, 0x100000, need, None) == 3
-    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 8
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 9
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(k=9))) == 0
     # shared expert grows the workspace
     d2 = _desc(Fs=256, shared_gate_up=0x6000, shared_down=0x7000)
@@ -89,10 +89,13 @@ def test_layer_workspace_size_and_small_workspace(L):
 
 def test_step_entry_points_validate_on_host(L):
     # router: k > E, D not multiple of 64, misaligned x
-    assert L.moe_router_topk(0x1000, 0x2000, None, 4, 128, 4, 5, 0x3000, 0x4000, None) == 1
-    assert L.moe_router_topk(0x1000, 0x2000, None, 4, 100, 4, 2, 0x3000, 0x4000, None) == 2
-    assert L.moe_router_topk(0x1001, 0x2000, None, 4, 128, 4, 2, 0x3000, 0x4000, None) == 3
-    assert L.moe_router_topk(None, 0x2000, None, 4, 128, 4, 2, 0x3000, 0x4000, None) == 1
+    rws = L.moe_router_topk_workspace_size(4, 128, 4)
+    assert rws >= 256 + 4 * 32 * 4
+    assert L.moe_router_topk(0x1000, 0x2000, None, 4, 128, 4, 5, 0x3000, 0x4000, 0x100000, rws, None) == 1
+    assert L.moe_router_topk(0x1000, 0x2000, None, 4, 100, 4, 2, 0x3000, 0x4000, 0x100000, rws, None) == 2
+    assert L.moe_router_topk(0x1001, 0x2000, None, 4, 128, 4, 2, 0x3000, 0x4000, 0x100000, rws, None) == 3
+    assert L.moe_router_topk(None, 0x2000, None, 4, 128, 4, 2, 0x3000, 0x4000, 0x100000, rws, None) == 1
+    assert L.moe_router_topk(0x1000, 0x2000, None, 4, 128, 4, 2, 0x3000, 0x4000, 0x100000, rws - 1, None) == 4
     # permute: workspace too small, x without x_perm
     need = L.moe_permute_workspace_size(300, 8, 2)
     assert need >= 256 + 2 * 8 * 4
