@@ -31,6 +31,7 @@
 // own in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -60,6 +61,7 @@ struct alignas(64) GemmParams {
   int ld_out[2];    // row stride of the output (elements)
   int k_splits;     // kRouter: K is split into this many contiguous k-block ranges
   int n_sets;
+  int withhold_first_load;  // test only: never issue the first stage's copies (its wait then times out)
   int* err;
 };
 
@@ -231,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
           }
           uint8_t* sb = smem + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          if (p.withhold_first_load && it == 0) continue;  // the bytes never arrive
           const int kx = kb * kBK;
           if constexpr (C::kTiled) {
             tma_load_2d(amap, &full[stage], sb, kx, ti.row0 + ti.m * kBM);
@@ -499,6 +502,10 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int
   p.n_sets = n_sets;
   p.k_splits = k_splits;
   p.err = err;
+  // Fault-path test hook: with MOE_TEST_WITHHOLD_LOAD=1 the producer skips its first copies, so
+  // the consumers' bounded waits expire and the kernel reports MOE_ERR_TIMEOUT and returns.
+  const char* hold = getenv("MOE_TEST_WITHHOLD_LOAD");
+  p.withhold_first_load = (hold != nullptr && hold[0] == '1') ? 1 : 0;
   const uint32_t a_box = C::kTiled ? kBM : NT;
   const uint32_t w_box = (C::kTiled && KIND != kGateUp) ? 256 : 128;
   for (int i = 0; i < n_sets; ++i) {
