@@ -17,12 +17,16 @@
 //             top-k kernel in a fixed order)
 //   tiled (prefill, NT = 0): a tile is 128 activation rows of one expert segment x 256 MMA
 //       columns (gate_up: 128 gate + 128 up weight rows, so both halves of a SwiGLU output land
-//       in the same TMEM lane; down: 256 weight rows).  MMA M=128, N=256, K=16.
+//       in the same TMEM lane; down: 256 weight rows).  MMA M=128, N=256, K=16.  The last tile
+//       of a segment computes up to 127 padding rows, which are never stored.
 //   streaming (decode, NT > 0): swap-AB.  A unit is 128 weight rows of one active expert (two
 //       accumulators for gate_up) x the <= NT tokens routed to it, MMA M=128, N=NT.  Each active
 //       expert's weights are read exactly once.
 // Grid: one persistent CTA per SM walks a static round-robin list of tiles built on the device
-// from the segment offsets (no host synchronisation).  Warp roles per CTA:
+// from the segment offsets (no host synchronisation).  Tiles are uniform (128 rows x 256
+// columns x K), so CTAs b, b+1, ... stay in step on the m-tiles of one weight tile and share it
+// through L2; the two SMs of a TPC, which take consecutive CTAs, even merge their requests for
+// it.  Warp roles per CTA:
 //   warp 0 (one lane)  : TMA producer, multi-stage ring of shared-memory stages (mbarrier full/empty)
 //   warp 1 (one lane)  : tcgen05.mma issuer; commits free a stage / publish an accumulator
 //   warps 2-5          : epilogue; tcgen05.ld of their 32-lane quarter of TMEM, math, global stores
@@ -46,6 +50,7 @@ constexpr int kBK = 64;             // K per stage (one 128-byte swizzle row of 
 constexpr int kThreads = 192;       // 6 warps
 constexpr int kMaxGroups = 1025;    // E <= 1024 routed + 1 shared
 constexpr int kTileBytesA = kBM * kBK * 2;  // 16 KB
+constexpr int kBarBytes = 256;      // mbarriers and the TMEM address slot
 
 struct alignas(64) GemmParams {
   CUtensorMap a_map[2];  // activations per set (box rows: 128 tiled / NT streaming)
@@ -80,7 +85,7 @@ struct Cfg {
   static constexpr int kOutPerTile = kTiled ? (KIND == kGateUp ? 128 : 256) : 128;
   static constexpr uint32_t kIdesc = kTiled ? idesc_bf16_f32(kBM, 256) : idesc_bf16_f32(kBM, NT);
   static constexpr size_t kSmemBytes =
-      1024 /*alignment slack*/ + (size_t)kStages * kStageBytes + 256 /*barriers*/ + 4 * (kMaxGroups + 1);
+      1024 /*alignment slack*/ + (size_t)kStages * kStageBytes + kBarBytes + 4 * (kMaxGroups + 1);
   static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -154,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
   uint64_t* acc_full = empty + C::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  int* tile_start = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + 256);
+  int* tile_start = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.n_groups[0] + (p.n_sets > 1 ? p.n_groups[1] : 0);
@@ -180,6 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
+  // everything above overlaps the previous kernel; the offsets and operands are its outputs
+  pdl_wait();
+  pdl_trigger();
   // per-group tile counts, then an exclusive scan (warp 0) -> tile_start[0..G]
   for (int g = threadIdx.x; g < G; g += kThreads) {
     const int s = g < p.n_groups[0] ? 0 : 1;
@@ -531,8 +539,7 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  grouped_gemm_kernel<KIND, NT><<<num_sms(), kThreads, C::kSmemBytes, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<KIND, NT>, dim3(num_sms()), dim3(kThreads), C::kSmemBytes, s, p);
 }
 
 }  // namespace
@@ -570,6 +577,7 @@ int router_k_splits(int T, int D, int E, int num_sm) {
   const int kbs = D / kBK;
   const long long base = T <= 64 ? (E + 127) / 128 : (long long)((T + kBM - 1) / kBM) * ((E + 255) / 256);
   long long want = (num_sm + base - 1) / base;  // enough tiles to give every SM one
+  if (want > 16) want = 16;                      // bounds the partial sums the top-k kernel adds
   if (want < 1) want = 1;
   if (want > kbs) want = kbs;
   const int per = (int)((kbs + want - 1) / want);

@@ -33,6 +33,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// ---- programmatic dependent launch --------------------------------------------------------------
+// Every kernel of the layer is launched with programmatic stream serialisation: it may start (and
+// run its prologue) while the previous kernel drains.  Each kernel executes pdl_wait() before it
+// reads anything an earlier kernel (or the caller) wrote, and pdl_trigger() once its own
+// dependents may be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---- host launchers (defined in the .cu files) ---------------------------------------------
 // Router: logits on the tensor cores (split-K partial sums, [k_splits][T][ld] fp32, ld = E rounded
 // up to 32), then a warp-level top-k + softmax kernel that reduces the splits in a fixed order.

@@ -340,7 +340,8 @@ moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16
 
 int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  return 2 /*router GEMM, top-k*/ + 4 /*hist, scan, scatter, gather*/ + 2 /*grouped GEMMs*/ + 1 /*combine*/;
+  const int dispatch = desc->T <= 256 ? 1 /*fused hist+scan+scatter*/ : 3 /*hist, scan, scatter*/;
+  return 2 /*router GEMM, top-k*/ + dispatch + 1 /*gather*/ + 2 /*grouped GEMMs*/ + 1 /*combine*/;
 }
 
 moe_status_t moe_get_device_error(void* ws, moe_stream_t stream) {

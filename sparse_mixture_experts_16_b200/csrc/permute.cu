@@ -11,6 +11,7 @@
 //                equal experts inside each 32-slot step come from __match_any_sync + popc, and
 //                a shared running counter per expert carries them across steps
 //   4. gather  : x_perm[r] = x[perm_token[r]], one warp per row, 16-byte vector moves
+// For T <= 256 steps 1-3 run as one single-block kernel (dispatch_small_kernel).
 // Within an expert, rows are therefore ordered by token id (a token picks an expert at most once).
 #include "moe_common.cuh"
 
@@ -23,6 +24,7 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
                                                    int32_t* __restrict__ block_counts, int* err) {
   extern __shared__ int cnt[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  pdl_wait();
   __syncthreads();
   const int t0 = blockIdx.x * kTokPerBlock;
   const int n_items = min(T - t0, kTokPerBlock) * k;
@@ -36,6 +38,7 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) block_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+  pdl_trigger();
 }
 
 // One block of 1024 threads.  block_counts[b][e] becomes the exclusive prefix over blocks.
@@ -44,6 +47,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
   __shared__ int32_t warp_tot[32];
   const int e = threadIdx.x;  // E <= 1024
   int total = 0;
+  pdl_wait();
   if (e < E) {
     for (int b = 0; b < nb; ++b) {
       const int v = block_counts[(size_t)b * E + e];
@@ -75,6 +79,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
   if (warp > 0) incl += warp_tot[warp - 1];
   if (e < E) offsets[e + 1] = incl;
   if (e == 0) offsets[0] = 0;
+  pdl_trigger();
 }
 
 // One warp per block of 256 tokens; order-preserving ranks.
@@ -85,6 +90,7 @@ __global__ void __launch_bounds__(32) scatter_kernel(const int32_t* __restrict__
                                                      float* __restrict__ p_perm) {
   extern __shared__ int run[];  // next free row per expert
   const int lane = threadIdx.x;
+  pdl_wait();
   for (int e = lane; e < E; e += 32) run[e] = offsets[e] + block_off[(size_t)blockIdx.x * E + e];
   __syncwarp();
   const int t0 = blockIdx.x * kTokPerBlock;
@@ -113,6 +119,84 @@ __global__ void __launch_bounds__(32) scatter_kernel(const int32_t* __restrict__
     if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
     __syncwarp();
   }
+  pdl_trigger();
+}
+
+// T <= 256 (one counting block): histogram, scan and the order-preserving scatter in one block of
+// 256 threads -- the same three steps as above without two launches and the per-block scratch.
+__global__ void __launch_bounds__(256) dispatch_small_kernel(const int32_t* __restrict__ idx,
+                                                             const float* __restrict__ w, int T, int E, int k,
+                                                             int32_t* __restrict__ counts,
+                                                             int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ perm_token,
+                                                             int32_t* __restrict__ inv_perm,
+                                                             float* __restrict__ p_perm, int* err) {
+  extern __shared__ int sm[];
+  int* cnt = sm;       // [E] counts
+  int* run = sm + E;   // [E] next free row per expert
+  __shared__ int warp_tot[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < E; e += 256) cnt[e] = 0;
+  pdl_wait();
+  __syncthreads();
+  const int n_items = T * k;
+  for (int i = tid; i < n_items; i += 256) {
+    const int e = idx[i];
+    if ((unsigned)e < (unsigned)E)
+      atomicAdd(&cnt[e], 1);
+    else
+      set_error(err, kErrBadIndex);
+  }
+  __syncthreads();
+  // exclusive scan over experts: thread tid owns experts [tid*per, tid*per + per)
+  const int per = (E + 255) / 256;
+  const int lo = min(E, tid * per), hi = min(E, lo + per);
+  int sum = 0;
+  for (int e = lo; e < hi; ++e) sum += cnt[e];
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int q = 0; q < warp; ++q) before += warp_tot[q];
+  int r0 = before + incl - sum;
+  for (int e = lo; e < hi; ++e) {
+    counts[e] = cnt[e];
+    offsets[e] = r0;
+    run[e] = r0;
+    r0 += cnt[e];
+  }
+  if (tid == 255) offsets[E] = before + incl;
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int i0 = 0; i0 < n_items; i0 += 32) {
+      const int i = i0 + lane;
+      int e = -1;
+      if (i < n_items) {
+        e = idx[i];
+        if ((unsigned)e >= (unsigned)E) {
+          inv_perm[i] = -1;
+          e = -1;
+        }
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0) {
+        const int r = run[e] + __popc(peers & lt_mask);
+        perm_token[r] = i / k;
+        inv_perm[i] = r;
+        p_perm[r] = w[i];
+      }
+      __syncwarp();
+      if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  pdl_trigger();
 }
 
 // x_perm[r] = x[perm_token[r]] for r < offsets[E]; one warp per row, 16-byte moves.
@@ -120,6 +204,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           const int32_t* __restrict__ perm_token,
                                                           const int32_t* __restrict__ offsets, int E, int T,
                                                           int D, uint16_t* __restrict__ x_perm) {
+  pdl_wait();
   const int n_rows = offsets[E];
   const int lane = threadIdx.x & 31;
   const int nv = D / 8;
@@ -130,6 +215,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * D);
     for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
   }
+  pdl_trigger();
 }
 
 }  // namespace
@@ -144,22 +230,35 @@ cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16
                            uint16_t* x_perm, int32_t* scratch, int* err, cudaStream_t s, int* n_launches) {
   const int nb = (T + kTokPerBlock - 1) / kTokPerBlock;
   int launches = 0;
-  if (nb > 0) {
-    hist_kernel<<<nb, 256, E * sizeof(int), s>>>(idx, T, E, k, scratch, err);
+  if (nb == 1) {
+    cudaError_t e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(256), 2 * E * sizeof(int), s, idx, topk_w, T, E,
+                               k, counts, offsets, perm_token, inv_perm, p_perm, err);
+    if (e != cudaSuccess) return e;
+    ++launches;
+  } else if (nb > 0) {
+    cudaError_t e = launch_pdl(hist_kernel, dim3(nb), dim3(256), E * sizeof(int), s, idx, T, E, k, scratch, err);
+    if (e != cudaSuccess) return e;
     ++launches;
   }
-  scan_kernel<<<1, 1024, 0, s>>>(scratch, nb, E, counts, offsets);
-  ++launches;
-  if (nb > 0) {
-    scatter_kernel<<<nb, 32, E * sizeof(int), s>>>(idx, topk_w, T, E, k, scratch, offsets, perm_token, inv_perm,
-                                                 p_perm);
+  cudaError_t e = cudaSuccess;
+  if (nb != 1) {
+    e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, scratch, nb, E, counts, offsets);
+    if (e != cudaSuccess) return e;
+    ++launches;
+  }
+  if (nb > 1) {
+    e = launch_pdl(scatter_kernel, dim3(nb), dim3(32), E * sizeof(int), s, idx, topk_w, T, E, k,
+                   (const int32_t*)scratch, (const int32_t*)offsets, perm_token, inv_perm, p_perm);
+    if (e != cudaSuccess) return e;
     ++launches;
   }
   if (x != nullptr && x_perm != nullptr && T > 0) {
     const long long rows = (long long)T * k;
     long long blocks = (rows + 7) / 8;
     if (blocks > 148LL * 16) blocks = 148LL * 16;
-    gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, perm_token, offsets, E, T, D, x_perm);
+    e = launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, (const int32_t*)perm_token,
+                   (const int32_t*)offsets, E, T, D, x_perm);
+    if (e != cudaSuccess) return e;
     ++launches;
   }
   if (n_launches) *n_launches = launches;

@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(kThreads) router_select_kernel(const float* __
                                                                  float* __restrict__ w_out) {
   const int lane = threadIdx.x & 31;
   const int e0 = lane * EJ;
+  pdl_wait();
   float bj[EJ];
 #pragma unroll
   for (int j = 0; j < EJ; ++j) bj[j] = (bias != nullptr && e0 + j < E) ? bias[e0 + j] : 0.f;
@@ -35,19 +36,20 @@ __global__ void __launch_bounds__(kThreads) router_select_kernel(const float* __
     float l[EJ];
 #pragma unroll
     for (int j = 0; j < EJ; ++j) l[j] = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float* row = part + ((size_t)s * T + t) * ld + e0;
-      if (EJ % 4 == 0 && e0 + EJ <= E) {
+    // split partials in split order; loads of up to 4 splits are issued before their adds
+    const size_t split_stride = (size_t)T * ld;
+    const float* row0 = part + (size_t)t * ld + e0;
+    for (int s0 = 0; s0 < S; s0 += 4) {
+      float v[4][EJ];
 #pragma unroll
-        for (int q = 0; q < EJ / 4; ++q) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(row) + q);
-          l[4 * q] += v.x, l[4 * q + 1] += v.y, l[4 * q + 2] += v.z, l[4 * q + 3] += v.w;
-        }
-      } else {
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
         for (int j = 0; j < EJ; ++j)
-          if (e0 + j < E) l[j] += __ldg(row + j);
-      }
+          v[u][j] = (s0 + u < S && e0 + j < E) ? __ldg(row0 + (size_t)(s0 + u) * split_stride + j) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int j = 0; j < EJ; ++j) l[j] += v[u][j];
     }
     uint32_t taken = 0;
     int my_idx = -1;
@@ -84,6 +86,7 @@ __global__ void __launch_bounds__(kThreads) router_select_kernel(const float* __
       w_out[(size_t)t * k + lane] = ex / z;
     }
   }
+  pdl_trigger();
 }
 
 template <int EJ>
@@ -91,8 +94,8 @@ cudaError_t launch(const float* part, int S, int T, int ld, const float* bias, i
                    cudaStream_t s) {
   long long blocks = ((long long)T + 7) / 8;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
-  router_select_kernel<EJ><<<(unsigned)blocks, kThreads, 0, s>>>(part, S, T, ld, bias, E, k, idx, w);
-  return cudaGetLastError();
+  return launch_pdl(router_select_kernel<EJ>, dim3((unsigned)blocks), dim3(kThreads), 0, s, part, S, T, ld, bias, E,
+                    k, idx, w);
 }
 
 }  // namespace

@@ -80,7 +80,8 @@ def test_layer_workspace_size_and_small_workspace(L):
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, need - 1, None) == 4
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100010, need, None) == 3  # ws not 256-aligned
     assert L.moe_layer_forward(ctypes.byref(d), 0x4008, 0x5000, 0x100000, need, None) == 3
-    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 9
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 7  # T=16: fused dispatch
+    assert L.moe_layer_kernel_count(ctypes.byref(_desc(T=300))) == 9
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(k=9))) == 0
     # shared expert grows the workspace
     d2 = _desc(Fs=256, shared_gate_up=0x6000, shared_down=0x7000)
