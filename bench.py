@@ -35,6 +35,30 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (read + write) of the dominant kernel per launch, from one ncu capture of the same
+# bench command (profiles/grouped_gemm_kernels.md), valid only while the GEMM sources are unchanged.
+_GEMM_SOURCES = ("sparse_mixture_experts_16_b200/csrc/grouped_gemm_sm100.cu",
+                 "sparse_mixture_experts_16_b200/csrc/sm100_ptx.cuh",
+                 "sparse_mixture_experts_16_b200/csrc/moe_common.cuh")
+_TRAFFIC_SOURCE_SHA256 = "c3f2678bfe5892ef2e25f811bf17341a5e59dc90db846cb22854a09d07975035"
+_TRAFFIC_BYTES = {  # workload -> gate_up launch: dram__bytes_read.sum + dram__bytes_write.sum
+    "mixtral": 1.946781e9 + 0.228668e9,
+    "deepseek_decode": 5.876604e9 + 0.004840e9,
+}
+
+
+def measured_traffic(workload: str):
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in _GEMM_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != _TRAFFIC_SOURCE_SHA256:
+        return None
+    return _TRAFFIC_BYTES.get(workload)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -308,13 +332,13 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         achieved = bytes_gu / (gate_ms / 1e3) / 1e9
         peak = pk["hbm_gbs"]
         roof = {"kernel": "grouped_gemm_kernel<gate_up, stream>", "bound": "hbm", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name),
                 "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)"}
     else:
         achieved = gateup_flops(w) / (gate_ms / 1e3) / 1e12
         peak = pk["bf16_tflops_sustained"]
         roof = {"kernel": "grouped_gemm_kernel<gate_up, tiled>", "bound": "tensor", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name),
                 "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
                 "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4)}
     layer_tflops = w.flops / (ms_per_step / 1e3) / 1e12 * world

@@ -1,0 +1,58 @@
+"""Host-side logic of bench.py (no GPU): the metric formulas, pinned to the pages' worked
+decode estimate and to closed forms, and the clock-record parsing."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(scope="module")
+def bench():
+    sys.argv = ["bench.py"]
+    import bench as b
+
+    return b
+
+
+def test_decode_bound_matches_the_pages_gpt_oss_estimate(bench):
+    """keryc.com, "Por que MoEs importan": 800 GB/s / (3.6e9 active params x 2 B) ~ 111 tok/s."""
+    with open(os.path.join(GOLDEN, "decode_bound_gptoss20b.txt")) as f:
+        row = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")][0]
+    bw, params, bpp, expected, tol = map(float, row)
+    assert abs(bench.decode_tokens_per_s_bound(bw, params, bpp) - expected) <= tol
+
+
+def test_flop_and_byte_accounting(bench):
+    import moe_inputs as mi
+
+    w = mi.WORKLOADS["mixtral"]
+    # gate_up: 2 FLOP x D x 2F per routed row; down: 2 x D x F per routed row; router 2 x D x E
+    assert bench.gateup_flops(w) == w.T * w.k * 4.0 * w.D * w.F
+    assert bench.down_flops(w) == w.T * w.k * 2.0 * w.D * w.F
+    assert w.flops == bench.gateup_flops(w) + bench.down_flops(w) + 2.0 * w.T * w.D * w.E
+    ds = mi.WORKLOADS["deepseek"]
+    assert ds.flops == pytest.approx(6.524e12, rel=1e-3)  # the layer's algorithmic FLOPs
+    # active-weight bytes: bf16 gate_up (2F x D) + down (D x F) per active expert, plus the shared one
+    assert bench.active_weight_bytes(ds, 1) == 2 * (3 * ds.D * ds.F + 3 * ds.D * ds.Fs)
+    assert bench.active_weight_bytes(ds, 10, "gate_up") == 2 * (10 * 2 * ds.F * ds.D + 2 * ds.Fs * ds.D)
+
+
+def test_traffic_is_reported_only_for_captured_workloads(bench):
+    assert bench.measured_traffic("tiny") is None
+    v = bench.measured_traffic("mixtral")
+    assert v is None or v > 1.9e9  # None once the kernel sources differ from the captured ones
+
+
+def test_clock_summary_flags_throttling(bench):
+    s = bench.ClockSampler("0")
+    s.lines = ["0, 1500, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active",
+               "0, 1400, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active",
+               "0, 210, 1965, 120.0, 0x0, Not Active, Not Active, Not Active, Not Active"]
+    out = s.summary()
+    assert out["sm_mhz"] == 1450 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3 and out["samples_under_load"] == 2
+    s.lines = ["0, 1000, 1965, 700.0, 0x8, Active, Not Active, Not Active, Not Active"]
+    assert s.summary()["reasons"] == ["hw_slowdown"]
