@@ -45,6 +45,8 @@ def _L():
         L.oracle_expert_ffn.restype = None
         L.oracle_layer.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, P, P, P, i32]
         L.oracle_layer_eager.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, P]
+        L.oracle_update_bias.argtypes = [P, i32, ctypes.c_float, P, P]
+        L.oracle_update_bias.restype = None
         _lib = L
     return _lib
 
@@ -177,6 +179,15 @@ def layer_eager(x, wg, bias, gate_up, down, k, shared_gate_up=None, shared_down=
     if rc != 0:
         raise ValueError(f"oracle_layer_eager rc={rc}")
     return y
+
+
+def update_bias(counts, gamma, bias):
+    """One aux-loss-free balancing step: bias + gamma * sign(mean(counts) - counts), fp32."""
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    b = np.ascontiguousarray(bias, dtype=np.float32)
+    out = np.empty_like(b)
+    _L().oracle_update_bias(c.ctypes.data, c.size, gamma, b.ctypes.data, out.ctypes.data)
+    return out
 
 
 # ----------------------------------------------------------------------------- gap-enforced inputs

@@ -260,4 +260,22 @@ int oracle_layer_eager(const uint16_t* x, const uint16_t* wg, const float* bias,
   return 0;
 }
 
+// Aux-loss-free balancing (gotburnout.io glossary "MoE", section 2 item 4: router biases are
+// adjusted dynamically so that no expert is overloaded).  The pages give no rule; the reading
+// taken: after a batch with per-expert loads c_e (slots routed to e), every bias moves by a fixed
+// step gamma towards balance,
+//     bias_e <- bias_e + gamma * sign(mean(c) - c_e),
+// an underloaded expert gaining score and an overloaded one losing it.  The comparison with the
+// mean is done exactly as sign(sum(c) - E * c_e).  Each new bias is the fp32 value of the exact
+// sum (the addition of two fp32 numbers rounded once).
+void oracle_update_bias(const int32_t* counts, int E, float gamma, const float* bias_in, float* bias_out) {
+  long long total = 0;
+  for (int e = 0; e < E; ++e) total += counts[e];
+  for (int e = 0; e < E; ++e) {
+    const long long diff = total - (long long)E * counts[e];
+    const double step = diff > 0 ? (double)gamma : (diff < 0 ? -(double)gamma : 0.0);
+    bias_out[e] = (float)((double)bias_in[e] + step);
+  }
+}
+
 }  // extern "C"

@@ -266,3 +266,47 @@ def test_sparse_expert_dict_matches_packed():
     y2, _, _ = oracle.layer(x, inp["wg"], None, {e: inp["gate_up"][e] for e in used},
                             {e: inp["down"][e] for e in used}, w.k)
     np.testing.assert_array_equal(y1, y2)
+
+
+# ----------------------------------------------------------------------------- balancing bias
+def test_bias_update_leaves_balanced_loads_alone():
+    b = np.linspace(-1, 1, 8).astype(np.float32)
+    assert (oracle.update_bias(np.full(8, 37, np.int32), 0.01, b) == b).all()
+
+
+def test_bias_update_closed_form():
+    """Loads 10, 30, 20 (mean 20): +gamma, -gamma, 0; the result is the fp32 sum."""
+    b = np.array([0.5, 0.25, -1.0], np.float32)
+    out = oracle.update_bias(np.array([10, 30, 20], np.int32), 0.125, b)
+    assert out.tolist() == [0.625, 0.125, -1.0]
+    # a step of half an ulp (on either side of 1024) rounds back to 1024 (ties to even)
+    big = np.array([1024.0, 1024.0], np.float32)
+    assert (oracle.update_bias(np.array([1, 3], np.int32), 2.0 ** -15, big) == big).all()
+
+
+def test_bias_update_is_scale_free_and_follows_loads():
+    rng = np.random.default_rng(18)
+    c = rng.integers(0, 500, 64).astype(np.int32)
+    b = (rng.standard_normal(64) * 0.3).astype(np.float32)
+    out = oracle.update_bias(c, 0.01, b)
+    assert (oracle.update_bias(c * 7, 0.01, b) == out).all()  # only relative loads matter
+    mean = c.mean()
+    assert (out[c > mean] < b[c > mean]).all() and (out[c < mean] > b[c < mean]).all()
+
+
+def test_bias_update_moves_routing_towards_balance():
+    """A few steps on a strongly skewed router lower the max/mean load (the rule's purpose)."""
+    rng = np.random.default_rng(19)
+    T, D, E, k = 512, 64, 16, 2
+    x, wg, *_ = _rand_layer(rng, T, D, E, 8)
+    bias = np.zeros(E, np.float32)
+    bias[:3] = 3.0  # three favourite experts
+    def imbalance(b):
+        idx, _ = oracle.router(x, wg, b, k)
+        c = np.bincount(idx.ravel(), minlength=E)
+        return c.max() / c.mean(), c
+    start, c = imbalance(bias)
+    for _ in range(40):
+        bias = oracle.update_bias(c.astype(np.int32), 0.1, bias)
+        _, c = imbalance(bias)
+    assert imbalance(bias)[0] < 0.6 * start
