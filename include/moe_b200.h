@@ -203,6 +203,24 @@ moe_status_t moe_layer_forward_timed(const moe_layer_desc_t* desc, const moe_bf1
 /* Number of kernels one moe_layer_forward launches for this descriptor (0 if invalid). */
 int moe_layer_kernel_count(const moe_layer_desc_t* desc);
 
+/* ----------------------------------------------------------------------------------------
+ * Aux-loss-free balancing (gotburnout.io glossary "MoE", section 2 item 4: router biases are
+ * adjusted dynamically so that no expert is overloaded).  The pages give no update rule; this
+ * library applies the sign rule on the loads of the last batch:
+ *     bias[e] += gamma * sign(mean(counts) - counts[e])        (fp32 add, round to nearest)
+ * with the comparison done exactly in integers.  counts [E] int32 (device; e.g. from
+ * moe_permute or moe_layer_expert_counts), bias [E] fp32 (device, updated in place),
+ * 1 <= E <= 1024, gamma >= 0.  One kernel; asynchronous on `stream`.
+ * ---------------------------------------------------------------------------------------- */
+moe_status_t moe_update_router_bias(const int32_t* counts, int E, float gamma, float* bias,
+                                    moe_stream_t stream);
+
+/* Device address of the per-expert loads counts[E] (int32) that moe_layer_forward leaves in
+ * its workspace (valid once the forward has run on the stream, until the next forward).  Host
+ * call only: nothing is launched. */
+moe_status_t moe_layer_expert_counts(const moe_layer_desc_t* desc, void* ws, size_t ws_bytes,
+                                     const int32_t** counts);
+
 /* Synchronises `stream`, returns the status held in the workspace's error word (MOE_OK,
  * MOE_ERR_DEVICE_INDEX or MOE_ERR_TIMEOUT) and clears it. */
 moe_status_t moe_get_device_error(void* ws, moe_stream_t stream);

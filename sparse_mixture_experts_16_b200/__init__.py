@@ -29,7 +29,8 @@ EXPORTS = (
     "moe_router_topk_workspace_size", "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
     "moe_grouped_swiglu_ffn_workspace_size",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_layer_workspace_size", "moe_layer_forward",
-    "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_get_device_error",
+    "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_update_router_bias",
+    "moe_layer_expert_counts", "moe_get_device_error",
     "moe_status_string",
 )
 
@@ -75,6 +76,8 @@ def lib():
             "moe_layer_forward_host": ([ctypes.POINTER(LayerDesc), P, P, P, Z, P], I),
             "moe_layer_forward_timed": ([ctypes.POINTER(LayerDesc), P, P, P, Z, P, ctypes.POINTER(P), I], I),
             "moe_layer_kernel_count": ([ctypes.POINTER(LayerDesc)], I),
+            "moe_update_router_bias": ([P, I, ctypes.c_float, P, P], I),
+            "moe_layer_expert_counts": ([ctypes.POINTER(LayerDesc), P, Z, ctypes.POINTER(P)], I),
             "moe_get_device_error": ([P, P], I),
             "moe_status_string": ([I], ctypes.c_char_p),
         }
@@ -292,11 +295,34 @@ class MoELayer:
                                              _stream(stream), handles, len(events)), "moe_layer_forward_timed")
         return y
 
+    def expert_counts(self, T: int):
+        """counts[E] int32 left in the workspace by the last forward of T tokens (a view, not a copy)."""
+        import torch
+
+        ws = self.workspace(T)
+        d = self.desc(T)
+        ptr = ctypes.c_void_p()
+        _check(lib().moe_layer_expert_counts(ctypes.byref(d), ws.data_ptr(), ws.numel(), ctypes.byref(ptr)),
+               "moe_layer_expert_counts")
+        off = ptr.value - ws.data_ptr()
+        return ws[off:off + 4 * self.E].view(torch.int32)
+
     def device_error(self, stream=None) -> int:
         """Synchronises and returns (and clears) the workspace's device error status."""
         if self._ws is None:
             return 0
         return lib().moe_get_device_error(self._ws.data_ptr(), _stream(stream))
+
+
+def moe_update_router_bias(counts, gamma, bias, stream=None):
+    """One aux-loss-free balancing step in place: bias += gamma * sign(mean(counts) - counts)."""
+    import torch
+
+    _need(counts, torch.int32, None, "counts")
+    _need(bias, torch.float32, tuple(counts.shape), "bias")
+    _check(lib().moe_update_router_bias(counts.data_ptr(), counts.numel(), float(gamma), bias.data_ptr(),
+                                        _stream(stream)), "moe_update_router_bias")
+    return bias
 
 
 def moe_get_device_error(ws, stream=None) -> int:

@@ -70,6 +70,8 @@ cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wg, int T, int
 cudaError_t launch_router_select(const float* partials, int k_splits, int T, int ld, const float* bias, int E, int k,
                                  int32_t* idx, float* w, cudaStream_t s);
 
+cudaError_t launch_update_bias(const int32_t* counts, int E, float gamma, float* bias, cudaStream_t s);
+
 size_t permute_scratch_bytes(int T, int E);
 cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16_t* x, int T, int D, int E,
                            int k, int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,

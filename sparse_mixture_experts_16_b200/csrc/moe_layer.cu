@@ -344,6 +344,29 @@ int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   return 2 /*router GEMM, top-k*/ + dispatch + 1 /*gather*/ + 2 /*grouped GEMMs*/ + 1 /*combine*/;
 }
 
+moe_status_t moe_update_router_bias(const int32_t* counts, int E, float gamma, float* bias, moe_stream_t stream) {
+  if (!counts || !bias || E <= 0) return MOE_ERR_INVALID_ARG;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!(gamma >= 0.0f) || gamma > 1e30f) return MOE_ERR_INVALID_ARG;  // also rejects NaN
+  if (!aligned(counts, 4) || !aligned(bias, 4)) return MOE_ERR_ALIGNMENT;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  MOE_CUDA_TRY(launch_update_bias(counts, E, gamma, bias, (cudaStream_t)stream));
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_expert_counts(const moe_layer_desc_t* desc, void* ws, size_t ws_bytes,
+                                     const int32_t** counts) {
+  moe_status_t st = validate_desc(desc);
+  if (st != MOE_OK) return st;
+  if (!ws || !counts) return MOE_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;
+  const LayerWs w = layer_ws(*desc);
+  if (ws_bytes < w.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  *counts = reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(ws) + w.counts);
+  return MOE_OK;
+}
+
 moe_status_t moe_get_device_error(void* ws, moe_stream_t stream) {
   if (!ws) return MOE_ERR_INVALID_ARG;
   if (!aligned(ws, 256)) return MOE_ERR_ALIGNMENT;

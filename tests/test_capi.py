@@ -135,3 +135,18 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(ImportError):
         moe.lib()
+
+
+def test_bias_update_and_counts_validate_on_host(L):
+    assert L.moe_update_router_bias(None, 8, 0.01, 0x2000, None) == 1
+    assert L.moe_update_router_bias(0x1000, 0, 0.01, 0x2000, None) == 1
+    assert L.moe_update_router_bias(0x1000, 1025, 0.01, 0x2000, None) == 2
+    assert L.moe_update_router_bias(0x1000, 8, -1.0, 0x2000, None) == 1
+    assert L.moe_update_router_bias(0x1000, 8, float("nan"), 0x2000, None) == 1
+    assert L.moe_update_router_bias(0x1002, 8, 0.01, 0x2000, None) == 3
+    d = _desc()
+    need = L.moe_layer_workspace_size(ctypes.byref(d))
+    ptr = ctypes.c_void_p()
+    assert L.moe_layer_expert_counts(ctypes.byref(d), 0x100000, need, ctypes.byref(ptr)) == 0
+    assert 0x100000 < ptr.value < 0x100000 + need and ptr.value % 256 == 0
+    assert L.moe_layer_expert_counts(ctypes.byref(d), 0x100000, need - 1, ctypes.byref(ptr)) == 4
