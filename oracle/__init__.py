@@ -47,6 +47,14 @@ def _L():
         L.oracle_layer_eager.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, P]
         L.oracle_update_bias.argtypes = [P, i32, ctypes.c_float, P, P]
         L.oracle_update_bias.restype = None
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_quantize_rows_fp8.argtypes = [P, i64, i64, P, P]
+        L.oracle_quantize_rows_fp8.restype = None
+        L.oracle_expert_ffn_fp8.argtypes = [P, P, P, P, P, i64, i64, P]
+        L.oracle_expert_ffn_fp8.restype = None
         _lib = L
     return _lib
 
@@ -188,6 +196,54 @@ def update_bias(counts, gamma, bias):
     out = np.empty_like(b)
     _L().oracle_update_bias(c.ctypes.data, c.size, gamma, b.ctypes.data, out.ctypes.data)
     return out
+
+
+def e4m3_value(code: int) -> float:
+    return _L().oracle_e4m3_value(code)
+
+
+def e4m3_encode(v: float) -> int:
+    return _L().oracle_e4m3_encode(v)
+
+
+def quantize_rows_fp8(w):
+    """Per-row E4M3 quantisation of a bf16 [rows, K] array: (codes uint8 [rows, K], scales fp32 [rows])."""
+    w = _u16(w)
+    K = w.shape[-1]
+    rows = w.size // K
+    q = np.empty(w.shape, np.uint8)
+    sc = np.empty(w.shape[:-1], np.float32)
+    _L().oracle_quantize_rows_fp8(w.ctypes.data, rows, K, q.ctypes.data, sc.ctypes.data)
+    return q, sc
+
+
+def expert_ffn_fp8(x_row, gu_q, gu_s, dn_q, dn_s):
+    x_row = _u16(x_row)
+    gu_q, dn_q = np.ascontiguousarray(gu_q, np.uint8), np.ascontiguousarray(dn_q, np.uint8)
+    gu_s, dn_s = np.ascontiguousarray(gu_s, np.float32), np.ascontiguousarray(dn_s, np.float32)
+    D = x_row.shape[-1]
+    F = dn_q.shape[1]
+    assert gu_q.shape == (2 * F, D) and dn_q.shape == (D, F) and gu_s.shape == (2 * F,) and dn_s.shape == (D,)
+    out = np.empty(D, np.float64)
+    _L().oracle_expert_ffn_fp8(x_row.ctypes.data, gu_q.ctypes.data, gu_s.ctypes.data, dn_q.ctypes.data,
+                               dn_s.ctypes.data, D, F, out.ctypes.data)
+    return out
+
+
+def layer_fp8(x, wg, bias, k, q, shared=None):
+    """y[T, D] of the layer with E4M3 expert weights.  q: dict(gu_q [E,2F,D], gu_s [E,2F],
+    dn_q [E,D,F], dn_s [E,D]) (or dicts {expert: array} for the experts used); shared: the same
+    four arrays for the shared expert or None.  Returns (y, idx, p)."""
+    idx, p = router(x, wg, bias, k)
+    T, D = x.shape
+    y = np.zeros((T, D), np.float64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            y[t] += p[t, j] * expert_ffn_fp8(x[t], q["gu_q"][e], q["gu_s"][e], q["dn_q"][e], q["dn_s"][e])
+        if shared is not None:
+            y[t] += expert_ffn_fp8(x[t], shared["gu_q"], shared["gu_s"], shared["dn_q"], shared["dn_s"])
+    return y, idx, p
 
 
 # ----------------------------------------------------------------------------- gap-enforced inputs

@@ -278,4 +278,71 @@ void oracle_update_bias(const int32_t* counts, int E, float gamma, const float* 
   }
 }
 
+// ---- FP8 (E4M3) expert weights -------------------------------------------------------------
+// keryc.com "Mixture of Experts optimiza...", section "Resultados practicos": quantising "per
+// expert" makes sense once the experts are packed.  Reading taken: each row of a packed weight
+// tensor (one output feature of one expert) gets its own fp32 scale s = amax(row) / 448 and the
+// codes q = E4M3(w / s), round to nearest even, saturating at +-448.  The row is dequantised as
+// q * s.  E4M3 (OCP FP8): 1 sign, 4 exponent (bias 7), 3 mantissa bits; normal values
+// 2^(e-7) * (1 + m/8) for e = 1..15 (e = 15 with m = 7 is NaN, so the largest is 448);
+// subnormals m * 2^-9.
+
+// Value of an E4M3 code.
+double oracle_e4m3_value(uint8_t code) {
+  const int sgn = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  double v = (e == 0) ? m * std::ldexp(1.0, -9) : std::ldexp(1.0 + m / 8.0, e - 7);
+  if (e == 15 && m == 7) v = NAN;
+  return sgn ? -v : v;
+}
+
+// Nearest E4M3 code to a finite value (ties to the even code), saturating at +-448.
+uint8_t oracle_e4m3_encode(double v) {
+  const uint8_t sgn = std::signbit(v) ? 0x80 : 0;
+  const double a = std::fabs(v);
+  // walk the 127 non-negative finite codes (0x00 .. 0x7E) in increasing order
+  uint8_t best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    const double err = std::fabs(oracle_e4m3_value((uint8_t)c) - a);
+    if (err < best_err || (err == best_err && (c & 1) == 0)) best = (uint8_t)c, best_err = err;
+  }
+  return sgn | best;
+}
+
+// Per-row quantisation of a bf16 [rows, K] tensor: scales[r] = amax / 448 (fp32), codes of
+// (w / scale) computed in fp32.  All-zero rows get scale 1 and zero codes.
+void oracle_quantize_rows_fp8(const uint16_t* w, int64_t rows, int64_t K, uint8_t* q, float* scales) {
+  for (int64_t r = 0; r < rows; ++r) {
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) amax = std::max(amax, (float)std::fabs(bf16_value(w[r * K + k])));
+    const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+    scales[r] = s;
+    for (int64_t k = 0; k < K; ++k) {
+      const float v = (float)bf16_value(w[r * K + k]) / s;
+      q[r * K + k] = oracle_e4m3_encode((double)v);
+    }
+  }
+}
+
+// One SwiGLU expert on one token with E4M3 weights: the definition of expert_ffn above on the
+// dequantised weights (q * scale, exact in fp64).
+void oracle_expert_ffn_fp8(const uint16_t* x_row, const uint8_t* gu_q, const float* gu_s, const uint8_t* dn_q,
+                           const float* dn_s, int64_t D, int64_t F, double* out) {
+  std::vector<double> a(F);
+  for (int64_t n = 0; n < F; ++n) {
+    double g = 0.0, u = 0.0;
+    for (int64_t d = 0; d < D; ++d) {
+      const double xv = bf16_value(x_row[d]);
+      g += oracle_e4m3_value(gu_q[n * D + d]) * (double)gu_s[n] * xv;
+      u += oracle_e4m3_value(gu_q[(F + n) * D + d]) * (double)gu_s[F + n] * xv;
+    }
+    a[n] = g / (1.0 + std::exp(-g)) * u;
+  }
+  for (int64_t d = 0; d < D; ++d) {
+    double acc = 0.0;
+    for (int64_t n = 0; n < F; ++n) acc += oracle_e4m3_value(dn_q[d * F + n]) * (double)dn_s[d] * a[n];
+    out[d] = acc;
+  }
+}
+
 }  // extern "C"

@@ -310,3 +310,62 @@ def test_bias_update_moves_routing_towards_balance():
         bias = oracle.update_bias(c.astype(np.int32), 0.1, bias)
         _, c = imbalance(bias)
     assert imbalance(bias)[0] < 0.6 * start
+
+
+# ----------------------------------------------------------------------------- FP8 (E4M3) weights
+def test_e4m3_code_values():
+    """OCP FP8 E4M3: bias 7, 3 mantissa bits, no infinities, S.1111.111 is NaN."""
+    assert oracle.e4m3_value(0x38) == 1.0
+    assert oracle.e4m3_value(0x7E) == 448.0
+    assert oracle.e4m3_value(0x08) == 2.0 ** -6          # smallest normal
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9          # smallest subnormal
+    assert oracle.e4m3_value(0x07) == 7 * 2.0 ** -9
+    assert oracle.e4m3_value(0xB8) == -1.0
+    assert math.isnan(oracle.e4m3_value(0x7F)) and math.isnan(oracle.e4m3_value(0xFF))
+
+
+def test_e4m3_encode_rounds_to_nearest_even_and_saturates():
+    assert oracle.e4m3_encode(1.0) == 0x38
+    assert oracle.e4m3_encode(1.0625) == 0x38            # halfway 1 .. 1.125 -> even
+    assert oracle.e4m3_encode(1.1875) == 0x3A            # halfway 1.125 .. 1.25 -> even
+    assert oracle.e4m3_encode(1.06) == 0x38 and oracle.e4m3_encode(1.07) == 0x39
+    assert oracle.e4m3_encode(2.0 ** -10) == 0x00        # halfway 0 .. 2^-9 -> even (zero)
+    assert oracle.e4m3_encode(3 * 2.0 ** -10) == 0x02    # halfway 2^-9 .. 2^-8 -> even
+    assert oracle.e4m3_encode(447.9) == 0x7E and oracle.e4m3_encode(1e6) == 0x7E
+    assert oracle.e4m3_encode(-1e6) == 0xFE
+    for c in list(range(0x00, 0x7F)) + list(range(0x81, 0xFF)):  # every finite non-zero code
+        assert oracle.e4m3_encode(oracle.e4m3_value(c)) == c
+
+
+def test_row_quantisation_scales_to_448():
+    rng = np.random.default_rng(20)
+    w = _bf16(rng.standard_normal((16, 256)) * 0.02)
+    w[3] = 0  # an all-zero row
+    q, s = oracle.quantize_rows_fp8(w)
+    W = f64(w)
+    assert s[3] == 1.0 and (q[3] == 0).all()
+    for r in [0, 5, 15]:
+        amax = np.abs(W[r]).max()
+        assert s[r] == np.float32(np.float32(amax) / np.float32(448.0))
+        vals = np.array([oracle.e4m3_value(c) for c in q[r]]) * s[r]
+        assert np.abs(vals).max() == pytest.approx(amax, rel=1e-6)
+        # within half an E4M3 step (relative 2^-4 for normals) of the original
+        assert (np.abs(vals - W[r]) <= np.maximum(np.abs(W[r]) * 2.0 ** -4, 2.0 ** -10 * s[r]) + 1e-12).all()
+
+
+def test_fp8_ffn_equals_bf16_ffn_on_exactly_representable_weights():
+    """If every weight is an E4M3 value times a power-of-two scale, dequantisation is exact and the
+    FP8-weight expert equals the bf16 expert bit for bit."""
+    rng = np.random.default_rng(21)
+    D, F = 32, 16
+    codes = rng.integers(0, 0x7E, (2 * F + D, max(D, F))).astype(np.uint8)
+    codes |= rng.integers(0, 2, codes.shape).astype(np.uint8) << 7
+    codes[:, 0] = 0x7E  # every row reaches 448, so its scale is exactly the power of two below
+    vals = np.vectorize(oracle.e4m3_value)(codes) * 2.0 ** -12
+    gu = _bf16(vals[: 2 * F, :D])
+    dn = _bf16(vals[2 * F:, :F])
+    assert (f64(gu) == vals[: 2 * F, :D]).all()  # exactly representable in bf16 too
+    x = _bf16(rng.standard_normal(D))
+    gq, gs = oracle.quantize_rows_fp8(gu)
+    dq, ds = oracle.quantize_rows_fp8(dn)
+    np.testing.assert_array_equal(oracle.expert_ffn_fp8(x, gq, gs, dq, ds), oracle.expert_ffn(x, gu, dn))
