@@ -167,6 +167,9 @@ moe_status_t moe_combine(const float* out_perm, const int32_t* inv_perm, const f
 #define MOE_FLAG_FORCE_PREFILL 1
 #define MOE_FLAG_FORCE_DECODE 2 /* only valid for T <= 64 */
 
+#define MOE_WEIGHTS_BF16 0     /* gate_up / down (and shared_*) hold bf16 weights            */
+#define MOE_WEIGHTS_FP8_E4M3 1 /* *_fp8 hold E4M3 codes with one fp32 scale per weight row  */
+
 typedef struct {
   int32_t T, D, E, k, F, Fs;       /* Fs = 0: no shared expert                              */
   const moe_bf16_t* w_gate;        /* [E, D]                                                */
@@ -176,7 +179,28 @@ typedef struct {
   const moe_bf16_t* shared_gate_up;/* [2Fs, D] or NULL                                      */
   const moe_bf16_t* shared_down;   /* [D, Fs] or NULL                                       */
   int32_t flags;                   /* 0 or MOE_FLAG_*                                       */
+  /* Expert weights as E4M3 codes (the pages' per-expert quantisation, keryc.com "Mixture of
+   * Experts optimiza...", section "Resultados practicos"; codes from moe_quantize_rows_fp8):
+   * used when weight_format == MOE_WEIGHTS_FP8_E4M3, where the bf16 gate_up / down / shared_*
+   * pointers are ignored.  Row r of a tensor dequantises to code * scale[r].  Decode only
+   * (T <= 64; larger T returns MOE_ERR_UNSUPPORTED_SHAPE); activations run in f16. */
+  int32_t weight_format;                /* MOE_WEIGHTS_BF16 or MOE_WEIGHTS_FP8_E4M3          */
+  const uint8_t* gate_up_fp8;           /* [E, 2F, D] codes                                  */
+  const float* gate_up_scale;           /* [E, 2F]                                           */
+  const uint8_t* down_fp8;              /* [E, D, F] codes                                   */
+  const float* down_scale;              /* [E, D]                                            */
+  const uint8_t* shared_gate_up_fp8;    /* [2Fs, D] codes or NULL                            */
+  const float* shared_gate_up_scale;    /* [2Fs] or NULL                                     */
+  const uint8_t* shared_down_fp8;       /* [D, Fs] codes or NULL                             */
+  const float* shared_down_scale;       /* [D] or NULL                                       */
 } moe_layer_desc_t;
+
+/* Per-row E4M3 quantisation of a packed bf16 weight tensor w [rows, K] (device; K a multiple of
+ * 64): scales[r] = amax(|w[r]|) / 448 (1 for an all-zero row) and q[r][k] = E4M3(w[r][k] /
+ * scales[r]), round to nearest even, saturating at +-448.  q [rows, K] uint8, scales [rows] fp32
+ * (device).  Asynchronous on `stream`. */
+moe_status_t moe_quantize_rows_fp8(const moe_bf16_t* w, int64_t rows, int K, uint8_t* q, float* scales,
+                                   moe_stream_t stream);
 
 /* Device workspace bytes for moe_layer_forward / moe_layer_forward_host (0 if desc invalid). */
 size_t moe_layer_workspace_size(const moe_layer_desc_t* desc);

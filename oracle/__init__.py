@@ -51,7 +51,7 @@ def _L():
         L.oracle_e4m3_value.restype = ctypes.c_double
         L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
-        L.oracle_quantize_rows_fp8.argtypes = [P, i64, i64, P, P]
+        L.oracle_quantize_rows_fp8.argtypes = [P, i64, i64, P, P, i32]
         L.oracle_quantize_rows_fp8.restype = None
         L.oracle_expert_ffn_fp8.argtypes = [P, P, P, P, P, i64, i64, P]
         L.oracle_expert_ffn_fp8.restype = None
@@ -213,7 +213,7 @@ def quantize_rows_fp8(w):
     rows = w.size // K
     q = np.empty(w.shape, np.uint8)
     sc = np.empty(w.shape[:-1], np.float32)
-    _L().oracle_quantize_rows_fp8(w.ctypes.data, rows, K, q.ctypes.data, sc.ctypes.data)
+    _L().oracle_quantize_rows_fp8(w.ctypes.data, rows, K, q.ctypes.data, sc.ctypes.data, _nthreads())
     return q, sc
 
 
@@ -234,15 +234,22 @@ def layer_fp8(x, wg, bias, k, q, shared=None):
     """y[T, D] of the layer with E4M3 expert weights.  q: dict(gu_q [E,2F,D], gu_s [E,2F],
     dn_q [E,D,F], dn_s [E,D]) (or dicts {expert: array} for the experts used); shared: the same
     four arrays for the shared expert or None.  Returns (y, idx, p)."""
+    from concurrent.futures import ThreadPoolExecutor
+
     idx, p = router(x, wg, bias, k)
     T, D = x.shape
-    y = np.zeros((T, D), np.float64)
-    for t in range(T):
+
+    def token(t):  # tokens are independent; the C call releases the GIL
+        yt = np.zeros(D, np.float64)
         for j in range(k):
             e = int(idx[t, j])
-            y[t] += p[t, j] * expert_ffn_fp8(x[t], q["gu_q"][e], q["gu_s"][e], q["dn_q"][e], q["dn_s"][e])
+            yt += p[t, j] * expert_ffn_fp8(x[t], q["gu_q"][e], q["gu_s"][e], q["dn_q"][e], q["dn_s"][e])
         if shared is not None:
-            y[t] += expert_ffn_fp8(x[t], shared["gu_q"], shared["gu_s"], shared["dn_q"], shared["dn_s"])
+            yt += expert_ffn_fp8(x[t], shared["gu_q"], shared["gu_s"], shared["dn_q"], shared["dn_s"])
+        return yt
+
+    with ThreadPoolExecutor(max_workers=_nthreads()) as pool:
+        y = np.stack(list(pool.map(token, range(T)))) if T else np.zeros((0, D), np.float64)
     return y, idx, p
 
 

@@ -295,24 +295,33 @@ double oracle_e4m3_value(uint8_t code) {
   return sgn ? -v : v;
 }
 
-// Nearest E4M3 code to a finite value (ties to the even code), saturating at +-448.
+// Nearest E4M3 code to a finite value (ties to the even code), saturating at +-448.  The
+// non-negative finite codes 0x00..0x7E have increasing values, so the nearest one is found by
+// bisection over their values.
 uint8_t oracle_e4m3_encode(double v) {
+  static const std::vector<double> table = [] {
+    std::vector<double> t(127);
+    for (int c = 0; c <= 0x7E; ++c) t[c] = oracle_e4m3_value((uint8_t)c);
+    return t;
+  }();
   const uint8_t sgn = std::signbit(v) ? 0x80 : 0;
   const double a = std::fabs(v);
-  // walk the 127 non-negative finite codes (0x00 .. 0x7E) in increasing order
-  uint8_t best = 0;
-  double best_err = INFINITY;
-  for (int c = 0; c <= 0x7E; ++c) {
-    const double err = std::fabs(oracle_e4m3_value((uint8_t)c) - a);
-    if (err < best_err || (err == best_err && (c & 1) == 0)) best = (uint8_t)c, best_err = err;
+  if (a >= table[0x7E]) return sgn | 0x7E;
+  int lo = 0, hi = 0x7E;  // table[lo] <= a < table[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) / 2;
+    if (table[mid] <= a) lo = mid; else hi = mid;
   }
-  return sgn | best;
+  const double dlo = a - table[lo], dhi = table[hi] - a;
+  const int c = dlo < dhi ? lo : (dhi < dlo ? hi : ((lo & 1) == 0 ? lo : hi));
+  return sgn | (uint8_t)c;
 }
 
 // Per-row quantisation of a bf16 [rows, K] tensor: scales[r] = amax / 448 (fp32), codes of
 // (w / scale) computed in fp32.  All-zero rows get scale 1 and zero codes.
-void oracle_quantize_rows_fp8(const uint16_t* w, int64_t rows, int64_t K, uint8_t* q, float* scales) {
-  for (int64_t r = 0; r < rows; ++r) {
+void oracle_quantize_rows_fp8(const uint16_t* w, int64_t rows, int64_t K, uint8_t* q, float* scales,
+                              int nthreads) {
+  for_tokens(rows, nthreads, [&](int64_t r) {  // rows are independent
     float amax = 0.0f;
     for (int64_t k = 0; k < K; ++k) amax = std::max(amax, (float)std::fabs(bf16_value(w[r * K + k])));
     const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
@@ -321,7 +330,7 @@ void oracle_quantize_rows_fp8(const uint16_t* w, int64_t rows, int64_t K, uint8_
       const float v = (float)bf16_value(w[r * K + k]) / s;
       q[r * K + k] = oracle_e4m3_encode((double)v);
     }
-  }
+  });
 }
 
 // One SwiGLU expert on one token with E4M3 weights: the definition of expert_ffn above on the

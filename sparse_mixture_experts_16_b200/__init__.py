@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_FLAG_FORCE_PREFILL = 1
 MOE_FLAG_FORCE_DECODE = 2
+MOE_WEIGHTS_BF16 = 0
+MOE_WEIGHTS_FP8_E4M3 = 1
 
 STATUS = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE", 3: "MOE_ERR_ALIGNMENT",
@@ -26,7 +28,7 @@ STATUS = {
 
 # every symbol include/moe_b200.h declares
 EXPORTS = (
-    "moe_router_topk_workspace_size", "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
+    "moe_quantize_rows_fp8", "moe_router_topk_workspace_size", "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
     "moe_grouped_swiglu_ffn_workspace_size",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_layer_workspace_size", "moe_layer_forward",
     "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_update_router_bias",
@@ -48,6 +50,11 @@ class LayerDesc(ctypes.Structure):
         ("w_gate", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("gate_up", ctypes.c_void_p),
         ("down", ctypes.c_void_p), ("shared_gate_up", ctypes.c_void_p), ("shared_down", ctypes.c_void_p),
         ("flags", ctypes.c_int32),
+        ("weight_format", ctypes.c_int32),
+        ("gate_up_fp8", ctypes.c_void_p), ("gate_up_scale", ctypes.c_void_p),
+        ("down_fp8", ctypes.c_void_p), ("down_scale", ctypes.c_void_p),
+        ("shared_gate_up_fp8", ctypes.c_void_p), ("shared_gate_up_scale", ctypes.c_void_p),
+        ("shared_down_fp8", ctypes.c_void_p), ("shared_down_scale", ctypes.c_void_p),
     ]
 
 
@@ -63,6 +70,7 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         sig = {
+            "moe_quantize_rows_fp8": ([P, ctypes.c_int64, I, P, P, P], I),
             "moe_router_topk_workspace_size": ([I, I, I], Z),
             "moe_router_topk": ([P, P, P, I, I, I, I, P, P, P, Z, P], I),
             "moe_permute_workspace_size": ([I, I, I], Z),
@@ -113,6 +121,20 @@ def _need(t, dtype, shape, name):
 
 
 # ------------------------------------------------------------------------------ steps
+def moe_quantize_rows_fp8(w, stream=None):
+    """Per-row E4M3 codes of a bf16 tensor [..., K]: (codes uint8 [..., K], scales fp32 [...])."""
+    import torch
+
+    _need(w, torch.bfloat16, None, "w")
+    K = w.shape[-1]
+    rows = w.numel() // K
+    q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    sc = torch.empty(w.shape[:-1], dtype=torch.float32, device=w.device)
+    _check(lib().moe_quantize_rows_fp8(w.data_ptr(), rows, K, q.data_ptr(), sc.data_ptr(), _stream(stream)),
+           "moe_quantize_rows_fp8")
+    return q, sc
+
+
 def moe_router_topk(x, w_gate, bias, k, topk_idx=None, topk_w=None, ws=None, stream=None):
     """Router projection + top-k + softmax over the chosen k -> (topk_idx[T,k] int32, topk_w[T,k] fp32)."""
     import torch
@@ -228,11 +250,16 @@ class MoELayer:
 
     w_gate [E,D] bf16, bias [E] fp32 or None, gate_up [E,2F,D] bf16, down [E,D,F] bf16,
     shared_gate_up [2Fs,D] / shared_down [D,Fs] bf16 or None.  Tensors must stay alive.
+    With ``scales`` = dict(gate_up=[E,2F], down=[E,D], shared_gate_up=[2Fs], shared_down=[D]) the
+    weight tensors are E4M3 codes (uint8, from moe_quantize_rows_fp8) and the layer runs its
+    FP8-weight decode kernels (T <= 64).
     """
 
-    def __init__(self, w_gate, gate_up, down, k, bias=None, shared_gate_up=None, shared_down=None, flags=0):
+    def __init__(self, w_gate, gate_up, down, k, bias=None, shared_gate_up=None, shared_down=None, flags=0,
+                 scales=None):
         self.w_gate, self.gate_up, self.down, self.bias = w_gate, gate_up, down, bias
         self.shared_gate_up, self.shared_down = shared_gate_up, shared_down
+        self.scales = scales
         self.E, self.D = w_gate.shape
         self.F = gate_up.shape[1] // 2
         self.Fs = 0 if shared_gate_up is None else shared_gate_up.shape[0] // 2
@@ -241,9 +268,16 @@ class MoELayer:
         self._ws = None
 
     def desc(self, T: int) -> LayerDesc:
+        if self.scales is None:
+            return LayerDesc(T, self.D, self.E, self.k, self.F, self.Fs, self.w_gate.data_ptr(), _ptr(self.bias),
+                             self.gate_up.data_ptr(), self.down.data_ptr(), _ptr(self.shared_gate_up),
+                             _ptr(self.shared_down), self.flags, MOE_WEIGHTS_BF16)
+        sc = self.scales
         return LayerDesc(T, self.D, self.E, self.k, self.F, self.Fs, self.w_gate.data_ptr(), _ptr(self.bias),
-                         self.gate_up.data_ptr(), self.down.data_ptr(), _ptr(self.shared_gate_up),
-                         _ptr(self.shared_down), self.flags)
+                         None, None, None, None, self.flags, MOE_WEIGHTS_FP8_E4M3,
+                         self.gate_up.data_ptr(), sc["gate_up"].data_ptr(), self.down.data_ptr(),
+                         sc["down"].data_ptr(), _ptr(self.shared_gate_up), _ptr(sc.get("shared_gate_up")),
+                         _ptr(self.shared_down), _ptr(sc.get("shared_down")))
 
     def workspace(self, T: int):
         import torch

@@ -105,4 +105,18 @@ enum GemmKind { kGateUp = 0, kDown = 1, kRouter = 2 };
 cudaError_t launch_grouped_gemm(GemmKind kind, const GemmSetHost* sets, int n_sets, int decode_nt, int* err,
                                 cudaStream_t s);
 
+// Weight-streaming grouped GEMMs with E4M3 expert weights (one fp32 scale per weight row,
+// w_scales[set]) and f16 activations (sets[i].a); gate_up writes f16 h.  decode_nt: 16..64.
+cudaError_t launch_stream_fp8w(GemmKind kind, const GemmSetHost* sets, const float* const* w_scales, int n_sets,
+                               int decode_nt, int* err, cudaStream_t s);
+
+// Per-row E4M3 quantisation: scales[r] = amax(row) / 448, q = E4M3(w / scale).  K % 8 == 0.
+cudaError_t launch_quantize_rows_fp8(const uint16_t* w, long long rows, int K, uint8_t* q, float* scales,
+                                     cudaStream_t s);
+
+// x_perm rows as f16 (x_perm16[r] = f16(x[perm_token[r]])) and a plain bf16 -> f16 cast.
+cudaError_t launch_gather_rows_f16(const uint16_t* x, const int32_t* perm_token, const int32_t* offsets, int E,
+                                   int T, int D, uint16_t* x_perm16, cudaStream_t s);
+cudaError_t launch_cast_bf16_to_f16(const uint16_t* src, long long n, uint16_t* dst, cudaStream_t s);
+
 }  // namespace moe

@@ -40,7 +40,7 @@ moe_status_t shape_status(long long T, long long D, long long E, long long k) {
 
 struct LayerWs {
   size_t router, topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
-      out_sh, x_stage, y_stage, total;
+      out_sh, x16, x_stage, y_stage, total;
 };
 
 LayerWs layer_ws(const moe_layer_desc_t& d) {
@@ -66,6 +66,7 @@ LayerWs layer_ws(const moe_layer_desc_t& d) {
   w.h_sh = take(T * Fs * 2);
   w.out_perm = take(M * D * 4);
   w.out_sh = take(T * D * 4);
+  w.x16 = take(T * D * 2);
   w.x_stage = take(T * D * 2);
   w.y_stage = take(T * D * 2);
   w.total = o;
@@ -80,9 +81,26 @@ moe_status_t validate_desc(const moe_layer_desc_t* d) {
   if (d->F % 64 != 0 || d->Fs % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if ((long long)d->E * 2 * d->F >= (1LL << 31) || (long long)d->T * d->k * d->F >= (1LL << 40))
     return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (!d->w_gate || !d->gate_up || !d->down) return MOE_ERR_INVALID_ARG;
-  if ((d->Fs > 0) != (d->shared_gate_up != nullptr) || (d->Fs > 0) != (d->shared_down != nullptr))
+  if (!d->w_gate) return MOE_ERR_INVALID_ARG;
+  if (d->weight_format == MOE_WEIGHTS_BF16) {
+    if (!d->gate_up || !d->down) return MOE_ERR_INVALID_ARG;
+    if ((d->Fs > 0) != (d->shared_gate_up != nullptr) || (d->Fs > 0) != (d->shared_down != nullptr))
+      return MOE_ERR_INVALID_ARG;
+  } else if (d->weight_format == MOE_WEIGHTS_FP8_E4M3) {
+    if (!d->gate_up_fp8 || !d->down_fp8 || !d->gate_up_scale || !d->down_scale) return MOE_ERR_INVALID_ARG;
+    const bool sh = d->Fs > 0;
+    if (sh != (d->shared_gate_up_fp8 != nullptr) || sh != (d->shared_down_fp8 != nullptr) ||
+        sh != (d->shared_gate_up_scale != nullptr) || sh != (d->shared_down_scale != nullptr))
+      return MOE_ERR_INVALID_ARG;
+    if (d->flags & MOE_FLAG_FORCE_PREFILL) return MOE_ERR_INVALID_ARG;
+    if (d->T > kDecodeTMax) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(d->gate_up_fp8, 16) || !aligned(d->down_fp8, 16) || !aligned(d->shared_gate_up_fp8, 16) ||
+        !aligned(d->shared_down_fp8, 16) || !aligned(d->gate_up_scale, 4) || !aligned(d->down_scale, 4) ||
+        !aligned(d->shared_gate_up_scale, 4) || !aligned(d->shared_down_scale, 4))
+      return MOE_ERR_ALIGNMENT;
+  } else {
     return MOE_ERR_INVALID_ARG;
+  }
   if ((d->flags & ~(MOE_FLAG_FORCE_PREFILL | MOE_FLAG_FORCE_DECODE)) != 0) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_FORCE_PREFILL) && (d->flags & MOE_FLAG_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_FORCE_DECODE) && d->T > kDecodeTMax) return MOE_ERR_INVALID_ARG;
@@ -173,15 +191,45 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
   MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
                                     Fp(w.topk_w), s));
   if (ev) MOE_CUDA_TRY(record(ev[1]));
-  MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), x, T, D, E, k, I(w.counts), I(w.offsets),
-                              I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), H(w.x_perm), I(w.scratch), err, s,
-                              nullptr));
+  const bool fp8 = d->weight_format == MOE_WEIGHTS_FP8_E4M3;
+  MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), fp8 ? nullptr : x, T, D, E, k, I(w.counts),
+                              I(w.offsets), I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), fp8 ? nullptr : H(w.x_perm),
+                              I(w.scratch), err, s, nullptr));
+  if (fp8) {
+    MOE_CUDA_TRY(launch_gather_rows_f16(x, I(w.perm_token), I(w.offsets), E, T, D, H(w.x_perm), s));
+    if (Fs > 0) MOE_CUDA_TRY(launch_cast_bf16_to_f16(x, (long long)T * D, H(w.x16), s));
+  }
   if (ev) MOE_CUDA_TRY(record(ev[2]));
   const int nt = use_decode(*d) ? decode_tile(T) : 0;
+  if (fp8) {
+    GemmSetHost g[2];
+    memset(g, 0, sizeof(g));
+    const float* gs[2] = {d->gate_up_scale, d->shared_gate_up_scale};
+    g[0].K = D, g[0].a = H(w.x_perm), g[0].a_rows = M, g[0].w = reinterpret_cast<const uint16_t*>(d->gate_up_fp8);
+    g[0].n_groups = E, g[0].offsets = I(w.offsets), g[0].n_out = F, g[0].out = H(w.h);
+    if (Fs > 0) {
+      g[1].K = D, g[1].a = H(w.x16), g[1].a_rows = T, g[1].w = reinterpret_cast<const uint16_t*>(d->shared_gate_up_fp8);
+      g[1].n_groups = 1, g[1].m_rows = T, g[1].n_out = Fs, g[1].out = H(w.h_sh);
+    }
+    MOE_CUDA_TRY(launch_stream_fp8w(kGateUp, g, gs, Fs > 0 ? 2 : 1, nt, err, s));
+    if (ev) MOE_CUDA_TRY(record(ev[3]));
+    GemmSetHost dn[2];
+    memset(dn, 0, sizeof(dn));
+    const float* ds[2] = {d->down_scale, d->shared_down_scale};
+    dn[0].K = F, dn[0].a = H(w.h), dn[0].a_rows = M, dn[0].w = reinterpret_cast<const uint16_t*>(d->down_fp8);
+    dn[0].n_groups = E, dn[0].offsets = I(w.offsets), dn[0].n_out = D, dn[0].out = Fp(w.out_perm);
+    dn[0].row_scale = Fp(w.p_perm);
+    if (Fs > 0) {
+      dn[1].K = Fs, dn[1].a = H(w.h_sh), dn[1].a_rows = T, dn[1].w = reinterpret_cast<const uint16_t*>(d->shared_down_fp8);
+      dn[1].n_groups = 1, dn[1].m_rows = T, dn[1].n_out = D, dn[1].out = Fp(w.out_sh);
+    }
+    MOE_CUDA_TRY(launch_stream_fp8w(kDown, dn, ds, Fs > 0 ? 2 : 1, nt, err, s));
+  } else {
   st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), Fp(w.out_perm), x,
                T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, err, s, ev ? ev[3] : nullptr,
                rec_flags);
   if (st != MOE_OK) return st;
+  }
   if (ev) MOE_CUDA_TRY(record(ev[4]));
   MOE_CUDA_TRY(launch_combine(Fp(w.out_perm), I(w.inv_perm), Fs > 0 ? Fp(w.out_sh) : nullptr, T, D, k, y, s));
   if (ev) MOE_CUDA_TRY(record(ev[5]));
@@ -230,6 +278,17 @@ moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, cons
   cudaStream_t s = (cudaStream_t)stream;
   MOE_CUDA_TRY(launch_router_gemm(x, w_gate, T, D, E, part, router_ld(E), splits, reinterpret_cast<int*>(b), s));
   MOE_CUDA_TRY(launch_router_select(part, splits, T, router_ld(E), bias, E, k, topk_idx, topk_w, s));
+  return MOE_OK;
+}
+
+moe_status_t moe_quantize_rows_fp8(const moe_bf16_t* w, int64_t rows, int K, uint8_t* q, float* scales,
+                                   moe_stream_t stream) {
+  if (!w || !q || !scales || rows < 0 || K <= 0) return MOE_ERR_INVALID_ARG;
+  if (K % 64 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(w, 16) || !aligned(q, 16) || !aligned(scales, 4)) return MOE_ERR_ALIGNMENT;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  MOE_CUDA_TRY(launch_quantize_rows_fp8(w, rows, K, q, scales, (cudaStream_t)stream));
   return MOE_OK;
 }
 
@@ -341,7 +400,8 @@ moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16
 int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK || desc->T == 0) return 0;
   const int dispatch = desc->T <= 256 ? 1 /*fused hist+scan+scatter*/ : 3 /*hist, scan, scatter*/;
-  return 2 /*router GEMM, top-k*/ + dispatch + 1 /*gather*/ + 2 /*grouped GEMMs*/ + 1 /*combine*/;
+  const int cast = (desc->weight_format == MOE_WEIGHTS_FP8_E4M3 && desc->Fs > 0) ? 1 : 0;  // x -> f16
+  return 2 /*router GEMM, top-k*/ + dispatch + 1 /*gather*/ + cast + 2 /*grouped GEMMs*/ + 1 /*combine*/;
 }
 
 moe_status_t moe_update_router_bias(const int32_t* counts, int E, float gamma, float* bias, moe_stream_t stream) {

@@ -13,6 +13,8 @@
 //   4. gather  : x_perm[r] = x[perm_token[r]], one warp per row, 16-byte vector moves
 // For T <= 256 steps 1-3 run as one single-block kernel (dispatch_small_kernel).
 // Within an expert, rows are therefore ordered by token id (a token picks an expert at most once).
+#include <cuda_fp16.h>
+
 #include "moe_common.cuh"
 
 namespace moe {
@@ -218,6 +220,45 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   pdl_trigger();
 }
 
+// bf16 -> f16 for 8 values (the FP8-weight GEMMs take f16 activations)
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 q) {
+  const uint32_t in[4] = {q.x, q.y, q.z, q.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = __floats2half2_rn(bf16_lo(in[i]), bf16_hi(in[i]));
+    o[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// x_perm16[r] = f16(x[perm_token[r]]) for r < offsets[E]; one warp per row.
+__global__ void __launch_bounds__(256) gather_rows_f16_kernel(const uint16_t* __restrict__ x,
+                                                              const int32_t* __restrict__ perm_token,
+                                                              const int32_t* __restrict__ offsets, int E, int T,
+                                                              int D, uint16_t* __restrict__ x_perm16) {
+  pdl_wait();
+  const int n_rows = offsets[E];
+  const int lane = threadIdx.x & 31;
+  const int nv = D / 8;
+  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n_rows; r += (gridDim.x * blockDim.x) >> 5) {
+    const int t = perm_token[r];
+    if ((unsigned)t >= (unsigned)T) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm16 + (size_t)r * D);
+    for (int v = lane; v < nv; v += 32) dst[v] = bf16x8_to_f16x8(__ldg(src + v));
+  }
+  pdl_trigger();
+}
+
+__global__ void __launch_bounds__(256) cast_bf16_to_f16_kernel(const uint16_t* __restrict__ src, long long n8,
+                                                               uint16_t* __restrict__ dst) {
+  pdl_wait();
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x)
+    reinterpret_cast<uint4*>(dst)[i] = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(src) + i));
+  pdl_trigger();
+}
+
 }  // namespace
 
 size_t permute_scratch_bytes(int T, int E) {
@@ -263,6 +304,23 @@ cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16
   }
   if (n_launches) *n_launches = launches;
   return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows_f16(const uint16_t* x, const int32_t* perm_token, const int32_t* offsets, int E,
+                                   int T, int D, uint16_t* x_perm16, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  long long blocks = ((long long)T * 32 + 7) / 8;  // T*k rows at most; k <= 32
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  return launch_pdl(gather_rows_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, perm_token, offsets, E, T,
+                    D, x_perm16);
+}
+
+cudaError_t launch_cast_bf16_to_f16(const uint16_t* src, long long n, uint16_t* dst, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const long long n8 = n / 8;
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 148LL * 8) blocks = 148LL * 8;
+  return launch_pdl(cast_bf16_to_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, src, n8, dst);
 }
 
 }  // namespace moe

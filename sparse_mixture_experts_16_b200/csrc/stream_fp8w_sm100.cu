@@ -1,0 +1,506 @@
+// stream_fp8w_sm100.cu -- weight-streaming (decode) grouped GEMMs with E4M3 expert weights.
+//
+// The decode path of the layer reads every active expert's weights once, so its time is the
+// weight bytes over HBM bandwidth (keryc.com "Mixture of Experts optimiza...", section "Por que
+// MoEs importan": decode speed = bandwidth / active bytes).  Storing the weights as E4M3 codes
+// with one fp32 scale per row (quantize_fp8.cu; the pages' per-expert quantisation, section
+// "Resultados practicos") halves those bytes.
+//
+// Same maths and tiling as the bf16 weight-streaming kernels in grouped_gemm_sm100.cu (swap-AB:
+// 128 weight rows of one active expert are the MMA M operand, the <= NT tokens routed to it the N
+// operand), with three differences:
+//   * the weight tiles arrive as E4M3 bytes (TMA, no swizzle) and four converter warps turn them
+//     into f16 tiles in the 128-byte-swizzled K-major layout the MMA reads (E4M3 values are
+//     exact in f16); the tensor cores run kind::f16 with f16 A and B;
+//   * the activations (x rows, and h between the two GEMMs) are f16, so A and B share a type;
+//   * the epilogue multiplies each accumulator row by its weight row's scale (TMEM lane = weight
+//     row), before the SwiGLU (gate_up) or together with the router weight (down).
+// Warp roles: 0 TMA producer, 1 MMA issuer (+TMEM), 2-5 epilogue, 6-9 converters.  All waits are
+// bounded as in the bf16 kernels.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "moe_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;            // MMA M: weight rows per unit
+constexpr int kBK = 64;             // K per stage
+constexpr int kThreads = 320;       // 10 warps
+constexpr int kConvThreads = 128;   // warps 6..9
+constexpr int kMaxGroups = 1025;
+constexpr int kRawW = kBM * kBK;    // one E4M3 weight tile: 128 rows x 64 bytes = 8 KB
+constexpr int kConvW = kBM * kBK * 2;  // the same tile in f16: 16 KB
+constexpr int kBarBytes = 512;
+
+struct alignas(64) Fp8Params {
+  CUtensorMap a_map[2];  // f16 activations [rows, K], 128-byte swizzle, box {64, NT}
+  CUtensorMap w_map[2];  // E4M3 weights [groups * w_rows, K], no swizzle, box {64 bytes, 128}
+  const float* w_scale[2];  // per weight row
+  const int32_t* offsets[2];
+  void* out[2];             // gate_up: f16 h [rows, F]; down: fp32 [rows, D]
+  const float* row_scale[2];
+  int n_groups[2];
+  int m_rows[2];
+  int n_out[2];
+  int w_rows[2];
+  int k_blocks[2];
+  int n_sets;
+  int withhold_first_load;
+  int* err;
+};
+
+// f16 MMA inputs (A and B formats 0 = F16), fp32 accumulator
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+template <int KIND, int NT>
+struct Fp8Cfg {
+  static constexpr int kW = KIND == kGateUp ? 2 : 1;             // weight tiles per stage
+  static constexpr int kActBytes = NT * kBK * 2;                  // f16 activation tile
+  static constexpr int kRawStage = kActBytes + kW * kRawW;        // TMA target: [act | w0 | w1]
+  static constexpr int kConvStage = kW * kConvW;                  // converter target: [w0 | w1]
+  static constexpr int kRawStages = KIND == kGateUp ? 6 : 8;
+  static constexpr int kConvStages = 2;
+  static constexpr int kAccCols = kW * NT;
+  static constexpr int kTmemCols = (2 * kAccCols <= 32) ? 32 : (2 * kAccCols <= 64) ? 64
+                                 : (2 * kAccCols <= 128) ? 128 : 256;
+  static constexpr uint32_t kIdesc = idesc_f16_f32(kBM, NT);
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kRawStages * kRawStage + (size_t)kConvStages * kConvStage +
+                                       kBarBytes + 4 * (kMaxGroups + 1);
+  static_assert(kRawStage % 1024 == 0 && kConvStage % 1024 == 0, "1024-byte aligned stages");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+struct Unit {
+  int set, gl, row0, rows, n;
+};
+
+__device__ __forceinline__ void unit_rows(const Fp8Params& p, int s, int gl, int& row0, int& rows) {
+  if (p.offsets[s] != nullptr) {
+    row0 = p.offsets[s][gl];
+    rows = p.offsets[s][gl + 1] - row0;
+  } else {
+    row0 = 0;
+    rows = p.m_rows[s];
+  }
+}
+
+__device__ __forceinline__ Unit decode_unit(const Fp8Params& p, const int* unit_start, int G, int t) {
+  int lo = 0, hi = G - 1;  // largest g with unit_start[g] <= t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (unit_start[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  Unit u;
+  u.set = lo < p.n_groups[0] ? 0 : 1;
+  u.gl = u.set == 0 ? lo : lo - p.n_groups[0];
+  unit_rows(p, u.set, u.gl, u.row0, u.rows);
+  u.n = t - unit_start[lo];
+  return u;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+// make the converters' ordinary shared-memory stores visible to the tensor cores
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16 E4M3 codes (one 16-byte word) -> 16 f16 values (two 16-byte words); E4M3 is exact in f16
+__device__ __forceinline__ void e4m3x16_to_f16(const uint4 in, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xFFFFu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
+    o[2 * i] = (uint32_t)a.x | ((uint32_t)a.y << 16);
+    o[2 * i + 1] = (uint32_t)b.x | ((uint32_t)b.y << 16);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <int KIND, int NT>
+__global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_constant__ Fp8Params p) {
+  using C = Fp8Cfg<KIND, NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* raw_base = smem;
+  uint8_t* conv_base = smem + C::kRawStages * C::kRawStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(conv_base + C::kConvStages * C::kConvStage);
+  uint64_t* empty = full + C::kRawStages;
+  uint64_t* cfull = empty + C::kRawStages;
+  uint64_t* cempty = cfull + C::kConvStages;
+  uint64_t* acc_full = cempty + C::kConvStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  int* unit_start = reinterpret_cast<int*>(conv_base + C::kConvStages * C::kConvStage + kBarBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.n_groups[0] + (p.n_sets > 1 ? p.n_groups[1] : 0);
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::kRawStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < C::kConvStages; ++s) {
+      mbar_init(&cfull[s], kConvThreads / 32);
+      mbar_init(&cempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    fence_barrier_init();
+    prefetch_tensormap(&p.a_map[0]);
+    prefetch_tensormap(&p.w_map[0]);
+    if (p.n_sets > 1) {
+      prefetch_tensormap(&p.a_map[1]);
+      prefetch_tensormap(&p.w_map[1]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  pdl_wait();
+  pdl_trigger();
+  // units (one per active group and 128-row weight block), then an exclusive scan
+  for (int g = threadIdx.x; g < G; g += kThreads) {
+    const int s = g < p.n_groups[0] ? 0 : 1;
+    const int gl = s == 0 ? g : g - p.n_groups[0];
+    int row0, rows;
+    unit_rows(p, s, gl, row0, rows);
+    if (rows > NT) set_error(p.err, kErrBadIndex);  // a segment longer than the token tile
+    unit_start[g] = rows > 0 ? (p.n_out[s] + kBM - 1) / kBM : 0;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int lo = lane * per, hi = min(G, lo + per);
+    int sum = 0;
+    for (int g = lo; g < hi; ++g) sum += unit_start[g];
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - sum;
+    for (int g = lo; g < hi; ++g) {
+      const int c = unit_start[g];
+      unit_start[g] = run;
+      run += c;
+    }
+    if (lane == 31) unit_start[G] = incl;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = unit_start[G];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Unit u = decode_unit(p, unit_start, G, t);
+        const int wbase = u.gl * p.w_rows[u.set];
+        for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
+          const int st = it % C::kRawStages;
+          if (!mbar_wait(&empty[st], ((it / C::kRawStages) & 1) ^ 1, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = raw_base + st * C::kRawStage;
+          mbar_arrive_expect_tx(&full[st], C::kRawStage);
+          if (p.withhold_first_load && it == 0) continue;  // test only: the bytes never arrive
+          const int kx = kb * kBK;
+          tma_load_2d(&p.a_map[u.set], &full[st], sb, kx, u.row0);
+          tma_load_2d(&p.w_map[u.set], &full[st], sb + C::kActBytes, kx, wbase + u.n * kBM);
+          if constexpr (KIND == kGateUp)
+            tma_load_2d(&p.w_map[u.set], &full[st], sb + C::kActBytes + kRawW, kx,
+                        wbase + p.n_out[u.set] + u.n * kBM);
+        }
+      }
+      if (!ok) set_error(p.err, kErrTimeout);
+      const uint32_t issued = it;
+      for (int s = 0; s < C::kRawStages; ++s) {
+        if ((uint32_t)s >= issued) break;
+        const uint32_t last = issued - 1 - ((issued - 1 - s) % C::kRawStages);
+        if (!mbar_wait(&full[s], (last / C::kRawStages) & 1, kWaitLimitNs)) set_error(p.err, kErrTimeout);
+      }
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------------ E4M3 -> f16 converters
+    const int ct = threadIdx.x - 6 * 32;  // 0..127
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const Unit u = decode_unit(p, unit_start, G, t);
+      for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
+        const int st = it % C::kRawStages, cs = it % C::kConvStages;
+        if (!mbar_wait(&full[st], (it / C::kRawStages) & 1, kWaitLimitNs) ||
+            !mbar_wait(&cempty[cs], ((it / C::kConvStages) & 1) ^ 1, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* src = raw_base + st * C::kRawStage + C::kActBytes;
+        uint8_t* dst = conv_base + cs * C::kConvStage;
+#pragma unroll
+        for (int w = 0; w < C::kW; ++w) {
+          // 128 rows x 4 sixteen-byte chunks; chunk j of row r becomes output chunks 2j, 2j+1 of the
+          // 128-byte f16 row, placed at (chunk ^ (r & 7)) as the 128-byte swizzle requires
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int c = ct + i * kConvThreads;
+            const int r = c >> 2, j = c & 3;
+            const uint4 in = *reinterpret_cast<const uint4*>(src + w * kRawW + r * kBK + j * 16);
+            uint4 lo, hi;
+            e4m3x16_to_f16(in, lo, hi);
+            uint8_t* row = dst + w * kConvW + r * 128;
+            *reinterpret_cast<uint4*>(row + (((2 * j) ^ (r & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(row + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cfull[cs]);
+      }
+    }
+    if (!ok) set_error(p.err, kErrTimeout);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tl = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tl) {
+        const uint32_t buf = tl & 1, use = tl >> 1;
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * C::kAccCols;
+        const Unit u = decode_unit(p, unit_start, G, t);
+        for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
+          const int st = it % C::kRawStages, cs = it % C::kConvStages;
+          if (!mbar_wait(&full[st], (it / C::kRawStages) & 1, kWaitLimitNs) ||
+              !mbar_wait(&cfull[cs], (it / C::kConvStages) & 1, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(raw_base + st * C::kRawStage);  // activations (B)
+          const uint32_t sw = smem_u32(conv_base + cs * C::kConvStage);  // f16 weights (A)
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0;
+            const uint64_t bdesc = sw128_kmajor_desc(sa + kk * 32);
+            umma_bf16(d, sw128_kmajor_desc(sw + kk * 32), bdesc, C::kIdesc, acc);
+            if constexpr (KIND == kGateUp)
+              umma_bf16(d + NT, sw128_kmajor_desc(sw + kConvW + kk * 32), bdesc, C::kIdesc, acc);
+          }
+          umma_commit(&empty[st]);   // the raw stage (and its activation tile) is free
+          umma_commit(&cempty[cs]);  // the converted stage is free
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+      }
+      if (!ok) set_error(p.err, kErrTimeout);
+      if (it > 0) {
+        const uint32_t last = it - 1;
+        if (!mbar_wait(&cempty[last % C::kConvStages], (last / C::kConvStages) & 1, kWaitLimitNs))
+          set_error(p.err, kErrTimeout);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    uint32_t tl = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tl) {
+      const uint32_t buf = tl & 1, use = tl >> 1;
+      if (!mbar_wait(&acc_full[buf], use & 1, kWaitLimitNs)) {
+        set_error(p.err, kErrTimeout);
+        break;
+      }
+      tc_fence_after();
+      const Unit u = decode_unit(p, unit_start, G, t);
+      const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * C::kAccCols;
+      const int n_out = p.n_out[u.set];
+      const int wbase = u.gl * p.w_rows[u.set];
+      const int col = u.n * kBM + q * 32 + lane;  // output column = weight row within the group
+      const bool col_ok = col < n_out;
+      const float* ws = p.w_scale[u.set];
+      if constexpr (KIND == kGateUp) {
+        const float sg = col_ok ? ws[wbase + col] : 0.f, su = col_ok ? ws[wbase + n_out + col] : 0.f;
+        __half* out_h = static_cast<__half*>(p.out[u.set]);
+#pragma unroll 1
+        for (int j0 = 0; j0 < NT; j0 += 16) {
+          if (j0 >= u.rows) break;
+          uint32_t g[16], v[16];
+          tmem_ld_32x32b_x16(tacc + j0, g);
+          tmem_ld_32x32b_x16(tacc + NT + j0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = j0 + jj;
+            if (j < u.rows && col_ok)
+              out_h[(size_t)(u.row0 + j) * n_out + col] =
+                  __float2half_rn(silu_mul(__uint_as_float(g[jj]) * sg, __uint_as_float(v[jj]) * su));
+          }
+        }
+      } else {
+        const float sd = col_ok ? ws[wbase + col] : 0.f;
+        const float* rs = p.row_scale[u.set];
+        float* out_f = static_cast<float*>(p.out[u.set]);
+#pragma unroll 1
+        for (int j0 = 0; j0 < NT; j0 += 16) {
+          if (j0 >= u.rows) break;
+          uint32_t a[16];
+          tmem_ld_32x32b_x16(tacc + j0, a);
+          tmem_ld_wait();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = j0 + jj;
+            if (j < u.rows && col_ok)
+              out_f[(size_t)(u.row0 + j) * n_out + col] =
+                  __uint_as_float(a[jj]) * sd * (rs != nullptr ? rs[u.row0 + j] : 1.0f);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D row-major [rows, cols] map; box = box_cols x box_rows elements
+bool make_map(CUtensorMap* m, CUtensorMapDataType type, int elem_bytes, const void* base, uint64_t rows,
+              uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int KIND, int NT>
+cudaError_t launch_fp8(const GemmSetHost* sets, const float* const* scales, int n_sets, int* err, cudaStream_t s) {
+  using C = Fp8Cfg<KIND, NT>;
+  Fp8Params p;
+  memset(&p, 0, sizeof(p));
+  p.n_sets = n_sets;
+  p.err = err;
+  const char* hold = getenv("MOE_TEST_WITHHOLD_LOAD");
+  p.withhold_first_load = (hold != nullptr && hold[0] == '1') ? 1 : 0;
+  for (int i = 0; i < n_sets; ++i) {
+    const GemmSetHost& st = sets[i];
+    const int K = st.K;
+    p.k_blocks[i] = K / kBK;
+    p.w_rows[i] = KIND == kGateUp ? 2 * st.n_out : st.n_out;
+    if (!make_map(&p.a_map[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, st.a, (uint64_t)st.a_rows, (uint64_t)K, kBK, NT,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    if (!make_map(&p.w_map[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, st.w, (uint64_t)st.n_groups * p.w_rows[i],
+                  (uint64_t)K, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    p.w_scale[i] = scales[i];
+    p.offsets[i] = st.offsets;
+    p.out[i] = st.out;
+    p.row_scale[i] = st.row_scale;
+    p.n_groups[i] = st.n_groups;
+    p.m_rows[i] = st.m_rows;
+    p.n_out[i] = st.n_out;
+  }
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(stream_fp8w_kernel<KIND, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  return launch_pdl(stream_fp8w_kernel<KIND, NT>, dim3(sm_count()), dim3(kThreads), C::kSmemBytes, s, p);
+}
+
+template <int KIND>
+cudaError_t launch_kind(const GemmSetHost* sets, const float* const* scales, int n_sets, int nt, int* err,
+                        cudaStream_t s) {
+  switch (nt) {
+    case 16: return launch_fp8<KIND, 16>(sets, scales, n_sets, err, s);
+    case 32: return launch_fp8<KIND, 32>(sets, scales, n_sets, err, s);
+    case 48: return launch_fp8<KIND, 48>(sets, scales, n_sets, err, s);
+    case 64: return launch_fp8<KIND, 64>(sets, scales, n_sets, err, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_stream_fp8w(GemmKind kind, const GemmSetHost* sets, const float* const* w_scales, int n_sets,
+                               int decode_nt, int* err, cudaStream_t s) {
+  if (n_sets < 1 || n_sets > 2) return cudaErrorInvalidValue;
+  int groups = 0;
+  for (int i = 0; i < n_sets; ++i) {
+    if (sets[i].K <= 0 || sets[i].K % kBK != 0 || w_scales[i] == nullptr) return cudaErrorInvalidValue;
+    groups += sets[i].n_groups;
+  }
+  if (groups > kMaxGroups) return cudaErrorInvalidValue;
+  if (kind == kGateUp) return launch_kind<kGateUp>(sets, w_scales, n_sets, decode_nt, err, s);
+  if (kind == kDown) return launch_kind<kDown>(sets, w_scales, n_sets, decode_nt, err, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

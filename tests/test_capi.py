@@ -47,7 +47,9 @@ def test_status_strings(L):
 
 def _desc(**kw):
     base = dict(T=16, D=128, E=8, k=2, F=128, Fs=0, w_gate=0x1000, bias=None, gate_up=0x2000, down=0x3000,
-                shared_gate_up=None, shared_down=None, flags=0)
+                shared_gate_up=None, shared_down=None, flags=0, weight_format=0, gate_up_fp8=None,
+                gate_up_scale=None, down_fp8=None, down_scale=None, shared_gate_up_fp8=None,
+                shared_gate_up_scale=None, shared_down_fp8=None, shared_down_scale=None)
     base.update(kw)
     return moe.LayerDesc(*[base[n] for n, _ in moe.LayerDesc._fields_])
 
@@ -150,3 +152,35 @@ def test_bias_update_and_counts_validate_on_host(L):
     assert L.moe_layer_expert_counts(ctypes.byref(d), 0x100000, need, ctypes.byref(ptr)) == 0
     assert 0x100000 < ptr.value < 0x100000 + need and ptr.value % 256 == 0
     assert L.moe_layer_expert_counts(ctypes.byref(d), 0x100000, need - 1, ctypes.byref(ptr)) == 4
+
+
+FP8 = dict(weight_format=1, gate_up=None, down=None, gate_up_fp8=0x8000, gate_up_scale=0x9000, down_fp8=0xA000,
+           down_scale=0xB000)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), 0),                                   # valid (reaches the device check or the no-GPU status)
+    (dict(weight_format=2), 1),
+    (dict(gate_up_scale=None), 1),
+    (dict(T=65), 2),                               # FP8 weights run the decode kernels only
+    (dict(flags=1), 1),                            # ... so forcing the tiled kernels is invalid
+    (dict(Fs=64, shared_gate_up_fp8=0xC000, shared_down_fp8=0xD000, shared_gate_up_scale=0xE000), 1),
+    (dict(gate_up_fp8=0x8008), 3),
+    (dict(down_scale=0xB002), 3),
+])
+def test_fp8_descriptor_validation(L, kw, status):
+    d = _desc(**{**FP8, **kw})
+    st = L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, 1 << 30, None)
+    if status == 0:
+        assert st in (0, 8) and L.moe_layer_workspace_size(ctypes.byref(d)) > 0
+    else:
+        assert st == status, moe.STATUS.get(st)
+
+
+def test_fp8_kernel_count_and_quantizer_validation(L):
+    d = _desc(**FP8, Fs=64, shared_gate_up_fp8=0xC000, shared_down_fp8=0xD000, shared_gate_up_scale=0xE000,
+              shared_down_scale=0xF000)
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 8  # + the f16 cast of x for the shared expert
+    assert L.moe_quantize_rows_fp8(None, 4, 64, 0x2000, 0x3000, None) == 1
+    assert L.moe_quantize_rows_fp8(0x1000, 4, 100, 0x2000, 0x3000, None) == 2
+    assert L.moe_quantize_rows_fp8(0x1008, 4, 64, 0x2000, 0x3000, None) == 3
