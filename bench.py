@@ -85,10 +85,15 @@ def down_flops(w: mi.Workload) -> float:
     return float(w.T) * (w.k * 2.0 * w.D * w.F + 2.0 * w.D * w.Fs)
 
 
-def active_weight_bytes(w: mi.Workload, n_active: int, part: str = "all") -> float:
-    """Bytes of weights that must be streamed: distinct active experts (+ shared expert)."""
-    gu = 2.0 * w.F * w.D * 2 * n_active + 2.0 * w.Fs * w.D * 2
-    dn = 1.0 * w.D * w.F * 2 * n_active + 1.0 * w.D * w.Fs * 2
+def active_weight_bytes(w: mi.Workload, n_active: int, part: str = "all", weights: str = "bf16") -> float:
+    """Bytes of weights that must be streamed: distinct active experts (+ shared expert).  bf16: 2
+    bytes per weight; fp8: 1 byte per E4M3 code plus a 4-byte scale per weight row."""
+    if weights == "fp8":
+        gu = (2.0 * w.F * w.D + 4 * 2.0 * w.F) * n_active + (2.0 * w.Fs * w.D + 4 * 2.0 * w.Fs)
+        dn = (1.0 * w.D * w.F + 4.0 * w.D) * n_active + ((1.0 * w.D * w.Fs + 4.0 * w.D) if w.Fs else 0.0)
+    else:
+        gu = 2.0 * w.F * w.D * 2 * n_active + 2.0 * w.Fs * w.D * 2
+        dn = 1.0 * w.D * w.F * 2 * n_active + 1.0 * w.D * w.Fs * 2
     return {"gate_up": gu, "down": dn, "all": gu + dn}[part]
 
 
@@ -163,9 +168,10 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------- CPU oracle
-def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, max_experts: int = 40):
+def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, max_experts: int = 40, weights: str = "bf16"):
     """The fp64 oracle, as it stands, on a bounded sample of the workload's tokens (all host
-    cores).  Returns (tokens/s, cores, description)."""
+    cores; with fp8 weights the oracle's E4M3 layer on weights it quantised itself, outside the
+    timed calls).  Returns (tokens/s, cores, description)."""
     import oracle
 
     cores = host_cores()
@@ -187,6 +193,19 @@ def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, max_experts: int = 4
     gu = dict(zip(experts, mi.host_gate_up(w, experts)))
     dn = dict(zip(experts, mi.host_down(w, experts)))
     sgu, sdn = mi.host_shared(w)
+    if weights == "fp8":
+        q = dict(gu_q={}, gu_s={}, dn_q={}, dn_s={})
+        for e in experts:
+            q["gu_q"][e], q["gu_s"][e] = oracle.quantize_rows_fp8(gu[e])
+            q["dn_q"][e], q["dn_s"][e] = oracle.quantize_rows_fp8(dn[e])
+        shared_q = None
+        if w.Fs:
+            a, b = oracle.quantize_rows_fp8(sgu)
+            c, d = oracle.quantize_rows_fp8(sdn)
+            shared_q = dict(gu_q=a, gu_s=b, dn_q=c, dn_s=d)
+        run = lambda x: oracle.layer_fp8(x, wg, bias, w.k, q, shared_q)  # noqa: E731
+    else:
+        run = lambda x: oracle.layer(x, wg, bias, gu, dn, w.k, sgu, sdn, nthreads=cores)  # noqa: E731
     chosen = np.array(chosen)
     # time a growing number of tokens until the budget is reached
     n, done, elapsed = min(len(chosen), cores), 0, 0.0
@@ -194,7 +213,7 @@ def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, max_experts: int = 4
         rows = chosen[np.arange(done, done + n) % len(chosen)]
         x = xp[rows]
         t0 = time.perf_counter()
-        oracle.layer(x, wg, bias, gu, dn, w.k, sgu, sdn, nthreads=cores)
+        run(x)
         dt = time.perf_counter() - t0
         done += n
         elapsed += dt
@@ -202,7 +221,8 @@ def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, max_experts: int = 4
             break
         n = max(1, int(n * min(4.0, max(1.5, (budget_s - elapsed) / max(dt, 1e-3)))))
     desc = (f"{done} tokens of workload {w.name} (full layer: routing over all E experts, top-{w.k} SwiGLU experts"
-            f"{', shared expert' if w.Fs else ''}) through the fp64 oracle on {cores} threads; tokens/s = "
+            f"{', shared expert' if w.Fs else ''}{', E4M3 weights' if weights == 'fp8' else ''}) through the "
+            f"fp64 oracle on {cores} threads; tokens/s = "
             f"{done} / {elapsed:.2f} s")
     return done / elapsed, cores, desc
 
@@ -222,8 +242,18 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     pk, pk_kind = peaks()
     with torch.cuda.stream(stream):
         inp = mi.device_inputs(w, device=dev)
+        if args.weights == "fp8":
+            # per-row E4M3 codes + fp32 scales, made on the device before timing; the bf16 copies go
+            scales = {}
+            for name in ("gate_up", "down", "shared_gate_up", "shared_down"):
+                if inp[name] is not None:
+                    inp[name], scales[name] = moe.moe_quantize_rows_fp8(inp[name], stream=stream)
+            stream.synchronize()
+            torch.cuda.empty_cache()
+        else:
+            scales = None
         layer = moe.MoELayer(inp["wg"], inp["gate_up"], inp["down"], w.k, bias=inp["bias"],
-                             shared_gate_up=inp["shared_gate_up"], shared_down=inp["shared_down"])
+                             shared_gate_up=inp["shared_gate_up"], shared_down=inp["shared_down"], scales=scales)
         x = inp["x"]
         y = torch.empty_like(x)
         ws = layer.workspace(w.T)
@@ -328,11 +358,14 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     down_ms = statistics.mean(stage_ms[3])
     decode = w.T <= 64
     if decode:
-        bytes_gu = active_weight_bytes(w, n_active, "gate_up") + w.T * w.k * w.D * 2.0 + w.T * (w.k * w.F + w.Fs) * 2.0
+        bytes_gu = (active_weight_bytes(w, n_active, "gate_up", args.weights) + w.T * w.k * w.D * 2.0
+                    + w.T * (w.k * w.F + w.Fs) * 2.0)
         achieved = bytes_gu / (gate_ms / 1e3) / 1e9
         peak = pk["hbm_gbs"]
-        roof = {"kernel": "grouped_gemm_kernel<gate_up, stream>", "bound": "hbm", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name),
+        fp8 = args.weights == "fp8"
+        roof = {"kernel": "stream_fp8w_kernel<gate_up>" if fp8 else "grouped_gemm_kernel<gate_up, stream>",
+                "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None if fp8 else measured_traffic(w.name),
                 "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)"}
     else:
         achieved = gateup_flops(w) / (gate_ms / 1e3) / 1e12
@@ -342,14 +375,17 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
                 "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
                 "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4)}
     layer_tflops = w.flops / (ms_per_step / 1e3) / 1e12 * world
-    layer_gbs = active_weight_bytes(w, n_active) / (ms_per_step / 1e3) / 1e9
+    layer_gbs = active_weight_bytes(w, n_active, "all", args.weights) / (ms_per_step / 1e3) / 1e9
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": len(plain_ms),
         "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "ms_per_step_with_stage_events": round(staged_ms_per_step, 4),
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init weights)",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16" if args.weights == "fp8" else "bf16",
+        "data": "synthetic (seeded; random-init weights)",
         "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias,
+                   "weights": ("E4M3 codes + per-row fp32 scales (f16 MMA, fp32 accumulation)"
+                               if args.weights == "fp8" else "bf16"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": ("L2 flushed (256 MB write) before every timed step" if flush is not None
                           else f"inputs larger than L2 (weights {weight_bytes / 1e9:.2f} GB), no flush"),
@@ -371,7 +407,7 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     }
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
-            v, cores, desc = cpu_oracle_rate(w)
+            v, cores, desc = cpu_oracle_rate(w, weights=args.weights)
             result["cpu_baseline"] = {"value": round(v, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                       "sample": desc}
         print(json.dumps(result), flush=True)
@@ -386,7 +422,7 @@ def run_reference(args, w: mi.Workload, rank: int, world: int):
     desc = None
     budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for s in range(args.warmup + args.steps):
-        v, cores, desc = cpu_oracle_rate(w, budget_s=budget)
+        v, cores, desc = cpu_oracle_rate(w, budget_s=budget, weights=args.weights)
         if s >= args.warmup:
             steps.append(v)
     value = statistics.mean(steps)
@@ -395,7 +431,8 @@ def run_reference(args, w: mi.Workload, rank: int, world: int):
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; random-init weights)",
-        "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias},
+        "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias,
+                   "weights": "E4M3 codes + per-row fp32 scales" if args.weights == "fp8" else "bf16"},
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"per step: {desc}"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -410,8 +447,12 @@ def main():
     ap.add_argument("--workload", default="mixtral", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="expert weight format; fp8 (E4M3, per-row scales) runs the decode kernels, T <= 64")
     args = ap.parse_args()
     w = mi.WORKLOADS[args.workload]
+    if args.weights == "fp8" and w.T > 64:
+        ap.error(f"--weights fp8 is the decode path (T <= 64); workload {w.name} has T = {w.T}")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -6,20 +6,24 @@
 // with one fp32 scale per row (quantize_fp8.cu; the pages' per-expert quantisation, section
 // "Resultados practicos") halves those bytes.
 //
-// Same maths and tiling as the bf16 weight-streaming kernels in grouped_gemm_sm100.cu (swap-AB:
-// 128 weight rows of one active expert are the MMA M operand, the <= NT tokens routed to it the N
-// operand), with three differences:
-//   * the weight tiles arrive as E4M3 bytes (TMA, no swizzle) and four converter warps turn them
-//     into f16 tiles in the 128-byte-swizzled K-major layout the MMA reads (E4M3 values are
-//     exact in f16); the tensor cores run kind::f16 with f16 A and B;
-//   * the activations (x rows, and h between the two GEMMs) are f16, so A and B share a type;
+// Same maths as the bf16 weight-streaming kernels in grouped_gemm_sm100.cu (swap-AB: 128 weight
+// rows of one active expert are the MMA M operand, the <= NT tokens routed to it the N operand),
+// built around where the converted weights live:
+//   * TMA brings each stage's codes as 128 rows x 128 bytes (K = 128) with the 128-byte swizzle,
+//     and the f16 activations as two 64-column swizzled atoms;
+//   * eight converter warps read their weight rows from shared memory (conflict-free under the
+//     swizzle), turn the codes into f16 (exact) and store them with tcgen05.st straight into
+//     tensor memory, where the MMA takes its A operand.  Shared memory then carries 2 bytes per
+//     code (TMA write + converter read) instead of 6 with an f16 copy in shared memory, which is
+//     what bounded the first design well below HBM bandwidth;
+//   * the tensor cores run kind::f16 (f16 A from TMEM, f16 B from shared memory);
 //   * the epilogue multiplies each accumulator row by its weight row's scale (TMEM lane = weight
 //     row), before the SwiGLU (gate_up) or together with the router weight (down).
-// Warp roles: 0 TMA producer, 1 MMA issuer (+TMEM), 2-5 epilogue, 6-9 converters.  All waits are
-// bounded as in the bf16 kernels.
+// K need only be a multiple of 64: the last stage's columns past K are zero-filled by TMA.
+// Warp roles: 0 TMA producer, 1 MMA issuer (+TMEM owner), 2-5 epilogue, 6-13 converters (warp w
+// owns TMEM lanes 32*(w%4).. and K half (w-6)/4).  All waits are bounded as in the bf16 kernels.
 #include <cuda.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include <cstdlib>
 #include <cstring>
@@ -31,18 +35,17 @@
 namespace moe {
 namespace {
 
-constexpr int kBM = 128;            // MMA M: weight rows per unit
-constexpr int kBK = 64;             // K per stage
-constexpr int kThreads = 320;       // 10 warps
-constexpr int kConvThreads = 128;   // warps 6..9
+constexpr int kBM = 128;             // MMA M: weight rows per unit
+constexpr int kBK = 128;             // K per stage (codes: one 128-byte swizzle row)
+constexpr int kThreads = 448;        // 14 warps
+constexpr int kConvWarps = 8;        // warps 6..13
 constexpr int kMaxGroups = 1025;
-constexpr int kRawW = kBM * kBK;    // one E4M3 weight tile: 128 rows x 64 bytes = 8 KB
-constexpr int kConvW = kBM * kBK * 2;  // the same tile in f16: 16 KB
+constexpr int kRawW = kBM * kBK;     // one E4M3 weight tile: 128 rows x 128 bytes = 16 KB
 constexpr int kBarBytes = 512;
 
 struct alignas(64) Fp8Params {
   CUtensorMap a_map[2];  // f16 activations [rows, K], 128-byte swizzle, box {64, NT}
-  CUtensorMap w_map[2];  // E4M3 weights [groups * w_rows, K], no swizzle, box {64 bytes, 128}
+  CUtensorMap w_map[2];  // E4M3 weights [groups * w_rows, K], 128-byte swizzle, box {128 bytes, 128}
   const float* w_scale[2];  // per weight row
   const int32_t* offsets[2];
   void* out[2];             // gate_up: f16 h [rows, F]; down: fp32 [rows, D]
@@ -51,7 +54,7 @@ struct alignas(64) Fp8Params {
   int m_rows[2];
   int n_out[2];
   int w_rows[2];
-  int k_blocks[2];
+  int k_blocks[2];          // ceil(K / 128)
   int n_sets;
   int withhold_first_load;
   int* err;
@@ -62,21 +65,25 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
+
 template <int KIND, int NT>
 struct Fp8Cfg {
-  static constexpr int kW = KIND == kGateUp ? 2 : 1;             // weight tiles per stage
-  static constexpr int kActBytes = NT * kBK * 2;                  // f16 activation tile
-  static constexpr int kRawStage = kActBytes + kW * kRawW;        // TMA target: [act | w0 | w1]
-  static constexpr int kConvStage = kW * kConvW;                  // converter target: [w0 | w1]
-  static constexpr int kRawStages = KIND == kGateUp ? 6 : 8;
-  static constexpr int kConvStages = 2;
-  static constexpr int kAccCols = kW * NT;
-  static constexpr int kTmemCols = (2 * kAccCols <= 32) ? 32 : (2 * kAccCols <= 64) ? 64
-                                 : (2 * kAccCols <= 128) ? 128 : 256;
+  static constexpr int kW = KIND == kGateUp ? 2 : 1;      // weight tiles per stage
+  static constexpr int kAtom = NT * 128;                   // one f16 activation atom: NT rows x 64 K
+  static constexpr int kStage = 2 * kAtom + kW * kRawW;    // [act k0-63 | act k64-127 | w0 | w1]
+  static constexpr int kAccCols = kW * NT;                 // one accumulator buffer
+  static constexpr int kACol = 2 * kAccCols;               // A stages follow the two buffers
+  static constexpr int kAStageCols = kW * 64;              // 128 K of f16 per tile = 64 columns
+  static constexpr int kAStages = (512 - kACol) / kAStageCols >= 4 ? 4 : (512 - kACol) / kAStageCols;
+  static constexpr int kTmemCols = pow2_cols(kACol + kAStages * kAStageCols);
+  static constexpr int kRawBudget = 232448 - 1024 - kBarBytes - 4 * (kMaxGroups + 1);
+  static constexpr int kStages = kRawBudget / kStage >= 8 ? 8 : kRawBudget / kStage;
   static constexpr uint32_t kIdesc = idesc_f16_f32(kBM, NT);
-  static constexpr size_t kSmemBytes = 1024 + (size_t)kRawStages * kRawStage + (size_t)kConvStages * kConvStage +
-                                       kBarBytes + 4 * (kMaxGroups + 1);
-  static_assert(kRawStage % 1024 == 0 && kConvStage % 1024 == 0, "1024-byte aligned stages");
+  static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStage + kBarBytes + 4 * (kMaxGroups + 1);
+  static_assert(kStage % 1024 == 0, "1024-byte aligned stages");
+  static_assert(kAStages >= 2 && kStages >= 3, "pipeline depth");
+  static_assert(kACol + kAStages * kAStageCols <= 512, "tensor memory");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -110,53 +117,31 @@ __device__ __forceinline__ Unit decode_unit(const Fp8Params& p, const int* unit_
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-// make the converters' ordinary shared-memory stores visible to the tensor cores
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 16 E4M3 codes (one 16-byte word) -> 16 f16 values (two 16-byte words); E4M3 is exact in f16
-__device__ __forceinline__ void e4m3x16_to_f16(const uint4 in, uint4& lo, uint4& hi) {
-  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-  uint32_t o[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xFFFFu), __NV_E4M3);
-    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
-    o[2 * i] = (uint32_t)a.x | ((uint32_t)a.y << 16);
-    o[2 * i + 1] = (uint32_t)b.x | ((uint32_t)b.y << 16);
-  }
-  lo = make_uint4(o[0], o[1], o[2], o[3]);
-  hi = make_uint4(o[4], o[5], o[6], o[7]);
-}
-
 template <int KIND, int NT>
 __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_constant__ Fp8Params p) {
   using C = Fp8Cfg<KIND, NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* raw_base = smem;
-  uint8_t* conv_base = smem + C::kRawStages * C::kRawStage;
-  uint64_t* full = reinterpret_cast<uint64_t*>(conv_base + C::kConvStages * C::kConvStage);
-  uint64_t* empty = full + C::kRawStages;
-  uint64_t* cfull = empty + C::kRawStages;
-  uint64_t* cempty = cfull + C::kConvStages;
-  uint64_t* acc_full = cempty + C::kConvStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStage);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* afull = empty + C::kStages;  // converted A stage in TMEM ready (8 converter warps)
+  uint64_t* aempty = afull + C::kAStages;  // A stage consumed by the MMAs (tcgen05.commit)
+  uint64_t* acc_full = aempty + C::kAStages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  int* unit_start = reinterpret_cast<int*>(conv_base + C::kConvStages * C::kConvStage + kBarBytes);
+  int* unit_start = reinterpret_cast<int*>(smem + C::kStages * C::kStage + kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.n_groups[0] + (p.n_sets > 1 ? p.n_groups[1] : 0);
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < C::kRawStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int s = 0; s < C::kConvStages; ++s) {
-      mbar_init(&cfull[s], kConvThreads / 32);
-      mbar_init(&cempty[s], 1);
+    for (int s = 0; s < C::kAStages; ++s) {
+      mbar_init(&afull[s], kConvWarps);
+      mbar_init(&aempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -218,67 +203,72 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Unit u = decode_unit(p, unit_start, G, t);
-        const int wbase = u.gl * p.w_rows[u.set];
+        const int wrow = u.gl * p.w_rows[u.set] + u.n * kBM;
         for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
-          const int st = it % C::kRawStages;
-          if (!mbar_wait(&empty[st], ((it / C::kRawStages) & 1) ^ 1, kWaitLimitNs)) {
+          const int st = it % C::kStages;
+          if (!mbar_wait(&empty[st], ((it / C::kStages) & 1) ^ 1, kWaitLimitNs)) {
             ok = false;
             break;
           }
-          uint8_t* sb = raw_base + st * C::kRawStage;
-          mbar_arrive_expect_tx(&full[st], C::kRawStage);
+          uint8_t* sb = smem + st * C::kStage;
+          mbar_arrive_expect_tx(&full[st], C::kStage);
           if (p.withhold_first_load && it == 0) continue;  // test only: the bytes never arrive
           const int kx = kb * kBK;
           tma_load_2d(&p.a_map[u.set], &full[st], sb, kx, u.row0);
-          tma_load_2d(&p.w_map[u.set], &full[st], sb + C::kActBytes, kx, wbase + u.n * kBM);
+          tma_load_2d(&p.a_map[u.set], &full[st], sb + C::kAtom, kx + 64, u.row0);
+          tma_load_2d(&p.w_map[u.set], &full[st], sb + 2 * C::kAtom, kx, wrow);
           if constexpr (KIND == kGateUp)
-            tma_load_2d(&p.w_map[u.set], &full[st], sb + C::kActBytes + kRawW, kx,
-                        wbase + p.n_out[u.set] + u.n * kBM);
+            tma_load_2d(&p.w_map[u.set], &full[st], sb + 2 * C::kAtom + kRawW, kx, wrow + p.n_out[u.set]);
         }
       }
       if (!ok) set_error(p.err, kErrTimeout);
       const uint32_t issued = it;
-      for (int s = 0; s < C::kRawStages; ++s) {
+      for (int s = 0; s < C::kStages; ++s) {
         if ((uint32_t)s >= issued) break;
-        const uint32_t last = issued - 1 - ((issued - 1 - s) % C::kRawStages);
-        if (!mbar_wait(&full[s], (last / C::kRawStages) & 1, kWaitLimitNs)) set_error(p.err, kErrTimeout);
+        const uint32_t last = issued - 1 - ((issued - 1 - s) % C::kStages);
+        if (!mbar_wait(&full[s], (last / C::kStages) & 1, kWaitLimitNs)) set_error(p.err, kErrTimeout);
       }
     }
   } else if (warp >= 6) {
-    // ------------------------------------------------------------------ E4M3 -> f16 converters
-    const int ct = threadIdx.x - 6 * 32;  // 0..127
+    // ------------------------------------------------------------------ E4M3 -> f16 into TMEM
+    // Thread = weight row r of its quadrant; it converts the 64 codes of K half h of row r (four
+    // 16-byte chunks, placed by the 128-byte swizzle at chunk ^ (r & 7)) and stores them as 32
+    // f16x2 columns of TMEM lane r.
+    const int q = warp & 3, h = (warp - 6) >> 2;
+    const int r = 32 * q + lane;
+    const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const Unit u = decode_unit(p, unit_start, G, t);
       for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
-        const int st = it % C::kRawStages, cs = it % C::kConvStages;
-        if (!mbar_wait(&full[st], (it / C::kRawStages) & 1, kWaitLimitNs) ||
-            !mbar_wait(&cempty[cs], ((it / C::kConvStages) & 1) ^ 1, kWaitLimitNs)) {
+        const int st = it % C::kStages, as = it % C::kAStages;
+        if (!mbar_wait(&full[st], (it / C::kStages) & 1, kWaitLimitNs) ||
+            !mbar_wait(&aempty[as], ((it / C::kAStages) & 1) ^ 1, kWaitLimitNs)) {
           ok = false;
           break;
         }
-        const uint8_t* src = raw_base + st * C::kRawStage + C::kActBytes;
-        uint8_t* dst = conv_base + cs * C::kConvStage;
+        tc_fence_after();
+        const uint32_t src = smem_u32(smem + st * C::kStage + 2 * C::kAtom) + r * kBK;
 #pragma unroll
         for (int w = 0; w < C::kW; ++w) {
-          // 128 rows x 4 sixteen-byte chunks; chunk j of row r becomes output chunks 2j, 2j+1 of the
-          // 128-byte f16 row, placed at (chunk ^ (r & 7)) as the 128-byte swizzle requires
+          uint4 in[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = ct + i * kConvThreads;
-            const int r = c >> 2, j = c & 3;
-            const uint4 in = *reinterpret_cast<const uint4*>(src + w * kRawW + r * kBK + j * 16);
-            uint4 lo, hi;
-            e4m3x16_to_f16(in, lo, hi);
-            uint8_t* row = dst + w * kConvW + r * 128;
-            *reinterpret_cast<uint4*>(row + (((2 * j) ^ (r & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4*>(row + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+          for (int c = 0; c < 4; ++c) in[c] = ld_shared_v4(src + w * kRawW + (((4 * h + c) ^ (r & 7)) << 4));
+          uint32_t o[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            e4m3x4_to_f16x4(in[c].x, o[8 * c + 0], o[8 * c + 1]);
+            e4m3x4_to_f16x4(in[c].y, o[8 * c + 2], o[8 * c + 3]);
+            e4m3x4_to_f16x4(in[c].z, o[8 * c + 4], o[8 * c + 5]);
+            e4m3x4_to_f16x4(in[c].w, o[8 * c + 6], o[8 * c + 7]);
           }
+          tmem_st_32x32b_x32(tmem_base + lane_addr + C::kACol + as * C::kAStageCols + w * 64 + h * 32, o);
         }
-        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&cfull[cs]);
+        if (lane == 0) mbar_arrive(&afull[as]);
       }
     }
     if (!ok) set_error(p.err, kErrTimeout);
@@ -297,25 +287,24 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
         const uint32_t d = tmem_base + buf * C::kAccCols;
         const Unit u = decode_unit(p, unit_start, G, t);
         for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
-          const int st = it % C::kRawStages, cs = it % C::kConvStages;
-          if (!mbar_wait(&full[st], (it / C::kRawStages) & 1, kWaitLimitNs) ||
-              !mbar_wait(&cfull[cs], (it / C::kConvStages) & 1, kWaitLimitNs)) {
+          const int st = it % C::kStages, as = it % C::kAStages;
+          if (!mbar_wait(&full[st], (it / C::kStages) & 1, kWaitLimitNs) ||
+              !mbar_wait(&afull[as], (it / C::kAStages) & 1, kWaitLimitNs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(raw_base + st * C::kRawStage);  // activations (B)
-          const uint32_t sw = smem_u32(conv_base + cs * C::kConvStage);  // f16 weights (A)
+          const uint32_t sa = smem_u32(smem + st * C::kStage);  // activation atoms (B)
+          const uint32_t acol = tmem_base + C::kACol + as * C::kAStageCols;  // converted weights (A)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint32_t acc = (kb | kk) != 0;
-            const uint64_t bdesc = sw128_kmajor_desc(sa + kk * 32);
-            umma_bf16(d, sw128_kmajor_desc(sw + kk * 32), bdesc, C::kIdesc, acc);
-            if constexpr (KIND == kGateUp)
-              umma_bf16(d + NT, sw128_kmajor_desc(sw + kConvW + kk * 32), bdesc, C::kIdesc, acc);
+            const uint64_t bdesc = sw128_kmajor_desc(sa + (kk >> 2) * C::kAtom + (kk & 3) * 32);
+            umma_f16_tmem_a(d, acol + kk * 8, bdesc, C::kIdesc, acc);
+            if constexpr (KIND == kGateUp) umma_f16_tmem_a(d + NT, acol + 64 + kk * 8, bdesc, C::kIdesc, acc);
           }
-          umma_commit(&empty[st]);   // the raw stage (and its activation tile) is free
-          umma_commit(&cempty[cs]);  // the converted stage is free
+          umma_commit(&empty[st]);   // the stage's codes and activations are free
+          umma_commit(&aempty[as]);  // the converted A stage is free
         }
         if (!ok) break;
         umma_commit(&acc_full[buf]);
@@ -323,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
       if (!ok) set_error(p.err, kErrTimeout);
       if (it > 0) {
         const uint32_t last = it - 1;
-        if (!mbar_wait(&cempty[last % C::kConvStages], (last / C::kConvStages) & 1, kWaitLimitNs))
+        if (!mbar_wait(&aempty[last % C::kAStages], (last / C::kAStages) & 1, kWaitLimitNs))
           set_error(p.err, kErrTimeout);
       }
     }
@@ -414,17 +403,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D row-major [rows, cols] map; box = box_cols x box_rows elements
+// 2-D row-major [rows, cols] map with the 128-byte swizzle; box = box_cols x box_rows elements
 bool make_map(CUtensorMap* m, CUtensorMapDataType type, int elem_bytes, const void* base, uint64_t rows,
-              uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+              uint64_t cols, uint32_t box_cols, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr || rows == 0 || cols == 0) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int sm_count() {
@@ -449,13 +439,12 @@ cudaError_t launch_fp8(const GemmSetHost* sets, const float* const* scales, int 
   for (int i = 0; i < n_sets; ++i) {
     const GemmSetHost& st = sets[i];
     const int K = st.K;
-    p.k_blocks[i] = K / kBK;
+    p.k_blocks[i] = (K + kBK - 1) / kBK;
     p.w_rows[i] = KIND == kGateUp ? 2 * st.n_out : st.n_out;
-    if (!make_map(&p.a_map[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, st.a, (uint64_t)st.a_rows, (uint64_t)K, kBK, NT,
-                  CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map(&p.a_map[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, st.a, (uint64_t)st.a_rows, (uint64_t)K, 64, NT))
       return cudaErrorInvalidValue;
     if (!make_map(&p.w_map[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, st.w, (uint64_t)st.n_groups * p.w_rows[i],
-                  (uint64_t)K, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+                  (uint64_t)K, kBK, kBM))
       return cudaErrorInvalidValue;
     p.w_scale[i] = scales[i];
     p.offsets[i] = st.offsets;
@@ -494,7 +483,7 @@ cudaError_t launch_stream_fp8w(GemmKind kind, const GemmSetHost* sets, const flo
   if (n_sets < 1 || n_sets > 2) return cudaErrorInvalidValue;
   int groups = 0;
   for (int i = 0; i < n_sets; ++i) {
-    if (sets[i].K <= 0 || sets[i].K % kBK != 0 || w_scales[i] == nullptr) return cudaErrorInvalidValue;
+    if (sets[i].K <= 0 || sets[i].K % 64 != 0 || w_scales[i] == nullptr) return cudaErrorInvalidValue;
     groups += sets[i].n_groups;
   }
   if (groups > kMaxGroups) return cudaErrorInvalidValue;

@@ -38,6 +38,11 @@ def test_flop_and_byte_accounting(bench):
     # active-weight bytes: bf16 gate_up (2F x D) + down (D x F) per active expert, plus the shared one
     assert bench.active_weight_bytes(ds, 1) == 2 * (3 * ds.D * ds.F + 3 * ds.D * ds.Fs)
     assert bench.active_weight_bytes(ds, 10, "gate_up") == 2 * (10 * 2 * ds.F * ds.D + 2 * ds.Fs * ds.D)
+    # E4M3: one byte per weight plus one fp32 scale per weight row (2F + D rows per expert)
+    assert bench.active_weight_bytes(ds, 1, "all", "fp8") == (3 * ds.D * ds.F + 4 * (2 * ds.F + ds.D)
+                                                              + 3 * ds.D * ds.Fs + 4 * (2 * ds.Fs + ds.D))
+    g = mi.WORKLOADS["gptoss_decode_T1"]
+    assert bench.active_weight_bytes(g, 4, "down", "fp8") == 4 * (g.D * g.F + 4 * g.D)
 
 
 def test_traffic_is_reported_only_for_captured_workloads(bench):
