@@ -35,28 +35,32 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# DRAM bytes (read + write) of the dominant kernel per launch, from one ncu capture of the same
-# bench command (profiles/grouped_gemm_kernels.md), valid only while the GEMM sources are unchanged.
-_GEMM_SOURCES = ("sparse_mixture_experts_16_b200/csrc/grouped_gemm_sm100.cu",
-                 "sparse_mixture_experts_16_b200/csrc/sm100_ptx.cuh",
-                 "sparse_mixture_experts_16_b200/csrc/moe_common.cuh")
-_TRAFFIC_SOURCE_SHA256 = "c3f2678bfe5892ef2e25f811bf17341a5e59dc90db846cb22854a09d07975035"
-_TRAFFIC_BYTES = {  # workload -> gate_up launch: dram__bytes_read.sum + dram__bytes_write.sum
-    "mixtral": 1.946781e9 + 0.228668e9,
-    "deepseek_decode": 5.876604e9 + 0.004840e9,
+# DRAM bytes (read + write) of the dominant kernel (the gate_up launch) per launch, from one ncu
+# capture of the same bench command (profiles/grouped_gemm_kernels.md, profiles/stream_fp8w_kernel.md):
+# valid only while that kernel's sources are unchanged, else reported as null.
+_CSRC = "sparse_mixture_experts_16_b200/csrc/"
+_TRAFFIC = {
+    # weights -> (kernel sources, their sha256, {workload: dram__bytes_read.sum + dram__bytes_write.sum})
+    "bf16": ((_CSRC + "grouped_gemm_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
+             "636f5c796994e65aec9db9f1c91d3bba777c9551af9d012877e3d0879989a768",
+             {"mixtral": 1.946486e9 + 0.226486e9, "deepseek_decode": 5.876486e9 + 0.004078e9}),
+    "fp8": ((_CSRC + "stream_fp8w_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
+            "d33af253c883b52c16557b50c8d3516c8200992db331ccc8d752899fff96ff3f",
+            {"deepseek_decode": 2.942076e9 + 0.005430e9, "gptoss_decode_T64": 0.556636e9 + 0.005026e9}),
 }
 
 
-def measured_traffic(workload: str):
+def measured_traffic(workload: str, weights: str = "bf16"):
     import hashlib
 
+    files, digest, table = _TRAFFIC[weights]
     h = hashlib.sha256()
-    for f in _GEMM_SOURCES:
+    for f in files:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
-    if h.hexdigest() != _TRAFFIC_SOURCE_SHA256:
+    if h.hexdigest() != digest:
         return None
-    return _TRAFFIC_BYTES.get(workload)
+    return table.get(workload)
 
 
 def peaks():
@@ -259,7 +263,10 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         ws = layer.workspace(w.T)
         n_kernels = layer.kernel_count(w.T)
         weight_bytes = sum(t.numel() * t.element_size() for t in (inp["gate_up"], inp["down"], inp["wg"]))
-        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if weight_bytes < 8 * L2_BYTES else None
+        # a decode step touches only its active experts (as little as ~L2's size at T = 1), so decode
+        # steps always start from a flushed L2; prefill steps stream weights far larger than L2
+        flush = (torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+                 if weight_bytes < 8 * L2_BYTES or w.T <= 64 else None)
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
         for e in evs:
             e.record(stream)
@@ -365,7 +372,7 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         fp8 = args.weights == "fp8"
         roof = {"kernel": "stream_fp8w_kernel<gate_up>" if fp8 else "grouped_gemm_kernel<gate_up, stream>",
                 "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None if fp8 else measured_traffic(w.name),
+                "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name, args.weights),
                 "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)"}
     else:
         achieved = gateup_flops(w) / (gate_ms / 1e3) / 1e12

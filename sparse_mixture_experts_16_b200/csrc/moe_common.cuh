@@ -17,6 +17,45 @@ constexpr size_t kWsHeader = 256;
 // wall-time limit of every spin-wait inside a kernel
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
+// ---- split-K of the weight-streaming (decode) GEMMs ---------------------------------------------
+// A decode step with fewer 128-row units than SMs splits each unit's K range.  Partial fp32
+// accumulators go to a workspace buffer; four counters per unit (one per TMEM lane quadrant) let
+// the last split finish the epilogue.  The counters must be zero when a launch starts; every
+// launch leaves them zero.
+constexpr int kMaxSplitUnits = 256;                                      // no split above this
+constexpr size_t kSplitCounterBytes = (size_t)kMaxSplitUnits * 4 * sizeof(int);
+constexpr int kMaxSplitItems = 4 * 148;                                  // partial capacity (items)
+constexpr int kMaxSplits = 16;
+
+// workspace the host hands to a weight-streaming launch for split-K (all null: never split)
+struct SplitBuf {
+  float* partial = nullptr;  // partial accumulators, fp32
+  size_t partial_bytes = 0;
+  int* counters = nullptr;   // kSplitCounterBytes, zero when the launch starts
+};
+
+// K range [begin, end) of split s of S over kb k-blocks (balanced, non-empty when S <= kb)
+__device__ __forceinline__ int split_begin(int kb, int s, int S) { return (int)((long long)kb * s / S); }
+__device__ __forceinline__ int split_end(int kb, int s, int S) { return (int)((long long)kb * (s + 1) / S); }
+
+// Number of K splits for `units` units on `grid` CTAs: S minimises waves / S + 0.02 * S, capped by
+// the smallest k-block count and the partial buffer's capacity.  Every CTA gets the same answer.
+__device__ __forceinline__ int split_count(int units, int grid, int kb_min, int max_items) {
+  if (max_items <= 0 || units <= 0 || units >= grid || units > kMaxSplitUnits) return 1;
+  const int s_max = min(kMaxSplits, min(kb_min, max_items / units));
+  int best_s = 1;
+  float best = 1e30f;
+  for (int s = 1; s <= s_max; ++s) {
+    const int waves = (units * s + grid - 1) / grid;
+    const float cost = (float)waves / (float)s + 0.02f * (float)s;
+    if (cost < best) {
+      best = cost;
+      best_s = s;
+    }
+  }
+  return best_s;
+}
+
 __device__ __forceinline__ void set_error(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }
@@ -108,7 +147,7 @@ cudaError_t launch_grouped_gemm(GemmKind kind, const GemmSetHost* sets, int n_se
 // Weight-streaming grouped GEMMs with E4M3 expert weights (one fp32 scale per weight row,
 // w_scales[set]) and f16 activations (sets[i].a); gate_up writes f16 h.  decode_nt: 16..64.
 cudaError_t launch_stream_fp8w(GemmKind kind, const GemmSetHost* sets, const float* const* w_scales, int n_sets,
-                               int decode_nt, int* err, cudaStream_t s);
+                               int decode_nt, SplitBuf split, int* err, cudaStream_t s);
 
 // Per-row E4M3 quantisation: scales[r] = amax(row) / 448, q = E4M3(w / scale).  K % 8 == 0.
 cudaError_t launch_quantize_rows_fp8(const uint16_t* w, long long rows, int K, uint8_t* q, float* scales,

@@ -38,8 +38,16 @@ moe_status_t shape_status(long long T, long long D, long long E, long long k) {
   return MOE_OK;
 }
 
+bool use_decode(const moe_layer_desc_t& d) {
+  if (d.flags & MOE_FLAG_FORCE_DECODE) return true;
+  if (d.flags & MOE_FLAG_FORCE_PREFILL) return false;
+  return d.T <= kDecodeTMax;
+}
+
+int decode_tile(int max_seg) { return ((max_seg + 15) / 16) * 16; }
+
 struct LayerWs {
-  size_t router, topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
+  size_t split_counters, split_partial, split_partial_bytes, router, topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
       out_sh, x16, x_stage, y_stage, total;
 };
 
@@ -52,6 +60,14 @@ LayerWs layer_ws(const moe_layer_desc_t& d) {
     return at;
   };
   const size_t T = d.T, D = d.D, E = d.E, k = d.k, F = d.F, Fs = d.Fs, M = T * k;
+  // split-K counters directly after the error word, so one memset clears both
+  w.split_counters = take(kSplitCounterBytes);
+  // split-K partials of the FP8 weight-streaming GEMMs: gate_up items are the larger, 2 * NT
+  // accumulator columns x 128 rows x fp32
+  w.split_partial_bytes = d.weight_format == MOE_WEIGHTS_FP8_E4M3
+                              ? (size_t)kMaxSplitItems * 2 * decode_tile(d.T) * 128 * sizeof(float)
+                              : 0;
+  w.split_partial = take(w.split_partial_bytes);
   w.router = take(router_scratch_bytes(d.T, d.D, d.E));
   w.topk_idx = take(M * 4);
   w.topk_w = take(M * 4);
@@ -110,13 +126,6 @@ moe_status_t validate_desc(const moe_layer_desc_t* d) {
   return MOE_OK;
 }
 
-bool use_decode(const moe_layer_desc_t& d) {
-  if (d.flags & MOE_FLAG_FORCE_DECODE) return true;
-  if (d.flags & MOE_FLAG_FORCE_PREFILL) return false;
-  return d.T <= kDecodeTMax;
-}
-
-int decode_tile(int max_seg) { return ((max_seg + 15) / 16) * 16; }
 
 #define MOE_CUDA_TRY(expr)                 \
   do {                                     \
@@ -185,7 +194,8 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
   auto record = [&](cudaEvent_t e) { return cudaEventRecordWithFlags(e, s, rec_flags); };
 
   if (ev) MOE_CUDA_TRY(record(ev[0]));
-  MOE_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));  // a fresh error word for this forward
+  // a fresh error word and zeroed split-K counters (they follow the header) for this forward
+  MOE_CUDA_TRY(cudaMemsetAsync(err, 0, w.split_counters + kSplitCounterBytes, s));
   const int splits = router_k_splits(T, D, E);
   MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s));
   MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
@@ -201,6 +211,12 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
   }
   if (ev) MOE_CUDA_TRY(record(ev[2]));
   const int nt = use_decode(*d) ? decode_tile(T) : 0;
+  SplitBuf split;  // split-K buffers of the FP8 weight-streaming GEMMs
+  if (w.split_partial_bytes > 0) {
+    split.partial = Fp(w.split_partial);
+    split.partial_bytes = w.split_partial_bytes;
+    split.counters = I(w.split_counters);
+  }
   if (fp8) {
     GemmSetHost g[2];
     memset(g, 0, sizeof(g));
@@ -211,7 +227,7 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
       g[1].K = D, g[1].a = H(w.x16), g[1].a_rows = T, g[1].w = reinterpret_cast<const uint16_t*>(d->shared_gate_up_fp8);
       g[1].n_groups = 1, g[1].m_rows = T, g[1].n_out = Fs, g[1].out = H(w.h_sh);
     }
-    MOE_CUDA_TRY(launch_stream_fp8w(kGateUp, g, gs, Fs > 0 ? 2 : 1, nt, err, s));
+    MOE_CUDA_TRY(launch_stream_fp8w(kGateUp, g, gs, Fs > 0 ? 2 : 1, nt, split, err, s));
     if (ev) MOE_CUDA_TRY(record(ev[3]));
     GemmSetHost dn[2];
     memset(dn, 0, sizeof(dn));
@@ -223,7 +239,7 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
       dn[1].K = Fs, dn[1].a = H(w.h_sh), dn[1].a_rows = T, dn[1].w = reinterpret_cast<const uint16_t*>(d->shared_down_fp8);
       dn[1].n_groups = 1, dn[1].m_rows = T, dn[1].n_out = D, dn[1].out = Fp(w.out_sh);
     }
-    MOE_CUDA_TRY(launch_stream_fp8w(kDown, dn, ds, Fs > 0 ? 2 : 1, nt, err, s));
+    MOE_CUDA_TRY(launch_stream_fp8w(kDown, dn, ds, Fs > 0 ? 2 : 1, nt, split, err, s));
   } else {
   st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), Fp(w.out_perm), x,
                T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, err, s, ev ? ev[3] : nullptr,

@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -55,6 +56,9 @@ struct alignas(64) Fp8Params {
   int n_out[2];
   int w_rows[2];
   int k_blocks[2];          // ceil(K / 128)
+  float* partial;           // split-K partial accumulators [items][kAccCols][128] or null (no split)
+  int* counters;            // per unit: splits finished (zero on entry, left zero on exit)
+  int max_items;            // capacity of `partial` in items
   int n_sets;
   int withhold_first_load;
   int* err;
@@ -116,6 +120,14 @@ __device__ __forceinline__ Unit decode_unit(const Fp8Params& p, const int* unit_
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+// split-K for small unit counts (moe_common.cuh): an item is (unit, split)
+__device__ __forceinline__ int choose_splits(const Fp8Params& p, int units, int grid) {
+  if (p.partial == nullptr) return 1;
+  int kb_min = p.k_blocks[0];
+  if (p.n_sets > 1) kb_min = min(kb_min, p.k_blocks[1]);
+  return split_count(units, grid, kb_min, p.max_items);
+}
 
 template <int KIND, int NT>
 __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_constant__ Fp8Params p) {
@@ -194,7 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = unit_start[G];
+  const int n_units = unit_start[G];
+  const int S = choose_splits(p, n_units, gridDim.x);  // identical in every CTA
+  const int total = n_units * S;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -202,9 +216,10 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Unit u = decode_unit(p, unit_start, G, t);
+        const Unit u = decode_unit(p, unit_start, G, t / S);
         const int wrow = u.gl * p.w_rows[u.set] + u.n * kBM;
-        for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
+        const int kb_end = split_end(p.k_blocks[u.set], t % S, S);
+        for (int kb = split_begin(p.k_blocks[u.set], t % S, S); kb < kb_end; ++kb, ++it) {
           const int st = it % C::kStages;
           if (!mbar_wait(&empty[st], ((it / C::kStages) & 1) ^ 1, kWaitLimitNs)) {
             ok = false;
@@ -240,8 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const Unit u = decode_unit(p, unit_start, G, t);
-      for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
+      const Unit u = decode_unit(p, unit_start, G, t / S);
+      const int kb_end = split_end(p.k_blocks[u.set], t % S, S);
+      for (int kb = split_begin(p.k_blocks[u.set], t % S, S); kb < kb_end; ++kb, ++it) {
         const int st = it % C::kStages, as = it % C::kAStages;
         if (!mbar_wait(&full[st], (it / C::kStages) & 1, kWaitLimitNs) ||
             !mbar_wait(&aempty[as], ((it / C::kAStages) & 1) ^ 1, kWaitLimitNs)) {
@@ -285,8 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
         }
         tc_fence_after();
         const uint32_t d = tmem_base + buf * C::kAccCols;
-        const Unit u = decode_unit(p, unit_start, G, t);
-        for (int kb = 0; kb < p.k_blocks[u.set]; ++kb, ++it) {
+        const Unit u = decode_unit(p, unit_start, G, t / S);
+        const int kb0 = split_begin(p.k_blocks[u.set], t % S, S), kb_end = split_end(p.k_blocks[u.set], t % S, S);
+        for (int kb = kb0; kb < kb_end; ++kb, ++it) {
           const int st = it % C::kStages, as = it % C::kAStages;
           if (!mbar_wait(&full[st], (it / C::kStages) & 1, kWaitLimitNs) ||
               !mbar_wait(&afull[as], (it / C::kAStages) & 1, kWaitLimitNs)) {
@@ -298,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
           const uint32_t acol = tmem_base + C::kACol + as * C::kAStageCols;  // converted weights (A)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint32_t acc = (kb | kk) != 0;
+            const uint32_t acc = (kb != kb0 || kk != 0) ? 1u : 0u;
             const uint64_t bdesc = sw128_kmajor_desc(sa + (kk >> 2) * C::kAtom + (kk & 3) * 32);
             umma_f16_tmem_a(d, acol + kk * 8, bdesc, C::kIdesc, acc);
             if constexpr (KIND == kGateUp) umma_f16_tmem_a(d + NT, acol + 64 + kk * 8, bdesc, C::kIdesc, acc);
@@ -318,7 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
     }
   } else {
     // ------------------------------------------------------------------ epilogue (warps 2..5)
+    // Thread = accumulator row r (TMEM lane) = output column n*128 + r of its unit.
     const int q = warp & 3;
+    const int r = q * 32 + lane;
     uint32_t tl = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tl) {
       const uint32_t buf = tl & 1, use = tl >> 1;
@@ -327,53 +346,73 @@ __global__ void __launch_bounds__(kThreads, 1) stream_fp8w_kernel(const __grid_c
         break;
       }
       tc_fence_after();
-      const Unit u = decode_unit(p, unit_start, G, t);
+      const Unit u = decode_unit(p, unit_start, G, t / S);
       const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * C::kAccCols;
       const int n_out = p.n_out[u.set];
       const int wbase = u.gl * p.w_rows[u.set];
-      const int col = u.n * kBM + q * 32 + lane;  // output column = weight row within the group
+      const int col = u.n * kBM + r;  // output column = weight row within the group
       const bool col_ok = col < n_out;
       const float* ws = p.w_scale[u.set];
-      if constexpr (KIND == kGateUp) {
-        const float sg = col_ok ? ws[wbase + col] : 0.f, su = col_ok ? ws[wbase + n_out + col] : 0.f;
-        __half* out_h = static_cast<__half*>(p.out[u.set]);
-#pragma unroll 1
-        for (int j0 = 0; j0 < NT; j0 += 16) {
-          if (j0 >= u.rows) break;
-          uint32_t g[16], v[16];
-          tmem_ld_32x32b_x16(tacc + j0, g);
-          tmem_ld_32x32b_x16(tacc + NT + j0, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int j = j0 + jj;
-            if (j < u.rows && col_ok)
-              out_h[(size_t)(u.row0 + j) * n_out + col] =
-                  __float2half_rn(silu_mul(__uint_as_float(g[jj]) * sg, __uint_as_float(v[jj]) * su));
-          }
+      const float s0 = col_ok ? ws[wbase + col] : 0.f;                                    // gate / down row
+      const float s1 = (KIND == kGateUp && col_ok) ? ws[wbase + n_out + col] : 0.f;      // up row
+      const float* rs = p.row_scale[u.set];
+      // final value of token j (accumulators a = gate or down, b = up), written to the output
+      auto store = [&](int j, float a, float b) {
+        if (!col_ok) return;
+        if constexpr (KIND == kGateUp) {
+          static_cast<__half*>(p.out[u.set])[(size_t)(u.row0 + j) * n_out + col] = __float2half_rn(silu_mul(a * s0, b * s1));
+        } else {
+          static_cast<float*>(p.out[u.set])[(size_t)(u.row0 + j) * n_out + col] =
+              a * s0 * (rs != nullptr ? rs[u.row0 + j] : 1.0f);
         }
-      } else {
-        const float sd = col_ok ? ws[wbase + col] : 0.f;
-        const float* rs = p.row_scale[u.set];
-        float* out_f = static_cast<float*>(p.out[u.set]);
+      };
+      float* part = S > 1 ? p.partial + (size_t)t * C::kAccCols * kBM : nullptr;
 #pragma unroll 1
-        for (int j0 = 0; j0 < NT; j0 += 16) {
-          if (j0 >= u.rows) break;
-          uint32_t a[16];
-          tmem_ld_32x32b_x16(tacc + j0, a);
-          tmem_ld_wait();
+      for (int j0 = 0; j0 < NT; j0 += 16) {
+        if (j0 >= u.rows) break;
+        uint32_t a[16], b[16];
+        tmem_ld_32x32b_x16(tacc + j0, a);
+        if constexpr (KIND == kGateUp) tmem_ld_32x32b_x16(tacc + NT + j0, b);
+        tmem_ld_wait();
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int j = j0 + jj;
-            if (j < u.rows && col_ok)
-              out_f[(size_t)(u.row0 + j) * n_out + col] =
-                  __uint_as_float(a[jj]) * sd * (rs != nullptr ? rs[u.row0 + j] : 1.0f);
+        for (int jj = 0; jj < 16; ++jj) {
+          const int j = j0 + jj;
+          if (j >= u.rows) continue;
+          const float av = __uint_as_float(a[jj]), bv = KIND == kGateUp ? __uint_as_float(b[jj]) : 0.f;
+          if (part == nullptr) {
+            store(j, av, bv);
+          } else {
+            part[(size_t)j * kBM + r] = av;
+            if constexpr (KIND == kGateUp) part[(size_t)(NT + j) * kBM + r] = bv;
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (part != nullptr) {
+        // publish this split's rows; the last of the S splits of this quadrant sums them in split
+        // order (deterministic) and finishes the epilogue
+        __threadfence();
+        __syncwarp();
+        int* counter = p.counters + (size_t)(t / S) * 4 + q;
+        int done = 0;
+        if (lane == 0) done = atomicAdd(counter, 1);
+        done = __shfl_sync(0xffffffffu, done, 0);
+        if (done == S - 1) {
+          __threadfence();
+          const float* base = p.partial + (size_t)(t / S) * S * C::kAccCols * kBM + r;
+          for (int j = 0; j < u.rows; ++j) {
+            float av = 0.f, bv = 0.f;
+            for (int sp = 0; sp < S; ++sp) {
+              av += __ldcg(base + ((size_t)sp * C::kAccCols + j) * kBM);
+              if constexpr (KIND == kGateUp) bv += __ldcg(base + ((size_t)sp * C::kAccCols + NT + j) * kBM);
+            }
+            store(j, av, bv);
+          }
+          if (lane == 0) *counter = 0;  // ready for the next launch
+        }
+      }
     }
   }
 
@@ -428,12 +467,19 @@ int sm_count() {
 }
 
 template <int KIND, int NT>
-cudaError_t launch_fp8(const GemmSetHost* sets, const float* const* scales, int n_sets, int* err, cudaStream_t s) {
+cudaError_t launch_fp8(const GemmSetHost* sets, const float* const* scales, int n_sets, float* partial,
+                       size_t partial_bytes, int* counters, int* err, cudaStream_t s) {
   using C = Fp8Cfg<KIND, NT>;
   Fp8Params p;
   memset(&p, 0, sizeof(p));
   p.n_sets = n_sets;
   p.err = err;
+  const size_t item_bytes = (size_t)C::kAccCols * kBM * sizeof(float);
+  if (partial != nullptr && counters != nullptr && partial_bytes >= 2 * item_bytes) {
+    p.partial = partial;
+    p.counters = counters;
+    p.max_items = (int)std::min<size_t>(partial_bytes / item_bytes, (size_t)kMaxSplitItems);
+  }
   const char* hold = getenv("MOE_TEST_WITHHOLD_LOAD");
   p.withhold_first_load = (hold != nullptr && hold[0] == '1') ? 1 : 0;
   for (int i = 0; i < n_sets; ++i) {
@@ -465,13 +511,13 @@ cudaError_t launch_fp8(const GemmSetHost* sets, const float* const* scales, int 
 }
 
 template <int KIND>
-cudaError_t launch_kind(const GemmSetHost* sets, const float* const* scales, int n_sets, int nt, int* err,
-                        cudaStream_t s) {
+cudaError_t launch_kind(const GemmSetHost* sets, const float* const* scales, int n_sets, int nt, float* partial,
+                        size_t partial_bytes, int* counters, int* err, cudaStream_t s) {
   switch (nt) {
-    case 16: return launch_fp8<KIND, 16>(sets, scales, n_sets, err, s);
-    case 32: return launch_fp8<KIND, 32>(sets, scales, n_sets, err, s);
-    case 48: return launch_fp8<KIND, 48>(sets, scales, n_sets, err, s);
-    case 64: return launch_fp8<KIND, 64>(sets, scales, n_sets, err, s);
+    case 16: return launch_fp8<KIND, 16>(sets, scales, n_sets, partial, partial_bytes, counters, err, s);
+    case 32: return launch_fp8<KIND, 32>(sets, scales, n_sets, partial, partial_bytes, counters, err, s);
+    case 48: return launch_fp8<KIND, 48>(sets, scales, n_sets, partial, partial_bytes, counters, err, s);
+    case 64: return launch_fp8<KIND, 64>(sets, scales, n_sets, partial, partial_bytes, counters, err, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -479,7 +525,7 @@ cudaError_t launch_kind(const GemmSetHost* sets, const float* const* scales, int
 }  // namespace
 
 cudaError_t launch_stream_fp8w(GemmKind kind, const GemmSetHost* sets, const float* const* w_scales, int n_sets,
-                               int decode_nt, int* err, cudaStream_t s) {
+                               int decode_nt, SplitBuf split, int* err, cudaStream_t s) {
   if (n_sets < 1 || n_sets > 2) return cudaErrorInvalidValue;
   int groups = 0;
   for (int i = 0; i < n_sets; ++i) {
@@ -487,8 +533,12 @@ cudaError_t launch_stream_fp8w(GemmKind kind, const GemmSetHost* sets, const flo
     groups += sets[i].n_groups;
   }
   if (groups > kMaxGroups) return cudaErrorInvalidValue;
-  if (kind == kGateUp) return launch_kind<kGateUp>(sets, w_scales, n_sets, decode_nt, err, s);
-  if (kind == kDown) return launch_kind<kDown>(sets, w_scales, n_sets, decode_nt, err, s);
+  if (kind == kGateUp)
+    return launch_kind<kGateUp>(sets, w_scales, n_sets, decode_nt, split.partial, split.partial_bytes, split.counters,
+                                err, s);
+  if (kind == kDown)
+    return launch_kind<kDown>(sets, w_scales, n_sets, decode_nt, split.partial, split.partial_bytes, split.counters,
+                              err, s);
   return cudaErrorInvalidValue;
 }
 

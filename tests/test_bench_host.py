@@ -47,8 +47,11 @@ def test_flop_and_byte_accounting(bench):
 
 def test_traffic_is_reported_only_for_captured_workloads(bench):
     assert bench.measured_traffic("tiny") is None
+    assert bench.measured_traffic("mixtral", "fp8") is None
     v = bench.measured_traffic("mixtral")
     assert v is None or v > 1.9e9  # None once the kernel sources differ from the captured ones
+    v = bench.measured_traffic("deepseek_decode", "fp8")
+    assert v is None or 2.9e9 < v < 3.0e9  # E4M3 codes: half the bf16 capture's 5.88 GB
 
 
 def test_clock_summary_flags_throttling(bench):

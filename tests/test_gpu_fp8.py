@@ -114,3 +114,25 @@ def test_fp8_full_size_sampled(cuda_device, name, n_tok):
     y_ref, _, _ = oracle.layer_fp8(x_h[rows], wg_h, bias_h, w.k, q, shared)
     got = bf16_np_to_f64(to_np_bf16(y[torch.from_numpy(rows).cuda()]))
     assert rel_rms_err(got, y_ref) <= REL_RMS_TOL
+
+
+def test_fp8_decode_split_k_deterministic_matches_oracle_and_leaves_counters_zero():
+    """One token on 4 of 16 experts with F = 1024: 4 x 8 units of 128 rows (+ the shared expert),
+    far fewer than SMs, so the FP8 GEMMs split K.  The last split of each unit sums the partials in
+    a fixed order: repeated forwards are bit-identical and match the oracle, and the split
+    counters (which follow the 256-byte error header of the workspace) are back to zero."""
+    w = W(1, 512, 16, 4, 1024, Fs=256)
+    rd = gap_redraw(w)
+    h, d, layer = _quantized_layer(w, rd)
+    ys = [to_np_bf16(layer(d["x"])) for _ in range(3)]
+    assert all((y == ys[0]).all() for y in ys[1:])
+    assert layer.device_error() == 0
+    ws = layer.workspace(w.T)
+    assert int(ws[256:256 + 4096].count_nonzero()) == 0
+    q = {}
+    q["gu_q"], q["gu_s"] = oracle.quantize_rows_fp8(h["gate_up"])
+    q["dn_q"], q["dn_s"] = oracle.quantize_rows_fp8(h["down"])
+    a, b = oracle.quantize_rows_fp8(h["shared_gate_up"])
+    c, e = oracle.quantize_rows_fp8(h["shared_down"])
+    y_ref, _, _ = oracle.layer_fp8(h["x"], h["wg"], h["bias"], w.k, q, dict(gu_q=a, gu_s=b, dn_q=c, dn_s=e))
+    assert rel_rms_err(bf16_np_to_f64(ys[0]), y_ref) <= REL_RMS_TOL

@@ -260,6 +260,20 @@ def test_layer_is_deterministic_and_reports_no_device_error():
     assert L.device_error() == 0
 
 
+def test_decode_path_is_deterministic_and_matches_oracle():
+    """Two tokens on 16 experts: the weight-streaming (decode) GEMMs; repeated forwards are
+    bit-identical and match the oracle."""
+    w = W(2, 512, 16, 2, 1024, Fs=256, bias="normal:0.5")
+    inp, _ = host_case(w)
+    d = device_from_host(inp)
+    y_ref, _, _ = oracle_layer(inp, w.k)
+    L = layer_from(d, w.k)
+    ys = [to_np_bf16(L(d["x"])) for _ in range(3)]
+    assert all((y == ys[0]).all() for y in ys[1:])
+    assert rel_rms_err(bf16_np_to_f64(ys[0]), y_ref) <= REL_RMS_TOL
+    assert L.device_error() == 0
+
+
 def test_layer_host_buffers_match_device_buffers():
     import torch
 
