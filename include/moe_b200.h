@@ -183,7 +183,11 @@ typedef struct {
    * Experts optimiza...", section "Resultados practicos"; codes from moe_quantize_rows_fp8):
    * used when weight_format == MOE_WEIGHTS_FP8_E4M3, where the bf16 gate_up / down / shared_*
    * pointers are ignored.  Row r of a tensor dequantises to code * scale[r].  Decode only
-   * (T <= 64; larger T returns MOE_ERR_UNSUPPORTED_SHAPE); activations run in f16. */
+   * (T <= 64; larger T returns MOE_ERR_UNSUPPORTED_SHAPE).  Activations (x and h) run in f16:
+   * x converts exactly for 2^-14 <= |x| <= 65504 (smaller values lose low bits, larger ones
+   * overflow).  Code pointers must be 16-byte aligned, scales 4-byte aligned.  Steps with fewer
+   * 128-row units than SMs split K; the partial sums are added in a fixed order, so results are
+   * deterministic. */
   int32_t weight_format;                /* MOE_WEIGHTS_BF16 or MOE_WEIGHTS_FP8_E4M3          */
   const uint8_t* gate_up_fp8;           /* [E, 2F, D] codes                                  */
   const float* gate_up_scale;           /* [E, 2F]                                           */
@@ -205,7 +209,8 @@ moe_status_t moe_quantize_rows_fp8(const moe_bf16_t* w, int64_t rows, int K, uin
 /* Device workspace bytes for moe_layer_forward / moe_layer_forward_host (0 if desc invalid). */
 size_t moe_layer_workspace_size(const moe_layer_desc_t* desc);
 
-/* x [T, D] bf16 (device) -> y [T, D] bf16 (device).  Clears the workspace's error word first. */
+/* x [T, D] bf16 (device) -> y [T, D] bf16 (device).  Clears the workspace's error word (and the
+ * split-K counters that follow it) first, with one memset on `stream`. */
 moe_status_t moe_layer_forward(const moe_layer_desc_t* desc, const moe_bf16_t* x, moe_bf16_t* y,
                                void* ws, size_t ws_bytes, moe_stream_t stream);
 
