@@ -114,8 +114,8 @@ cudaError_t launch_update_bias(const int32_t* counts, int E, float gamma, float*
 size_t permute_scratch_bytes(int T, int E);
 cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16_t* x, int T, int D, int E,
                            int k, int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* inv_perm,
-                           float* p_perm, uint16_t* x_perm, int32_t* scratch, int* err, cudaStream_t s,
-                           int* n_launches);
+                           float* p_perm, uint16_t* x_perm, bool x_perm_f16, uint16_t* x_cast, int32_t* scratch,
+                           int* err, cudaStream_t s, int* n_launches);
 
 cudaError_t launch_combine(const float* out_perm, const int32_t* inv_perm, const float* shared_out, int T, int D,
                            int k, uint16_t* y, cudaStream_t s);
@@ -154,8 +154,6 @@ cudaError_t launch_quantize_rows_fp8(const uint16_t* w, long long rows, int K, u
                                      cudaStream_t s);
 
 // x_perm rows as f16 (x_perm16[r] = f16(x[perm_token[r]])) and a plain bf16 -> f16 cast.
-cudaError_t launch_gather_rows_f16(const uint16_t* x, const int32_t* perm_token, const int32_t* offsets, int E,
-                                   int T, int D, uint16_t* x_perm16, cudaStream_t s);
 cudaError_t launch_cast_bf16_to_f16(const uint16_t* src, long long n, uint16_t* dst, cudaStream_t s);
 
 }  // namespace moe

@@ -202,13 +202,11 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
                                     Fp(w.topk_w), s));
   if (ev) MOE_CUDA_TRY(record(ev[1]));
   const bool fp8 = d->weight_format == MOE_WEIGHTS_FP8_E4M3;
-  MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), fp8 ? nullptr : x, T, D, E, k, I(w.counts),
-                              I(w.offsets), I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), fp8 ? nullptr : H(w.x_perm),
+  // dispatch + gather (one kernel for T <= 256); the FP8 path gathers f16 rows and, for the
+  // shared expert, an f16 copy of x
+  MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), x, T, D, E, k, I(w.counts), I(w.offsets), I(w.perm_token),
+                              I(w.inv_perm), Fp(w.p_perm), H(w.x_perm), fp8, (fp8 && Fs > 0) ? H(w.x16) : nullptr,
                               I(w.scratch), err, s, nullptr));
-  if (fp8) {
-    MOE_CUDA_TRY(launch_gather_rows_f16(x, I(w.perm_token), I(w.offsets), E, T, D, H(w.x_perm), s));
-    if (Fs > 0) MOE_CUDA_TRY(launch_cast_bf16_to_f16(x, (long long)T * D, H(w.x16), s));
-  }
   if (ev) MOE_CUDA_TRY(record(ev[2]));
   const int nt = use_decode(*d) ? decode_tile(T) : 0;
   SplitBuf split;  // split-K buffers of the FP8 weight-streaming GEMMs
@@ -329,7 +327,7 @@ moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, const moe
   if ((st = check_device()) != MOE_OK) return st;
   uint8_t* b = static_cast<uint8_t*>(ws);
   MOE_CUDA_TRY(launch_permute(topk_idx, topk_w, x, T, D, E, k, counts, offsets, perm_token, inv_perm, p_perm, x_perm,
-                              reinterpret_cast<int32_t*>(b + kWsHeader), reinterpret_cast<int*>(b),
+                              false, nullptr, reinterpret_cast<int32_t*>(b + kWsHeader), reinterpret_cast<int*>(b),
                               (cudaStream_t)stream, nullptr));
   return MOE_OK;
 }
@@ -415,9 +413,10 @@ moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16
 
 int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  const int dispatch = desc->T <= 256 ? 1 /*fused hist+scan+scatter*/ : 3 /*hist, scan, scatter*/;
-  const int cast = (desc->weight_format == MOE_WEIGHTS_FP8_E4M3 && desc->Fs > 0) ? 1 : 0;  // x -> f16
-  return 2 /*router GEMM, top-k*/ + dispatch + 1 /*gather*/ + cast + 2 /*grouped GEMMs*/ + 1 /*combine*/;
+  // T <= 256: one kernel sorts and gathers (and casts x for the FP8 path's shared expert, T <= 64);
+  // above: hist, scan, scatter, gather
+  const int dispatch = desc->T <= 256 ? 1 : 4;
+  return 2 /*router GEMM, top-k*/ + dispatch + 2 /*grouped GEMMs*/ + 1 /*combine*/;
 }
 
 moe_status_t moe_update_router_bias(const int32_t* counts, int E, float gamma, float* bias, moe_stream_t stream) {

@@ -11,9 +11,11 @@
 //                equal experts inside each 32-slot step come from __match_any_sync + popc, and
 //                a shared running counter per expert carries them across steps
 //   4. gather  : x_perm[r] = x[perm_token[r]], one warp per row, 16-byte vector moves
-// For T <= 256 steps 1-3 run as one single-block kernel (dispatch_small_kernel).
+// For T <= 256 steps 1-4 run as one kernel (dispatch_small_kernel: every CTA sorts, all gather).
 // Within an expert, rows are therefore ordered by token id (a token picks an expert at most once).
 #include <cuda_fp16.h>
+
+#include <algorithm>
 
 #include "moe_common.cuh"
 
@@ -124,19 +126,45 @@ __global__ void __launch_bounds__(32) scatter_kernel(const int32_t* __restrict__
   pdl_trigger();
 }
 
-// T <= 256 (one counting block): histogram, scan and the order-preserving scatter in one block of
-// 256 threads -- the same three steps as above without two launches and the per-block scratch.
+// bf16 -> f16 for 8 values (the FP8-weight GEMMs take f16 activations)
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 q) {
+  const uint32_t in[4] = {q.x, q.y, q.z, q.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h = __floats2half2_rn(bf16_lo(in[i]), bf16_hi(in[i]));
+    o[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+constexpr int kGatherNone = 0, kGatherBf16 = 1, kGatherF16 = 2;
+constexpr int kGatherChunk = 1024;  // columns per gather item
+
+// T <= 256 (one counting block): histogram, scan and the order-preserving scatter of the T*k slots
+// in one kernel -- the same three steps as above without two launches and the per-block scratch --
+// fused with the gather.  Every CTA sorts the (at most 8192) slots in shared memory, which costs a
+// few microseconds at most and needs no inter-CTA communication; CTA 0 alone writes the metadata.
+// Then all CTAs copy (row, 1024-column chunk) items x[perm_token[r]] -> x_perm[r], as bf16 or
+// converted to f16, followed (if x_cast is given) by x[t] -> x_cast[t] for every token.
+template <int GATHER>
 __global__ void __launch_bounds__(256) dispatch_small_kernel(const int32_t* __restrict__ idx,
                                                              const float* __restrict__ w, int T, int E, int k,
                                                              int32_t* __restrict__ counts,
                                                              int32_t* __restrict__ offsets,
                                                              int32_t* __restrict__ perm_token,
                                                              int32_t* __restrict__ inv_perm,
-                                                             float* __restrict__ p_perm, int* err) {
+                                                             float* __restrict__ p_perm, int* err,
+                                                             const uint16_t* __restrict__ x, int D,
+                                                             uint16_t* __restrict__ x_perm,
+                                                             uint16_t* __restrict__ x_cast) {
   extern __shared__ int sm[];
-  int* cnt = sm;       // [E] counts
-  int* run = sm + E;   // [E] next free row per expert
+  int* cnt = sm;         // [E] counts
+  int* run = sm + E;     // [E] next free row per expert
+  int* perm_s = sm + 2 * E;  // [T*k] token of each row (gathering only)
   __shared__ int warp_tot[8];
+  __shared__ int n_rows_s;
+  const bool lead = blockIdx.x == 0;  // writes the metadata
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += 256) cnt[e] = 0;
   pdl_wait();
@@ -146,7 +174,7 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(const int32_t* __re
     const int e = idx[i];
     if ((unsigned)e < (unsigned)E)
       atomicAdd(&cnt[e], 1);
-    else
+    else if (lead)
       set_error(err, kErrBadIndex);
   }
   __syncthreads();
@@ -167,12 +195,17 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(const int32_t* __re
   for (int q = 0; q < warp; ++q) before += warp_tot[q];
   int r0 = before + incl - sum;
   for (int e = lo; e < hi; ++e) {
-    counts[e] = cnt[e];
-    offsets[e] = r0;
+    if (lead) {
+      counts[e] = cnt[e];
+      offsets[e] = r0;
+    }
     run[e] = r0;
     r0 += cnt[e];
   }
-  if (tid == 255) offsets[E] = before + incl;
+  if (tid == 255) {
+    n_rows_s = before + incl;
+    if (lead) offsets[E] = before + incl;
+  }
   __syncthreads();
   if (warp == 0) {
     const unsigned lt_mask = (1u << lane) - 1u;
@@ -182,20 +215,40 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(const int32_t* __re
       if (i < n_items) {
         e = idx[i];
         if ((unsigned)e >= (unsigned)E) {
-          inv_perm[i] = -1;
+          if (lead) inv_perm[i] = -1;
           e = -1;
         }
       }
       const unsigned peers = __match_any_sync(0xffffffffu, e);
       if (e >= 0) {
         const int r = run[e] + __popc(peers & lt_mask);
-        perm_token[r] = i / k;
-        inv_perm[i] = r;
-        p_perm[r] = w[i];
+        if (lead) {
+          perm_token[r] = i / k;
+          inv_perm[i] = r;
+          p_perm[r] = w[i];
+        }
+        if (GATHER != kGatherNone) perm_s[r] = i / k;
       }
       __syncwarp();
       if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
       __syncwarp();
+    }
+  }
+  if constexpr (GATHER != kGatherNone) {
+    __syncthreads();
+    const int n_chunks = (D + kGatherChunk - 1) / kGatherChunk;
+    const int n_rows = n_rows_s;
+    const int n_work = (n_rows + (x_cast != nullptr ? T : 0)) * n_chunks;
+    for (int it = blockIdx.x * 8 + warp; it < n_work; it += gridDim.x * 8) {
+      const int r = it / n_chunks, c0 = (it - r * n_chunks) * kGatherChunk;
+      const int c1 = min(D, c0 + kGatherChunk);
+      const bool cast_row = r >= n_rows;  // x_cast[t] = x[t], t = r - n_rows
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(cast_row ? r - n_rows : perm_s[r]) * D);
+      uint4* dst = reinterpret_cast<uint4*>(cast_row ? x_cast + (size_t)(r - n_rows) * D : x_perm + (size_t)r * D);
+      for (int v = c0 / 8 + lane; v < c1 / 8; v += 32) {
+        const uint4 q = __ldg(src + v);
+        dst[v] = GATHER == kGatherF16 ? bf16x8_to_f16x8(q) : q;
+      }
     }
   }
   pdl_trigger();
@@ -218,18 +271,6 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
   }
   pdl_trigger();
-}
-
-// bf16 -> f16 for 8 values (the FP8-weight GEMMs take f16 activations)
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 q) {
-  const uint32_t in[4] = {q.x, q.y, q.z, q.w};
-  uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2 h = __floats2half2_rn(bf16_lo(in[i]), bf16_hi(in[i]));
-    o[i] = *reinterpret_cast<const uint32_t*>(&h);
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // x_perm16[r] = f16(x[perm_token[r]]) for r < offsets[E]; one warp per row.
@@ -268,51 +309,66 @@ size_t permute_scratch_bytes(int T, int E) {
 
 cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16_t* x, int T, int D, int E, int k,
                            int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* inv_perm, float* p_perm,
-                           uint16_t* x_perm, int32_t* scratch, int* err, cudaStream_t s, int* n_launches) {
+                           uint16_t* x_perm, bool x_perm_f16, uint16_t* x_cast, int32_t* scratch, int* err,
+                           cudaStream_t s, int* n_launches) {
   const int nb = (T + kTokPerBlock - 1) / kTokPerBlock;
+  const bool gather = x != nullptr && x_perm != nullptr && T > 0;
+  if (!x_perm_f16) x_cast = nullptr;  // the cast copy exists for the f16 (FP8-weight) path only
   int launches = 0;
-  if (nb == 1) {
-    cudaError_t e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(256), 2 * E * sizeof(int), s, idx, topk_w, T, E,
-                               k, counts, offsets, perm_token, inv_perm, p_perm, err);
-    if (e != cudaSuccess) return e;
-    ++launches;
-  } else if (nb > 0) {
-    cudaError_t e = launch_pdl(hist_kernel, dim3(nb), dim3(256), E * sizeof(int), s, idx, T, E, k, scratch, err);
-    if (e != cudaSuccess) return e;
-    ++launches;
-  }
   cudaError_t e = cudaSuccess;
-  if (nb != 1) {
-    e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, scratch, nb, E, counts, offsets);
+  if (nb == 1) {
+    // one fused kernel: sort in every CTA, gather (row, column chunk) items across the grid
+    const long long items =
+        gather ? ((long long)T * k + (x_cast != nullptr ? T : 0)) * ((D + kGatherChunk - 1) / kGatherChunk) : 0;
+    const unsigned blocks = gather ? (unsigned)std::min<long long>(148, (items + 7) / 8) : 1u;
+    const size_t smem = (2 * (size_t)E + (gather ? (size_t)T * k : 0)) * sizeof(int);
+    if (!gather)
+      e = launch_pdl(dispatch_small_kernel<kGatherNone>, dim3(1), dim3(256), smem, s, idx, topk_w, T, E, k, counts,
+                     offsets, perm_token, inv_perm, p_perm, err, x, D, x_perm, x_cast);
+    else if (x_perm_f16)
+      e = launch_pdl(dispatch_small_kernel<kGatherF16>, dim3(blocks), dim3(256), smem, s, idx, topk_w, T, E, k,
+                     counts, offsets, perm_token, inv_perm, p_perm, err, x, D, x_perm, x_cast);
+    else
+      e = launch_pdl(dispatch_small_kernel<kGatherBf16>, dim3(blocks), dim3(256), smem, s, idx, topk_w, T, E, k,
+                     counts, offsets, perm_token, inv_perm, p_perm, err, x, D, x_perm, x_cast);
+    if (e != cudaSuccess) return e;
+    if (n_launches) *n_launches = 1;
+    return cudaGetLastError();
+  }
+  if (nb > 0) {
+    e = launch_pdl(hist_kernel, dim3(nb), dim3(256), E * sizeof(int), s, idx, T, E, k, scratch, err);
     if (e != cudaSuccess) return e;
     ++launches;
   }
-  if (nb > 1) {
+  e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, scratch, nb, E, counts, offsets);
+  if (e != cudaSuccess) return e;
+  ++launches;
+  if (nb > 0) {
     e = launch_pdl(scatter_kernel, dim3(nb), dim3(32), E * sizeof(int), s, idx, topk_w, T, E, k,
                    (const int32_t*)scratch, (const int32_t*)offsets, perm_token, inv_perm, p_perm);
     if (e != cudaSuccess) return e;
     ++launches;
   }
-  if (x != nullptr && x_perm != nullptr && T > 0) {
+  if (gather) {
     const long long rows = (long long)T * k;
     long long blocks = (rows + 7) / 8;
     if (blocks > 148LL * 16) blocks = 148LL * 16;
-    e = launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, (const int32_t*)perm_token,
-                   (const int32_t*)offsets, E, T, D, x_perm);
+    if (x_perm_f16)
+      e = launch_pdl(gather_rows_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, (const int32_t*)perm_token,
+                     (const int32_t*)offsets, E, T, D, x_perm);
+    else
+      e = launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, (const int32_t*)perm_token,
+                     (const int32_t*)offsets, E, T, D, x_perm);
+    if (e != cudaSuccess) return e;
+    ++launches;
+  }
+  if (gather && x_cast != nullptr) {
+    e = launch_cast_bf16_to_f16(x, (long long)T * D, x_cast, s);
     if (e != cudaSuccess) return e;
     ++launches;
   }
   if (n_launches) *n_launches = launches;
   return cudaGetLastError();
-}
-
-cudaError_t launch_gather_rows_f16(const uint16_t* x, const int32_t* perm_token, const int32_t* offsets, int E,
-                                   int T, int D, uint16_t* x_perm16, cudaStream_t s) {
-  if (T == 0) return cudaSuccess;
-  long long blocks = ((long long)T * 32 + 7) / 8;  // T*k rows at most; k <= 32
-  if (blocks > 148LL * 16) blocks = 148LL * 16;
-  return launch_pdl(gather_rows_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, perm_token, offsets, E, T,
-                    D, x_perm16);
 }
 
 cudaError_t launch_cast_bf16_to_f16(const uint16_t* src, long long n, uint16_t* dst, cudaStream_t s) {

@@ -72,7 +72,7 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_idx, const float
   // Every entry the kernels read is written earlier in the same call, so the previous call's
   // contents need no clearing.  No error word: out-of-range ids are dropped but not reported.
   if (moe::launch_permute(topk_idx, topk_w, x, T, D, E, k, counts, offsets, perm_token, inv_perm, p_perm, x_perm,
-                          scratch, nullptr, (cudaStream_t)stream, nullptr) != cudaSuccess) {
+                          false, nullptr, scratch, nullptr, (cudaStream_t)stream, nullptr) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }

@@ -82,7 +82,7 @@ def test_layer_workspace_size_and_small_workspace(L):
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, need - 1, None) == 4
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100010, need, None) == 3  # ws not 256-aligned
     assert L.moe_layer_forward(ctypes.byref(d), 0x4008, 0x5000, 0x100000, need, None) == 3
-    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 7  # T=16: fused dispatch
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 6  # T=16: one kernel sorts and gathers
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(T=300))) == 9
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(k=9))) == 0
     # shared expert grows the workspace
@@ -180,7 +180,7 @@ def test_fp8_descriptor_validation(L, kw, status):
 def test_fp8_kernel_count_and_quantizer_validation(L):
     d = _desc(**FP8, Fs=64, shared_gate_up_fp8=0xC000, shared_down_fp8=0xD000, shared_gate_up_scale=0xE000,
               shared_down_scale=0xF000)
-    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 8  # + the f16 cast of x for the shared expert
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 6  # the f16 gather and cast of x ride in dispatch
     assert L.moe_quantize_rows_fp8(None, 4, 64, 0x2000, 0x3000, None) == 1
     assert L.moe_quantize_rows_fp8(0x1000, 4, 100, 0x2000, 0x3000, None) == 2
     assert L.moe_quantize_rows_fp8(0x1008, 4, 64, 0x2000, 0x3000, None) == 3
