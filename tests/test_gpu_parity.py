@@ -274,6 +274,25 @@ def test_decode_path_is_deterministic_and_matches_oracle():
     assert L.device_error() == 0
 
 
+def test_decode_layer_equals_the_step_by_step_path_bit_for_bit():
+    """The layer forward and the step-by-step entry points (router, permute, grouped FFN with the
+    same 16-token tile, combine) are the same computation and must give the same bits."""
+    w = W(16, 256, 32, 4, 384, bias="normal:0.5")
+    inp, _ = host_case(w)
+    d = device_from_host(inp)
+    L = layer_from(d, w.k)
+    y_layer = to_np_bf16(L(d["x"]))
+    assert L.device_error() == 0
+    idx, p = moe.moe_router_topk(d["x"], d["wg"], d["bias"], w.k)
+    pm = moe.moe_permute(idx, p, d["x"], w.E)
+    max_seg = int(pm["counts"].max().item())
+    assert 0 < max_seg <= 16
+    out_perm, _ = moe.moe_grouped_swiglu_ffn(pm["x_perm"], pm["offsets"], pm["p_perm"], d["gate_up"], d["down"],
+                                             max_seg=max_seg)
+    y_steps = to_np_bf16(moe.moe_combine(out_perm, pm["inv_perm"], None, w.T, w.k))
+    assert (y_layer == y_steps).all()
+
+
 def test_layer_host_buffers_match_device_buffers():
     import torch
 
