@@ -55,6 +55,9 @@ def _L():
         L.oracle_quantize_rows_fp8.restype = None
         L.oracle_expert_ffn_fp8.argtypes = [P, P, P, P, P, i64, i64, P]
         L.oracle_expert_ffn_fp8.restype = None
+        L.oracle_layer_f64.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, P, i32]
+        L.oracle_layer_backward_f64.argtypes = [P, P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64,
+                                                P, P, P, P, P, P, i32]
         _lib = L
     return _lib
 
@@ -251,6 +254,56 @@ def layer_fp8(x, wg, bias, k, q, shared=None):
     with ThreadPoolExecutor(max_workers=_nthreads()) as pool:
         y = np.stack(list(pool.map(token, range(T)))) if T else np.zeros((0, D), np.float64)
     return y, idx, p
+
+
+# ----------------------------------------------------------------------------- backward (training)
+def _f64(a):
+    """bf16 bit patterns (uint16) -> exact float64 values; float arrays -> contiguous float64."""
+    if a is None:
+        return None
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray((a.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def layer_f64(x, wg, bias, gate_up, down, k, shared_gate_up=None, shared_down=None):
+    """The layer forward on fp64 parameters (bf16 bit patterns are read exactly): y [T, D]."""
+    x, wg, gu, dn = _f64(x), _f64(wg), _f64(gate_up), _f64(down)
+    sgu, sdn = _f64(shared_gate_up), _f64(shared_down)
+    T, D = x.shape
+    E = wg.shape[0]
+    F = dn.shape[2]
+    Fs = 0 if sgu is None else sgu.shape[0] // 2
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    y = np.empty((T, D), np.float64)
+    rc = _L().oracle_layer_f64(x.ctypes.data, wg.ctypes.data, _ptr(b), gu.ctypes.data, dn.ctypes.data, _ptr(sgu),
+                               _ptr(sdn), T, D, E, k, F, Fs, y.ctypes.data, _nthreads())
+    if rc != 0:
+        raise ValueError(f"oracle_layer_f64 rc={rc}")
+    return y
+
+
+def layer_backward(x, wg, bias, gate_up, down, k, dy, shared_gate_up=None, shared_down=None):
+    """Gradients of L = sum(dy * y) for the layer forward: dict(dx, dw_gate, dgate_up, ddown,
+    dshared_gate_up, dshared_down), all float64 (shared entries None without a shared expert)."""
+    x, wg, gu, dn, dy = _f64(x), _f64(wg), _f64(gate_up), _f64(down), _f64(dy)
+    sgu, sdn = _f64(shared_gate_up), _f64(shared_down)
+    T, D = x.shape
+    E = wg.shape[0]
+    F = dn.shape[2]
+    Fs = 0 if sgu is None else sgu.shape[0] // 2
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    out = dict(dx=np.empty((T, D)), dw_gate=np.empty((E, D)), dgate_up=np.empty((E, 2 * F, D)),
+               ddown=np.empty((E, D, F)), dshared_gate_up=np.empty((2 * Fs, D)) if Fs else None,
+               dshared_down=np.empty((D, Fs)) if Fs else None)
+    rc = _L().oracle_layer_backward_f64(
+        x.ctypes.data, wg.ctypes.data, _ptr(b), gu.ctypes.data, dn.ctypes.data, _ptr(sgu), _ptr(sdn), dy.ctypes.data,
+        T, D, E, k, F, Fs, out["dx"].ctypes.data, out["dw_gate"].ctypes.data, out["dgate_up"].ctypes.data,
+        out["ddown"].ctypes.data, _ptr(out["dshared_gate_up"]), _ptr(out["dshared_down"]), _nthreads())
+    if rc != 0:
+        raise ValueError(f"oracle_layer_backward_f64 rc={rc}")
+    return out
 
 
 # ----------------------------------------------------------------------------- gap-enforced inputs

@@ -354,4 +354,197 @@ void oracle_expert_ffn_fp8(const uint16_t* x_row, const uint8_t* gu_q, const flo
   }
 }
 
+// ---- backward pass (training) ----------------------------------------------------------------
+// keryc.com, section "Entrenamiento: todavia desafiante, pero con avances", and dev.smart-guide.co.kr,
+// section "Entrenamiento MoE: 12x Mas Rapido": MoE layers are trained, with grouped-GEMM kernels.
+// The pages print no formulas for the backward pass, so it is the chain rule applied to the
+// forward defined above, step by step.  With L = sum(dy * y):
+//   slot (t, j), expert e = idx[t, j], o = Expert_e(x_t), h = silu(g) * u, g = G_e x_t, u = U_e x_t:
+//     dp_j = dy_t . o,           do = p_j dy_t,
+//     dh   = Down_e^T do,        dDown_e += do h^T,
+//     dg   = dh * u * silu'(g),  du = dh * silu(g),    silu'(z) = s(z) (1 + z (1 - s(z))),
+//     dx_t += G_e^T dg + U_e^T du,   dG_e += dg x_t^T,   dU_e += du x_t^T;
+//   softmax over the chosen k:  dl_j = p_j (dp_j - sum_i p_i dp_i), and the other logits get 0;
+//     dx_t += sum_j dl_j W_g[idx_j],   dW_g[idx_j] += dl_j x_t;
+//   the shared expert: the same with p = 1.
+// The top-k selection is piecewise constant: neither it nor the selection bias carries a gradient.
+// These entry points take fp64 parameters so that the gradient can be checked against finite
+// differences of oracle_layer_f64.
+
+namespace {
+
+// x as doubles: logits, g and u of one expert, its output
+void router_logits_f64(const double* x, const double* wg, int64_t D, int E, double* l) {
+  for (int e = 0; e < E; ++e) {
+    double acc = 0.0;
+    for (int64_t d = 0; d < D; ++d) acc += x[d] * wg[(int64_t)e * D + d];
+    l[e] = acc;
+  }
+}
+
+struct ExpertFwd {
+  std::vector<double> g, u, h, o;
+};
+
+void expert_fwd_f64(const double* x, const double* gate_up, const double* down, int64_t D, int64_t F,
+                    ExpertFwd& r) {
+  r.g.assign(F, 0.0), r.u.assign(F, 0.0), r.h.assign(F, 0.0), r.o.assign(D, 0.0);
+  for (int64_t f = 0; f < F; ++f) {
+    double g = 0.0, u = 0.0;
+    for (int64_t d = 0; d < D; ++d) {
+      g += gate_up[f * D + d] * x[d];
+      u += gate_up[(F + f) * D + d] * x[d];
+    }
+    r.g[f] = g, r.u[f] = u, r.h[f] = g / (1.0 + std::exp(-g)) * u;
+  }
+  for (int64_t d = 0; d < D; ++d) {
+    double acc = 0.0;
+    for (int64_t f = 0; f < F; ++f) acc += down[d * F + f] * r.h[f];
+    r.o[d] = acc;
+  }
+}
+
+// Backward of one expert applied to one token with output gradient do_ (already scaled by p):
+// dg, du [F] and this expert's contribution to dx (added into dx).
+void expert_bwd_f64(const double* gate_up, const double* down, int64_t D, int64_t F, const ExpertFwd& r,
+                    const double* do_, double* dg, double* du, double* dx) {
+  for (int64_t f = 0; f < F; ++f) {
+    double dh = 0.0;
+    for (int64_t d = 0; d < D; ++d) dh += down[d * F + f] * do_[d];
+    const double sg = 1.0 / (1.0 + std::exp(-r.g[f]));
+    const double silu = r.g[f] * sg;
+    const double dsilu = sg * (1.0 + r.g[f] * (1.0 - sg));
+    dg[f] = dh * r.u[f] * dsilu;
+    du[f] = dh * silu;
+  }
+  for (int64_t d = 0; d < D; ++d) {
+    double acc = 0.0;
+    for (int64_t f = 0; f < F; ++f) acc += gate_up[f * D + d] * dg[f] + gate_up[(F + f) * D + d] * du[f];
+    dx[d] += acc;
+  }
+}
+
+}  // namespace
+
+// fp64-parameter forward: the same definition as oracle_layer.  gate_up [E, 2F, D], down [E, D, F],
+// shared_* may be NULL (Fs = 0).  Returns 0, or -1 on invalid sizes.
+int oracle_layer_f64(const double* x, const double* wg, const float* bias, const double* gate_up,
+                     const double* down, const double* shared_gate_up, const double* shared_down, int64_t T,
+                     int64_t D, int E, int k, int64_t F, int64_t Fs, double* y, int nthreads) {
+  if (T < 0 || D < 1 || E < 1 || k < 1 || k > E || F < 1 || Fs < 0) return -1;
+  for_tokens(T, nthreads, [&](int64_t t) {
+    std::vector<double> l(E), p(k), yt(D, 0.0);
+    std::vector<int32_t> idx(k);
+    ExpertFwd r;
+    router_logits_f64(x + t * D, wg, D, E, l.data());
+    select_and_weight(l.data(), bias, E, k, idx.data(), p.data());
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[j];
+      expert_fwd_f64(x + t * D, gate_up + (int64_t)e * 2 * F * D, down + (int64_t)e * D * F, D, F, r);
+      for (int64_t d = 0; d < D; ++d) yt[d] += p[j] * r.o[d];
+    }
+    if (Fs > 0 && shared_gate_up && shared_down) {
+      expert_fwd_f64(x + t * D, shared_gate_up, shared_down, D, Fs, r);
+      for (int64_t d = 0; d < D; ++d) yt[d] += r.o[d];
+    }
+    std::copy(yt.begin(), yt.end(), y + t * D);
+  });
+  return 0;
+}
+
+// Gradients of L = sum(dy * y) (definitions above).  Outputs (overwritten, fp64): dx [T, D],
+// dwg [E, D], dgate_up [E, 2F, D], ddown [E, D, F], dshared_gate_up [2Fs, D], dshared_down [D, Fs]
+// (the last two may be NULL when Fs = 0).  Weight gradients are summed over tokens in token
+// order.  Returns 0, or -1 on invalid sizes.
+int oracle_layer_backward_f64(const double* x, const double* wg, const float* bias, const double* gate_up,
+                              const double* down, const double* shared_gate_up, const double* shared_down,
+                              const double* dy, int64_t T, int64_t D, int E, int k, int64_t F, int64_t Fs,
+                              double* dx, double* dwg, double* dgate_up, double* ddown, double* dshared_gate_up,
+                              double* dshared_down, int nthreads) {
+  if (T < 0 || D < 1 || E < 1 || k < 1 || k > E || F < 1 || Fs < 0) return -1;
+  const bool sh = Fs > 0 && shared_gate_up && shared_down;
+  // per slot: expert, dl, do [D], h [F], dg [F], du [F]; per token (shared): do = dy, h, dg, du
+  std::vector<int32_t> idx(T * k);
+  std::vector<double> dl(T * k), slot_do(T * k * D), slot_h(T * k * F), slot_dg(T * k * F), slot_du(T * k * F);
+  std::vector<double> sh_h(sh ? T * Fs : 0), sh_dg(sh ? T * Fs : 0), sh_du(sh ? T * Fs : 0);
+  for_tokens(T, nthreads, [&](int64_t t) {
+    const double* xt = x + t * D;
+    const double* dyt = dy + t * D;
+    double* dxt = dx + t * D;
+    std::fill(dxt, dxt + D, 0.0);
+    std::vector<double> l(E), p(k), dp(k);
+    ExpertFwd r;
+    router_logits_f64(xt, wg, D, E, l.data());
+    select_and_weight(l.data(), bias, E, k, &idx[t * k], p.data());
+    for (int j = 0; j < k; ++j) {
+      const int64_t slot = t * k + j;
+      const int e = idx[slot];
+      const double* gu = gate_up + (int64_t)e * 2 * F * D;
+      const double* dn = down + (int64_t)e * D * F;
+      expert_fwd_f64(xt, gu, dn, D, F, r);
+      double dpj = 0.0;
+      for (int64_t d = 0; d < D; ++d) dpj += dyt[d] * r.o[d];
+      dp[j] = dpj;
+      double* dos = &slot_do[slot * D];
+      for (int64_t d = 0; d < D; ++d) dos[d] = p[j] * dyt[d];
+      std::copy(r.h.begin(), r.h.end(), &slot_h[slot * F]);
+      expert_bwd_f64(gu, dn, D, F, r, dos, &slot_dg[slot * F], &slot_du[slot * F], dxt);
+    }
+    double s = 0.0;
+    for (int j = 0; j < k; ++j) s += p[j] * dp[j];
+    for (int j = 0; j < k; ++j) {
+      const double dlj = p[j] * (dp[j] - s);
+      dl[t * k + j] = dlj;
+      const double* w = wg + (int64_t)idx[t * k + j] * D;
+      for (int64_t d = 0; d < D; ++d) dxt[d] += dlj * w[d];
+    }
+    if (sh) {
+      expert_fwd_f64(xt, shared_gate_up, shared_down, D, Fs, r);
+      std::copy(r.h.begin(), r.h.end(), &sh_h[t * Fs]);
+      expert_bwd_f64(shared_gate_up, shared_down, D, Fs, r, dyt, &sh_dg[t * Fs], &sh_du[t * Fs], dxt);
+    }
+  });
+  // weight gradients: one expert per task, its slots in token order
+  for_tokens(E, nthreads, [&](int64_t e) {
+    double* dgu = dgate_up + e * 2 * F * D;
+    double* ddn = ddown + e * D * F;
+    double* dw = dwg + e * D;
+    std::fill(dgu, dgu + 2 * F * D, 0.0);
+    std::fill(ddn, ddn + D * F, 0.0);
+    std::fill(dw, dw + D, 0.0);
+    for (int64_t slot = 0; slot < T * k; ++slot) {
+      if (idx[slot] != e) continue;
+      const double* xt = x + (slot / k) * D;
+      const double* dos = &slot_do[slot * D];
+      const double* h = &slot_h[slot * F];
+      const double* dg = &slot_dg[slot * F];
+      const double* du = &slot_du[slot * F];
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t f = 0; f < F; ++f) ddn[d * F + f] += dos[d] * h[f];
+      for (int64_t f = 0; f < F; ++f)
+        for (int64_t d = 0; d < D; ++d) {
+          dgu[f * D + d] += dg[f] * xt[d];
+          dgu[(F + f) * D + d] += du[f] * xt[d];
+        }
+      for (int64_t d = 0; d < D; ++d) dw[d] += dl[slot] * xt[d];
+    }
+  });
+  if (sh) {
+    std::fill(dshared_gate_up, dshared_gate_up + 2 * Fs * D, 0.0);
+    std::fill(dshared_down, dshared_down + D * Fs, 0.0);
+    for (int64_t t = 0; t < T; ++t) {
+      const double* xt = x + t * D;
+      const double* dyt = dy + t * D;
+      for (int64_t d = 0; d < D; ++d)
+        for (int64_t f = 0; f < Fs; ++f) dshared_down[d * Fs + f] += dyt[d] * sh_h[t * Fs + f];
+      for (int64_t f = 0; f < Fs; ++f)
+        for (int64_t d = 0; d < D; ++d) {
+          dshared_gate_up[f * D + d] += sh_dg[t * Fs + f] * xt[d];
+          dshared_gate_up[(Fs + f) * D + d] += sh_du[t * Fs + f] * xt[d];
+        }
+    }
+  }
+  return 0;
+}
+
 }  // extern "C"

@@ -369,3 +369,83 @@ def test_fp8_ffn_equals_bf16_ffn_on_exactly_representable_weights():
     gq, gs = oracle.quantize_rows_fp8(gu)
     dq, ds = oracle.quantize_rows_fp8(dn)
     np.testing.assert_array_equal(oracle.expert_ffn_fp8(x, gq, gs, dq, ds), oracle.expert_ffn(x, gu, dn))
+
+
+# ----------------------------------------------------------------------------- backward pass
+def _bwd_problem(seed=0, T=6, D=16, E=6, k=2, F=8, Fs=8, bias=True):
+    """A small fp64 problem whose top-k choices are separated by at least 0.05 in score, so that the
+    finite-difference steps below cannot change the selection."""
+    rng = np.random.default_rng(seed)
+    for _ in range(200):
+        x = rng.normal(size=(T, D))
+        wg = rng.normal(size=(E, D)) * 0.5
+        b = (rng.normal(size=E) * 0.3).astype(np.float32) if bias else None
+        s = x @ wg.T + (0.0 if b is None else b.astype(np.float64))
+        top = -np.sort(-s, axis=1)[:, : min(k + 1, E)]
+        if k == E or (np.diff(-top, axis=1) > 0.05).all():
+            break
+    gu = rng.normal(size=(E, 2 * F, D)) * 0.3
+    dn = rng.normal(size=(E, D, F)) * 0.3
+    sgu = rng.normal(size=(2 * Fs, D)) * 0.3 if Fs else None
+    sdn = rng.normal(size=(D, Fs)) * 0.3 if Fs else None
+    dy = rng.normal(size=(T, D))
+    return dict(x=x, wg=wg, bias=b, gu=gu, dn=dn, sgu=sgu, sdn=sdn, dy=dy, k=k)
+
+
+def _loss(P, **over):
+    q = dict(P, **over)
+    y = oracle.layer_f64(q["x"], q["wg"], q["bias"], q["gu"], q["dn"], q["k"], q["sgu"], q["sdn"])
+    return float(np.sum(P["dy"] * y))
+
+
+@pytest.mark.parametrize("k,Fs", [(2, 8), (3, 0), (1, 8)])
+def test_backward_matches_finite_differences_of_the_forward(k, Fs):
+    """<grad, V> equals the central difference of L = sum(dy * y) along a random V, for every
+    input and parameter tensor (the fp64 forward is smooth while the selection stays fixed)."""
+    P = _bwd_problem(seed=k + Fs, k=k, Fs=Fs)
+    g = oracle.layer_backward(P["x"], P["wg"], P["bias"], P["gu"], P["dn"], k, P["dy"], P["sgu"], P["sdn"])
+    rng = np.random.default_rng(99)
+    eps = 1e-5
+    pairs = [("x", "dx"), ("wg", "dw_gate"), ("gu", "dgate_up"), ("dn", "ddown")]
+    if Fs:
+        pairs += [("sgu", "dshared_gate_up"), ("sdn", "dshared_down")]
+    for name, key in pairs:
+        V = rng.normal(size=P[name].shape)
+        fd = (_loss(P, **{name: P[name] + eps * V}) - _loss(P, **{name: P[name] - eps * V})) / (2 * eps)
+        assert float(np.sum(g[key] * V)) == pytest.approx(fd, rel=1e-7, abs=1e-9), name
+
+
+def test_backward_router_gradient_invariants():
+    """The softmax over the chosen k is invariant to adding one constant to their logits, so for
+    every token the logit gradients sum to zero and sum_e dW_g[e] = 0; with k = 1 the single weight
+    is 1 and dW_g vanishes."""
+    P = _bwd_problem(seed=3, E=8, k=3)
+    g = oracle.layer_backward(P["x"], P["wg"], P["bias"], P["gu"], P["dn"], 3, P["dy"], P["sgu"], P["sdn"])
+    assert np.abs(g["dw_gate"].sum(axis=0)).max() < 1e-12 * max(1.0, np.abs(g["dw_gate"]).max())
+    assert np.abs(g["dw_gate"]).max() > 1e-3
+    P1 = _bwd_problem(seed=4, E=8, k=1)
+    g1 = oracle.layer_backward(P1["x"], P1["wg"], P1["bias"], P1["gu"], P1["dn"], 1, P1["dy"], P1["sgu"], P1["sdn"])
+    assert (g1["dw_gate"] == 0).all()
+
+
+def test_backward_leaves_unselected_experts_at_zero():
+    """Weights of experts that no token selects get no gradient; selected ones do."""
+    P = _bwd_problem(seed=5, T=3, E=12, k=2)
+    g = oracle.layer_backward(P["x"], P["wg"], P["bias"], P["gu"], P["dn"], 2, P["dy"], P["sgu"], P["sdn"])
+    s = P["x"] @ P["wg"].T + P["bias"].astype(np.float64)
+    chosen = set(np.argsort(-s, axis=1)[:, :2].reshape(-1).tolist())
+    for e in range(12):
+        nz = np.abs(g["dgate_up"][e]).max() > 0 and np.abs(g["ddown"][e]).max() > 0
+        assert nz == (e in chosen), e
+        assert (np.abs(g["dw_gate"][e]).max() > 0) == (e in chosen), e
+
+
+def test_f64_forward_is_the_bf16_forward():
+    """oracle.layer_f64 on exact bf16 values is the same function as oracle.layer."""
+    w = mi.Workload("t", T=9, D=64, E=8, k=2, F=32, Fs=32, bias="normal:0.5")
+    h = mi.host_inputs(w)
+    y16, _, _ = oracle.layer(h["x"], h["wg"], h["bias"], h["gate_up"], h["down"], 2, h["shared_gate_up"],
+                             h["shared_down"])
+    y64 = oracle.layer_f64(h["x"], h["wg"], h["bias"], h["gate_up"], h["down"], 2, h["shared_gate_up"],
+                           h["shared_down"])
+    np.testing.assert_allclose(y64, y16, rtol=1e-13, atol=1e-15)
