@@ -166,6 +166,10 @@ moe_status_t moe_combine(const float* out_perm, const int32_t* inv_perm, const f
  * ---------------------------------------------------------------------------------------- */
 #define MOE_FLAG_FORCE_PREFILL 1
 #define MOE_FLAG_FORCE_DECODE 2 /* only valid for T <= 64 */
+/* Training forward: keep in the workspace what moe_layer_backward needs (the routing, x_perm, h
+ * and the SwiGLU inputs g | u of the gate_up GEMMs, bf16).  Uses the tiled kernels at any T;
+ * bf16 weights only. */
+#define MOE_FLAG_SAVE_FOR_BACKWARD 4
 
 #define MOE_WEIGHTS_BF16 0     /* gate_up / down (and shared_*) hold bf16 weights            */
 #define MOE_WEIGHTS_FP8_E4M3 1 /* *_fp8 hold E4M3 codes with one fp32 scale per weight row  */
@@ -231,6 +235,31 @@ moe_status_t moe_layer_forward_timed(const moe_layer_desc_t* desc, const moe_bf1
 
 /* Number of kernels one moe_layer_forward launches for this descriptor (0 if invalid). */
 int moe_layer_kernel_count(const moe_layer_desc_t* desc);
+
+/* ----------------------------------------------------------------------------------------
+ * Backward pass (training; keryc.com "Mixture of Experts optimiza...", section "Entrenamiento:
+ * todavia desafiante, pero con avances", dev.smart-guide.co.kr, section "Entrenamiento MoE: 12x
+ * Mas Rapido").  The pages give no formulas: the gradients are the chain rule of the forward, with
+ * L = sum(dy * y), no gradient through the top-k selection or the selection bias:
+ *   dx [T, D] bf16; dw_gate [E, D], dgate_up [E, 2F, D], ddown [E, D, F], dshared_gate_up [2Fs, D],
+ *   dshared_down [D, Fs] fp32 (overwritten, not accumulated; experts no token chose get zeros).
+ * Inputs: the descriptor of a forward run with MOE_FLAG_SAVE_FOR_BACKWARD on the same x, and that
+ * forward's workspace (fwd_ws, read only; the saved state), dy [T, D] bf16.  bwd_ws:
+ * >= moe_layer_backward_workspace_size(desc) bytes, 256-byte aligned, its first 256 bytes the
+ * device error word (moe_get_device_error).  Device pointers; asynchronous on `stream`.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct {
+  float* dw_gate;          /* [E, D]                  */
+  float* dgate_up;         /* [E, 2F, D]              */
+  float* ddown;            /* [E, D, F]               */
+  float* dshared_gate_up;  /* [2Fs, D] or NULL (Fs=0) */
+  float* dshared_down;     /* [D, Fs] or NULL (Fs=0)  */
+} moe_layer_grads_t;
+
+size_t moe_layer_backward_workspace_size(const moe_layer_desc_t* desc);
+moe_status_t moe_layer_backward(const moe_layer_desc_t* desc, const moe_bf16_t* x, const moe_bf16_t* dy,
+                                moe_bf16_t* dx, const moe_layer_grads_t* grads, const void* fwd_ws,
+                                size_t fwd_ws_bytes, void* bwd_ws, size_t bwd_ws_bytes, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
  * Aux-loss-free balancing (gotburnout.io glossary "MoE", section 2 item 4: router biases are

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_FLAG_FORCE_PREFILL = 1
 MOE_FLAG_FORCE_DECODE = 2
+MOE_FLAG_SAVE_FOR_BACKWARD = 4
 MOE_WEIGHTS_BF16 = 0
 MOE_WEIGHTS_FP8_E4M3 = 1
 
@@ -32,9 +33,14 @@ EXPORTS = (
     "moe_grouped_swiglu_ffn_workspace_size",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_layer_workspace_size", "moe_layer_forward",
     "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_update_router_bias",
-    "moe_layer_expert_counts", "moe_get_device_error",
+    "moe_layer_expert_counts", "moe_get_device_error", "moe_layer_backward_workspace_size", "moe_layer_backward",
     "moe_status_string",
 )
+
+
+class LayerGrads(ctypes.Structure):
+    """moe_layer_grads_t: fp32 gradient outputs (device pointers)."""
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dw_gate", "dgate_up", "ddown", "dshared_gate_up", "dshared_down")]
 
 
 class MoeError(RuntimeError):
@@ -87,6 +93,8 @@ def lib():
             "moe_update_router_bias": ([P, I, ctypes.c_float, P, P], I),
             "moe_layer_expert_counts": ([ctypes.POINTER(LayerDesc), P, Z, ctypes.POINTER(P)], I),
             "moe_get_device_error": ([P, P], I),
+            "moe_layer_backward_workspace_size": ([ctypes.POINTER(LayerDesc)], Z),
+            "moe_layer_backward": ([ctypes.POINTER(LayerDesc), P, P, P, ctypes.POINTER(LayerGrads), P, Z, P, Z, P], I),
             "moe_status_string": ([I], ctypes.c_char_p),
         }
         for name, (args, res) in sig.items():
@@ -340,6 +348,40 @@ class MoELayer:
                "moe_layer_expert_counts")
         off = ptr.value - ws.data_ptr()
         return ws[off:off + 4 * self.E].view(torch.int32)
+
+    def backward(self, x, dy, stream=None):
+        """Gradients of sum(dy * y) after forward(x) on a layer built with
+        flags=MOE_FLAG_SAVE_FOR_BACKWARD: (dx [T, D] bf16, dict of fp32 weight gradients
+        dw_gate, dgate_up, ddown, dshared_gate_up, dshared_down (None without a shared expert))."""
+        import torch
+
+        T = x.shape[0]
+        _need(dy, torch.bfloat16, (T, self.D), "dy")
+        d = self.desc(T)
+        need = lib().moe_layer_backward_workspace_size(ctypes.byref(d))
+        if need == 0:
+            raise MoeError(1, "moe_layer_backward_workspace_size")
+        if getattr(self, "_bws", None) is None or self._bws.numel() < need:
+            self._bws = torch.zeros(need, dtype=torch.uint8, device=x.device)
+        dev, f32 = x.device, torch.float32
+        g = dict(dw_gate=torch.empty(self.E, self.D, dtype=f32, device=dev),
+                 dgate_up=torch.empty(self.E, 2 * self.F, self.D, dtype=f32, device=dev),
+                 ddown=torch.empty(self.E, self.D, self.F, dtype=f32, device=dev),
+                 dshared_gate_up=torch.empty(2 * self.Fs, self.D, dtype=f32, device=dev) if self.Fs else None,
+                 dshared_down=torch.empty(self.D, self.Fs, dtype=f32, device=dev) if self.Fs else None)
+        grads = LayerGrads(*[_ptr(g[n]) for n in ("dw_gate", "dgate_up", "ddown", "dshared_gate_up", "dshared_down")])
+        dx = torch.empty_like(x)
+        ws = self.workspace(T)
+        _check(lib().moe_layer_backward(ctypes.byref(d), x.data_ptr(), dy.data_ptr(), dx.data_ptr(), ctypes.byref(grads),
+                                        ws.data_ptr(), ws.numel(), self._bws.data_ptr(), self._bws.numel(),
+                                        _stream(stream)), "moe_layer_backward")
+        return dx, g
+
+    def backward_error(self, stream=None) -> int:
+        """Synchronises and returns (and clears) the backward workspace's device error status."""
+        if getattr(self, "_bws", None) is None:
+            return 0
+        return lib().moe_get_device_error(self._bws.data_ptr(), _stream(stream))
 
     def device_error(self, stream=None) -> int:
         """Synchronises and returns (and clears) the workspace's device error status."""

@@ -65,6 +65,7 @@ struct alignas(64) GemmParams {
   int k_blocks[2];  // K / 64 per set (down: F routed, Fs shared)
   int ld_out[2];    // row stride of the output (elements)
   int k_splits;     // kRouter: K is split into this many contiguous k-block ranges
+  uint16_t* save_gu[2];  // tiled kGateUp in a training forward: g | u [rows, 2F] bf16, or NULL
   int n_sets;
   int withhold_first_load;  // test only: never issue the first stage's copies (its wait then times out)
   int* err;
@@ -352,6 +353,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             tmem_ld_32x32b_x32(tacc + c0, g);
             tmem_ld_32x32b_x32(tacc + 128 + c0, u);
             tmem_ld_wait();
+            if (row_ok && p.save_gu[ti.set] != nullptr) {  // the backward pass's SwiGLU inputs
+              uint16_t* srow = p.save_gu[ti.set] + grow * 2 * n_out;
+              uint32_t gk[16], uk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                gk[i] = pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                uk[i] = pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+              }
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                reinterpret_cast<uint4*>(srow + col)[v] = make_uint4(gk[4 * v], gk[4 * v + 1], gk[4 * v + 2], gk[4 * v + 3]);
+                reinterpret_cast<uint4*>(srow + n_out + col)[v] =
+                    make_uint4(uk[4 * v], uk[4 * v + 1], uk[4 * v + 2], uk[4 * v + 3]);
+              }
+            }
             if (row_ok) {
               uint32_t pk[16];
 #pragma unroll
@@ -528,6 +544,7 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int
     p.out[i] = st.out;
     p.row_scale[i] = st.row_scale;
     p.ld_out[i] = st.ld_out > 0 ? st.ld_out : st.n_out;
+    p.save_gu[i] = (KIND == kGateUp && NT == 0) ? st.save_gu : nullptr;
     p.n_groups[i] = st.n_groups;
     p.m_rows[i] = st.m_rows;
     p.n_out[i] = st.n_out;

@@ -134,9 +134,44 @@ struct GemmSetHost {
   void* out;                // [rows, n_out]: bf16 (gate_up -> h) or fp32 (down)
   const float* row_scale;   // per-row factor (down) or NULL
   int ld_out;               // output row stride in elements (0: n_out)
+  uint16_t* save_gu = nullptr;  // tiled gate_up, training: also store g | u [rows, 2 * n_out] bf16
 };
 
 enum GemmKind { kGateUp = 0, kDown = 1, kRouter = 2 };
+
+// ---- backward pass (grouped_gemm_bwd_sm100.cu, layer_backward.cu) ----------------------------
+enum BwdKind { kBwdDxDown = 0, kBwdDxGateUp = 1, kBwdDwDown = 2, kBwdDwGateUp = 3 };
+
+// One operand set of a backward GEMM launch (set 0: the routed experts, set 1: the shared expert).
+struct BwdSetHost {
+  const void* a = nullptr;  // bf16 A storage [a_rows, a_cols]
+  int64_t a_rows = 0;
+  int a_cols = 0;
+  const void* b = nullptr;  // bf16 B storage [b_rows, b_cols] (contracted index = row)
+  int64_t b_rows = 0;
+  int b_cols = 0;
+  const int32_t* offsets = nullptr;      // groups' unpadded rows (NULL: one group of m_rows rows)
+  const int32_t* pad_offsets = nullptr;  // groups' rows in the 64-row padded layout
+  int n_groups = 1, m_rows = 0;
+  int K = 0, M_total = 0, N_total = 0;
+  const float* p_perm = nullptr;
+  const uint16_t* gu_saved = nullptr;
+  uint16_t* dgu = nullptr;
+  float* dp_part = nullptr;
+  float* out = nullptr;
+};
+cudaError_t launch_bwd_gemm(BwdKind kind, const BwdSetHost* sets, int n_sets, int* err, cudaStream_t s);
+cudaError_t launch_pad_offsets(const int32_t* offsets, int E, int32_t* pad_offsets, cudaStream_t s);
+cudaError_t launch_gather_dy(const uint16_t* dy, const int32_t* offsets, const int32_t* pad_offsets, int E,
+                             const int32_t* perm_token, const float* p_perm, int D, int F2, long long rows_bound,
+                             uint16_t* dyp, uint16_t* dO, uint16_t* dgu, cudaStream_t s);
+cudaError_t launch_router_bwd(const int32_t* inv_perm, const float* topk_w, const float* dp_part, int n_tiles, int T,
+                              int k, float* dl_row, cudaStream_t s);
+cudaError_t launch_dwgate(const int32_t* offsets, const float* dl_row, const uint16_t* x_perm, int E, int D,
+                          float* dwg, cudaStream_t s);
+cudaError_t launch_unpermute(const float* dxp, const float* dx_sh, const int32_t* inv_perm, const int32_t* topk_idx,
+                             const int32_t* offsets, const int32_t* pad_offsets, const float* dl_row, const uint16_t* wg,
+                             int T, int D, int k, uint16_t* dx, cudaStream_t s);
 
 // Launch one grouped GEMM (gate_up + SwiGLU, or down + row scale) over up to two sets.
 // decode_nt > 0 selects the weight-streaming

@@ -39,6 +39,7 @@ moe_status_t shape_status(long long T, long long D, long long E, long long k) {
 }
 
 bool use_decode(const moe_layer_desc_t& d) {
+  if (d.flags & MOE_FLAG_SAVE_FOR_BACKWARD) return false;  // the tiled kernels save g | u
   if (d.flags & MOE_FLAG_FORCE_DECODE) return true;
   if (d.flags & MOE_FLAG_FORCE_PREFILL) return false;
   return d.T <= kDecodeTMax;
@@ -47,7 +48,7 @@ bool use_decode(const moe_layer_desc_t& d) {
 int decode_tile(int max_seg) { return ((max_seg + 15) / 16) * 16; }
 
 struct LayerWs {
-  size_t split_counters, split_partial, split_partial_bytes, router, topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
+  size_t split_counters, split_partial, split_partial_bytes, gu_saved, gu_saved_sh, router, topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
       out_sh, x16, x_stage, y_stage, total;
 };
 
@@ -68,6 +69,10 @@ LayerWs layer_ws(const moe_layer_desc_t& d) {
                               ? (size_t)kMaxSplitItems * 2 * decode_tile(d.T) * 128 * sizeof(float)
                               : 0;
   w.split_partial = take(w.split_partial_bytes);
+  // training forward: the SwiGLU inputs g | u of the routed rows and of the shared expert (bf16)
+  const bool save = (d.flags & MOE_FLAG_SAVE_FOR_BACKWARD) != 0;
+  w.gu_saved = take(save ? M * 2 * F * 2 : 0);
+  w.gu_saved_sh = take(save ? T * 2 * Fs * 2 : 0);
   w.router = take(router_scratch_bytes(d.T, d.D, d.E));
   w.topk_idx = take(M * 4);
   w.topk_w = take(M * 4);
@@ -108,7 +113,7 @@ moe_status_t validate_desc(const moe_layer_desc_t* d) {
     if (sh != (d->shared_gate_up_fp8 != nullptr) || sh != (d->shared_down_fp8 != nullptr) ||
         sh != (d->shared_gate_up_scale != nullptr) || sh != (d->shared_down_scale != nullptr))
       return MOE_ERR_INVALID_ARG;
-    if (d->flags & MOE_FLAG_FORCE_PREFILL) return MOE_ERR_INVALID_ARG;
+    if (d->flags & (MOE_FLAG_FORCE_PREFILL | MOE_FLAG_SAVE_FOR_BACKWARD)) return MOE_ERR_INVALID_ARG;
     if (d->T > kDecodeTMax) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!aligned(d->gate_up_fp8, 16) || !aligned(d->down_fp8, 16) || !aligned(d->shared_gate_up_fp8, 16) ||
         !aligned(d->shared_down_fp8, 16) || !aligned(d->gate_up_scale, 4) || !aligned(d->down_scale, 4) ||
@@ -117,7 +122,9 @@ moe_status_t validate_desc(const moe_layer_desc_t* d) {
   } else {
     return MOE_ERR_INVALID_ARG;
   }
-  if ((d->flags & ~(MOE_FLAG_FORCE_PREFILL | MOE_FLAG_FORCE_DECODE)) != 0) return MOE_ERR_INVALID_ARG;
+  if ((d->flags & ~(MOE_FLAG_FORCE_PREFILL | MOE_FLAG_FORCE_DECODE | MOE_FLAG_SAVE_FOR_BACKWARD)) != 0)
+    return MOE_ERR_INVALID_ARG;
+  if ((d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && (d->flags & MOE_FLAG_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_FORCE_PREFILL) && (d->flags & MOE_FLAG_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_FORCE_DECODE) && d->T > kDecodeTMax) return MOE_ERR_INVALID_ARG;
   if (!aligned(d->w_gate, 16) || !aligned(d->gate_up, 16) || !aligned(d->down, 16) ||
@@ -140,15 +147,15 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
                      // optional shared expert over x[T, D]
                      const uint16_t* x, int T, int Fs, const uint16_t* sgu, const uint16_t* sdn, uint16_t* h_sh,
                      float* out_sh, int decode_nt, int* err, cudaStream_t s, cudaEvent_t ev_mid,
-                     unsigned ev_flags) {
+                     unsigned ev_flags, uint16_t* save_gu = nullptr, uint16_t* save_gu_sh = nullptr) {
   GemmSetHost g[2];
   memset(g, 0, sizeof(g));
   g[0].K = D, g[0].a = x_perm, g[0].a_rows = M, g[0].w = gate_up, g[0].n_groups = E, g[0].offsets = offsets;
-  g[0].n_out = F, g[0].out = h;
+  g[0].n_out = F, g[0].out = h, g[0].save_gu = save_gu;
   int n_sets = 1;
   if (Fs > 0) {
     g[1].K = D, g[1].a = x, g[1].a_rows = T, g[1].w = sgu, g[1].n_groups = 1, g[1].m_rows = T;
-    g[1].n_out = Fs, g[1].out = h_sh;
+    g[1].n_out = Fs, g[1].out = h_sh, g[1].save_gu = save_gu_sh;
     n_sets = 2;
   }
   MOE_CUDA_TRY(launch_grouped_gemm(kGateUp, g, n_sets, decode_nt, err, s));
@@ -241,12 +248,53 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
   } else {
   st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), Fp(w.out_perm), x,
                T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, err, s, ev ? ev[3] : nullptr,
-               rec_flags);
+               rec_flags, (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) ? H(w.gu_saved) : nullptr,
+               (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && Fs > 0 ? H(w.gu_saved_sh) : nullptr);
   if (st != MOE_OK) return st;
   }
   if (ev) MOE_CUDA_TRY(record(ev[4]));
   MOE_CUDA_TRY(launch_combine(Fp(w.out_perm), I(w.inv_perm), Fs > 0 ? Fp(w.out_sh) : nullptr, T, D, k, y, s));
   if (ev) MOE_CUDA_TRY(record(ev[5]));
+  return MOE_OK;
+}
+
+// Backward workspace: per-row gradients in the 64-row padded per-expert layout (rows_pad rows at
+// most: every expert pads fewer than 64 rows).
+struct BwdWs {
+  size_t pad_offsets, dyp, d_o, dgu, dxp, dp_part, dl_row, dgu_sh, dx_sh, total;
+  int64_t rows_pad;
+  int n_tiles;  // 256-column tiles of F: the partial dp per row
+};
+
+BwdWs bwd_ws(const moe_layer_desc_t& d) {
+  BwdWs b;
+  size_t o = kWsHeader;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  const size_t T = d.T, D = d.D, E = d.E, k = d.k, F = d.F, Fs = d.Fs, M = T * k;
+  b.rows_pad = (int64_t)M + 64 * (int64_t)E;
+  b.n_tiles = (d.F + 255) / 256;
+  const size_t R = (size_t)b.rows_pad;
+  b.pad_offsets = take((E + 1) * 4);
+  b.dyp = take(R * D * 2);
+  b.d_o = take(R * D * 2);
+  b.dgu = take(R * 2 * F * 2);
+  b.dxp = take(R * D * 4);
+  b.dp_part = take(M * b.n_tiles * 4);
+  b.dl_row = take(M * 4);
+  b.dgu_sh = take(T * 2 * Fs * 2);
+  b.dx_sh = take(T * D * 4);
+  b.total = o;
+  return b;
+}
+
+moe_status_t validate_backward(const moe_layer_desc_t* d) {
+  moe_status_t st = validate_desc(d);
+  if (st != MOE_OK) return st;
+  if (!(d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) || d->weight_format != MOE_WEIGHTS_BF16) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -439,6 +487,117 @@ moe_status_t moe_layer_expert_counts(const moe_layer_desc_t* desc, void* ws, siz
   const LayerWs w = layer_ws(*desc);
   if (ws_bytes < w.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   *counts = reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(ws) + w.counts);
+  return MOE_OK;
+}
+
+size_t moe_layer_backward_workspace_size(const moe_layer_desc_t* desc) {
+  if (validate_backward(desc) != MOE_OK) return 0;
+  return bwd_ws(*desc).total;
+}
+
+moe_status_t moe_layer_backward(const moe_layer_desc_t* desc, const moe_bf16_t* x, const moe_bf16_t* dy,
+                                moe_bf16_t* dx, const moe_layer_grads_t* grads, const void* fwd_ws,
+                                size_t fwd_ws_bytes, void* bwd_ws_ptr, size_t bwd_ws_bytes, moe_stream_t stream) {
+  moe_status_t st = validate_backward(desc);
+  if (st != MOE_OK) return st;
+  const moe_layer_desc_t& d = *desc;
+  if (!x || !dy || !dx || !grads || !fwd_ws || !bwd_ws_ptr || !grads->dw_gate || !grads->dgate_up || !grads->ddown)
+    return MOE_ERR_INVALID_ARG;
+  if ((d.Fs > 0) != (grads->dshared_gate_up != nullptr) || (d.Fs > 0) != (grads->dshared_down != nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(dy, 16) || !aligned(dx, 16) || !aligned(grads->dw_gate, 16) ||
+      !aligned(grads->dgate_up, 16) || !aligned(grads->ddown, 16) || !aligned(grads->dshared_gate_up, 16) ||
+      !aligned(grads->dshared_down, 16) || !aligned(fwd_ws, 256) || !aligned(bwd_ws_ptr, 256))
+    return MOE_ERR_ALIGNMENT;
+  const LayerWs w = layer_ws(d);
+  const BwdWs b = bwd_ws(d);
+  if (fwd_ws_bytes < w.total || bwd_ws_bytes < b.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = check_device()) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int T = d.T, D = d.D, E = d.E, k = d.k, F = d.F, Fs = d.Fs, M = T * k;
+  const size_t nd = (size_t)E * D, ngu = (size_t)E * 2 * F * D, ndn = (size_t)E * D * F;
+  if (T == 0) {  // no tokens: every gradient is zero
+    MOE_CUDA_TRY(cudaMemsetAsync(grads->dw_gate, 0, nd * 4, s));
+    MOE_CUDA_TRY(cudaMemsetAsync(grads->dgate_up, 0, ngu * 4, s));
+    MOE_CUDA_TRY(cudaMemsetAsync(grads->ddown, 0, ndn * 4, s));
+    if (Fs > 0) {
+      MOE_CUDA_TRY(cudaMemsetAsync(grads->dshared_gate_up, 0, (size_t)2 * Fs * D * 4, s));
+      MOE_CUDA_TRY(cudaMemsetAsync(grads->dshared_down, 0, (size_t)D * Fs * 4, s));
+    }
+    return MOE_OK;
+  }
+  const uint8_t* f = static_cast<const uint8_t*>(fwd_ws);
+  uint8_t* bb = static_cast<uint8_t*>(bwd_ws_ptr);
+  auto FI = [&](size_t off) { return reinterpret_cast<const int32_t*>(f + off); };
+  auto FF = [&](size_t off) { return reinterpret_cast<const float*>(f + off); };
+  auto FH = [&](size_t off) { return reinterpret_cast<const uint16_t*>(f + off); };
+  auto BI = [&](size_t off) { return reinterpret_cast<int32_t*>(bb + off); };
+  auto BF = [&](size_t off) { return reinterpret_cast<float*>(bb + off); };
+  auto BH = [&](size_t off) { return reinterpret_cast<uint16_t*>(bb + off); };
+  int* err = reinterpret_cast<int*>(bb);
+  const int32_t* offsets = FI(w.offsets);
+  int32_t* pad = BI(b.pad_offsets);
+  const int n_sets = Fs > 0 ? 2 : 1;
+
+  MOE_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+  MOE_CUDA_TRY(launch_pad_offsets(offsets, E, pad, s));
+  MOE_CUDA_TRY(launch_gather_dy(dy, offsets, pad, E, FI(w.perm_token), FF(w.p_perm), D, 2 * F, b.rows_pad,
+                                BH(b.dyp), BH(b.d_o), BH(b.dgu), s));
+  // dHu = dy_perm Down_e, fused SwiGLU backward -> dGU, partial dp
+  BwdSetHost st2[2];
+  st2[0].a = BH(b.dyp), st2[0].a_rows = b.rows_pad, st2[0].a_cols = D;
+  st2[0].b = d.down, st2[0].b_rows = (int64_t)E * D, st2[0].b_cols = F;
+  st2[0].offsets = offsets, st2[0].pad_offsets = pad, st2[0].n_groups = E;
+  st2[0].K = D, st2[0].N_total = F, st2[0].p_perm = FF(w.p_perm), st2[0].gu_saved = FH(w.gu_saved);
+  st2[0].dgu = BH(b.dgu), st2[0].dp_part = BF(b.dp_part);
+  if (Fs > 0) {
+    st2[1].a = dy, st2[1].a_rows = T, st2[1].a_cols = D;
+    st2[1].b = d.shared_down, st2[1].b_rows = D, st2[1].b_cols = Fs;
+    st2[1].m_rows = T, st2[1].K = D, st2[1].N_total = Fs, st2[1].gu_saved = FH(w.gu_saved_sh);
+    st2[1].dgu = BH(b.dgu_sh);
+  }
+  MOE_CUDA_TRY(launch_bwd_gemm(kBwdDxDown, st2, n_sets, err, s));
+  // dX = dGU gate_up_e
+  BwdSetHost sx[2];
+  sx[0].a = BH(b.dgu), sx[0].a_rows = b.rows_pad, sx[0].a_cols = 2 * F;
+  sx[0].b = d.gate_up, sx[0].b_rows = (int64_t)E * 2 * F, sx[0].b_cols = D;
+  sx[0].offsets = offsets, sx[0].pad_offsets = pad, sx[0].n_groups = E;
+  sx[0].K = 2 * F, sx[0].N_total = D, sx[0].out = BF(b.dxp);
+  if (Fs > 0) {
+    sx[1].a = BH(b.dgu_sh), sx[1].a_rows = T, sx[1].a_cols = 2 * Fs;
+    sx[1].b = d.shared_gate_up, sx[1].b_rows = 2 * Fs, sx[1].b_cols = D;
+    sx[1].m_rows = T, sx[1].K = 2 * Fs, sx[1].N_total = D, sx[1].out = BF(b.dx_sh);
+  }
+  MOE_CUDA_TRY(launch_bwd_gemm(kBwdDxGateUp, sx, n_sets, err, s));
+  // dDown_e = dO_e^T h_e
+  BwdSetHost sd[2];
+  sd[0].a = BH(b.d_o), sd[0].a_rows = b.rows_pad, sd[0].a_cols = D;
+  sd[0].b = FH(w.h), sd[0].b_rows = M, sd[0].b_cols = F;
+  sd[0].offsets = offsets, sd[0].pad_offsets = pad, sd[0].n_groups = E;
+  sd[0].M_total = D, sd[0].N_total = F, sd[0].out = grads->ddown;
+  if (Fs > 0) {
+    sd[1].a = dy, sd[1].a_rows = T, sd[1].a_cols = D;
+    sd[1].b = FH(w.h_sh), sd[1].b_rows = T, sd[1].b_cols = Fs;
+    sd[1].m_rows = T, sd[1].M_total = D, sd[1].N_total = Fs, sd[1].out = grads->dshared_down;
+  }
+  MOE_CUDA_TRY(launch_bwd_gemm(kBwdDwDown, sd, n_sets, err, s));
+  // dGateUp_e = dGU_e^T x_perm_e
+  BwdSetHost su[2];
+  su[0].a = BH(b.dgu), su[0].a_rows = b.rows_pad, su[0].a_cols = 2 * F;
+  su[0].b = FH(w.x_perm), su[0].b_rows = M, su[0].b_cols = D;
+  su[0].offsets = offsets, su[0].pad_offsets = pad, su[0].n_groups = E;
+  su[0].M_total = 2 * F, su[0].N_total = D, su[0].out = grads->dgate_up;
+  if (Fs > 0) {
+    su[1].a = BH(b.dgu_sh), su[1].a_rows = T, su[1].a_cols = 2 * Fs;
+    su[1].b = x, su[1].b_rows = T, su[1].b_cols = D;
+    su[1].m_rows = T, su[1].M_total = 2 * Fs, su[1].N_total = D, su[1].out = grads->dshared_gate_up;
+  }
+  MOE_CUDA_TRY(launch_bwd_gemm(kBwdDwGateUp, su, n_sets, err, s));
+  // router: dp -> dl (softmax over the chosen k), dW_g, and dx
+  MOE_CUDA_TRY(launch_router_bwd(FI(w.inv_perm), FF(w.topk_w), BF(b.dp_part), b.n_tiles, T, k, BF(b.dl_row), s));
+  MOE_CUDA_TRY(launch_dwgate(offsets, BF(b.dl_row), FH(w.x_perm), E, D, grads->dw_gate, s));
+  MOE_CUDA_TRY(launch_unpermute(BF(b.dxp), Fs > 0 ? BF(b.dx_sh) : nullptr, FI(w.inv_perm), FI(w.topk_idx), offsets,
+                                pad, BF(b.dl_row), d.w_gate, T, D, k, dx, s));
   return MOE_OK;
 }
 
