@@ -421,6 +421,87 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     del graph, graph_plain
 
 
+def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
+    """A training step: the forward that saves the backward's inputs, then moe_layer_backward (dx and
+    the fp32 weight gradients), each a CUDA graph, replayed back to back with events between them."""
+    import torch
+
+    import sparse_mixture_experts_16_b200 as moe
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    pk, pk_kind = peaks()
+    with torch.cuda.stream(stream):
+        inp = mi.device_inputs(w, device=dev)
+        layer = moe.MoELayer(inp["wg"], inp["gate_up"], inp["down"], w.k, bias=inp["bias"],
+                             shared_gate_up=inp["shared_gate_up"], shared_down=inp["shared_down"],
+                             flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD)
+        x = inp["x"]
+        y = torch.empty_like(x)
+        dy = torch.empty_like(x)
+        mi.device_fill_rows_bf16(dy, mi.STREAM_X, 1.0, seed=w.seed + 1000)
+        for _ in range(max(args.warmup, 3)):
+            layer.forward(x, y, stream=stream)
+            dx, grads = layer.backward(x, dy, stream=stream)
+        stream.synchronize()
+        if layer.device_error(stream) != 0 or layer.backward_error(stream) != 0:
+            raise RuntimeError("device error during warm-up")
+        g_fwd, g_bwd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_fwd, stream=stream):
+            layer.forward(x, y, stream=stream)
+        with torch.cuda.graph(g_bwd, stream=stream):
+            layer.backward(x, dy, stream=stream)  # same output tensors: the layer keeps its workspaces
+        for _ in range(3):
+            g_fwd.replay()
+            g_bwd.replay()
+        stream.synchronize()
+    gpu_id = str(local_rank)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(gpu_id) as clk, torch.cuda.stream(stream):
+        for s in range(args.steps):
+            evs[s][0].record(stream)
+            g_fwd.replay()
+            evs[s][1].record(stream)
+            g_bwd.replay()
+            evs[s][2].record(stream)
+        stream.synchronize()
+    f_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in evs)
+    b_ms = statistics.mean(b.elapsed_time(c) for _, b, c in evs)
+    step_ms = f_ms + b_ms
+    gemm_fwd = w.T * (6.0 * w.k * w.D * w.F + 6.0 * w.D * w.Fs)
+    bwd_tflops = 2 * gemm_fwd / (b_ms / 1e3) / 1e12
+    peak = pk["bf16_tflops_sustained"]
+    n_fwd = layer.kernel_count(w.T)
+    n_bwd = 9  # pad offsets, dy gather, 4 grouped GEMMs, router backward, dW_g, un-permute
+    result = {
+        "metric": "MoE layer training step (forward saving g|u + backward) tokens/s at 1 B200",
+        "value": round(world * w.T / (step_ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init weights)",
+        "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias,
+                   "mode": "train", "parallelism": "single GPU",
+                   "l2": f"weights {sum(t.numel() * 2 for t in (inp['gate_up'], inp['down'])) / 1e9:.2f} GB, "
+                         "larger than L2, no flush",
+                   "timing": "two CUDA graphs (forward, backward) replayed back to back, events between them"},
+        "forward_ms": round(f_ms, 4), "backward_ms": round(b_ms, 4),
+        "roofline": {"kernel": "backward pass (4 grouped GEMMs + 5 CUDA-core kernels)", "bound": "tensor",
+                     "achieved": round(bwd_tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(bwd_tflops / peak, 4), "traffic": None,
+                     "peak_source": f"{pk_kind} bf16_tflops_sustained",
+                     "flops": "2 x the forward's grouped-GEMM FLOPs: T(12kDF + 12DFs)"},
+        "gpu_launches": (n_fwd + n_bwd) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    del g_fwd, g_bwd
+
+
 def run_reference(args, w: mi.Workload, rank: int, world: int):
     if rank != 0:
         return
@@ -454,6 +535,8 @@ def main():
     ap.add_argument("--workload", default="mixtral", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--train", action="store_true",
+                    help="time a training step (forward saving g|u + backward) instead of the forward")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="expert weight format; fp8 (E4M3, per-row scales) runs the decode kernels, T <= 64")
     args = ap.parse_args()
@@ -474,7 +557,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=__import__("torch").device("cuda", local_rank))
     try:
-        run_ours(args, w, rank, world, local_rank)
+        if args.train:
+            run_train(args, w, rank, world, local_rank)
+        else:
+            run_ours(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()

