@@ -41,7 +41,10 @@ constexpr int kStageBytes = kStageA + kStageB;
 constexpr int kStages = 4;
 constexpr int kAccCols = kBN;
 constexpr int kBarBytes = 256;
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kBarBytes + 4 * (kMaxGroups + 1);
+constexpr int kStagePitch = 33;  // fp32 staging row pitch (conflict-free transposes)
+constexpr int kStageFloats = 32 * kStagePitch;  // one epilogue warp's 32 x 32 chunk
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kBarBytes + 4 * (kMaxGroups + 1) +
+                              4 * kStageFloats * sizeof(float);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 __host__ __device__ constexpr bool is_dw(int kind) { return kind == kBwdDwDown || kind == kBwdDwGateUp; }
@@ -128,6 +131,21 @@ __host__ __device__ constexpr uint32_t bwd_idesc() {
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __expf(-z)); }
 
+// A warp's 32 x 32 fp32 chunk (lane i holds row i's 32 columns in a[]) written to rows
+// out + r * ld, r < n_rows, columns [0, 32): staged through shared memory so that each store
+// instruction writes 128 contiguous bytes of one row (instead of 32 lanes x 16 bytes in 32 rows).
+__device__ __forceinline__ void store_chunk_rows(float* stg, const uint32_t (&a)[32], float* out, size_t ld,
+                                                 int n_rows) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) stg[lane * kStagePitch + j] = __uint_as_float(a[j]);
+  __syncwarp();
+#pragma unroll 4
+  for (int r = 0; r < 32; ++r)
+    if (r < n_rows) out[(size_t)r * ld + lane] = stg[r * kStagePitch + lane];
+  __syncwarp();
+}
+
 template <int KIND>
 __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -138,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   int* tile_start = reinterpret_cast<int*>(smem + kStages * kStageBytes + kBarBytes);
+  float* stage_f = reinterpret_cast<float*>(tile_start + kMaxGroups + 1);  // [4 warps][32][33]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.n_groups[0] + (p.n_sets > 1 ? p.n_groups[1] : 0);
@@ -291,9 +310,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
       const int s = ti.set;
       const int N = p.N_total[s];
       const int lrow = ti.m * kBM + q * 32 + lane;  // row of the tile in its group
+      float* stg = stage_f + (warp - 2) * kStageFloats;
+      const int wrow0 = ti.m * kBM + q * 32;  // this warp's first tile row
       if constexpr (is_dw(KIND)) {
-        const bool row_ok = lrow < p.M_total[s];
-        float* orow = p.out[s] + ((size_t)ti.g * p.M_total[s] + lrow) * N;
+        const int n_rows = min(32, p.M_total[s] - wrow0);
+        float* obase = p.out[s] + ((size_t)ti.g * p.M_total[s] + wrow0) * N;
 #pragma unroll 1
         for (int c0 = 0; c0 < kBN; c0 += 32) {
           const int col = ti.n * kBN + c0;
@@ -306,20 +327,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
 #pragma unroll
             for (int j = 0; j < 32; ++j) a[j] = 0u;  // an expert without rows: zero gradient
           }
-          if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(orow + col);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
-                                   __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
-          }
+          if (n_rows > 0) store_chunk_rows(stg, a, obase + col, N, n_rows);
         }
       } else {
         const bool row_ok = lrow < ti.rows;
         const size_t prow = (size_t)ti.prow0 + lrow;  // padded row (A, dGU, dX)
         const size_t urow = (size_t)ti.row0 + lrow;   // unpadded row (p, saved g/u, dp)
         if constexpr (KIND == kBwdDxGateUp) {
-          float* orow = p.out[s] + prow * N;
+          const int n_rows = min(32, ti.rows - wrow0);
+          float* obase = p.out[s] + ((size_t)ti.prow0 + wrow0) * N;
 #pragma unroll 1
           for (int c0 = 0; c0 < kBN; c0 += 32) {
             const int col = ti.n * kBN + c0;
@@ -327,13 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
             uint32_t a[32];
             tmem_ld_32x32b_x32(tacc + c0, a);
             tmem_ld_wait();
-            if (row_ok) {
-              float4* dst = reinterpret_cast<float4*>(orow + col);
-#pragma unroll
-              for (int v = 0; v < 8; ++v)
-                dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
-                                     __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
-            }
+            if (n_rows > 0) store_chunk_rows(stg, a, obase + col, N, n_rows);
           }
         } else {
           // kDxDown: SwiGLU backward.  N = F; saved g in columns [0, F), u in [F, 2F)
