@@ -41,11 +41,13 @@ constexpr int kStageBytes = kStageA + kStageB;
 constexpr int kStages = 4;
 constexpr int kAccCols = kBN;
 constexpr int kBarBytes = 256;
-constexpr int kStagePitch = 33;  // fp32 staging row pitch (conflict-free transposes)
+constexpr int kStagePitch = 36;  // fp32 staging row pitch: 16-byte rows, conflict-free float4 phases
 constexpr int kStageFloats = 32 * kStagePitch;  // one epilogue warp's 32 x 32 chunk
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kBarBytes + 4 * (kMaxGroups + 1) +
+constexpr int kTileTableBytes = (4 * (kMaxGroups + 1) + 127) / 128 * 128;  // keeps the staging 128-byte aligned
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kBarBytes + kTileTableBytes +
                               4 * kStageFloats * sizeof(float);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert((kStages * kStageBytes + kBarBytes + kTileTableBytes) % 128 == 0, "16-byte aligned staging");
 
 __host__ __device__ constexpr bool is_dw(int kind) { return kind == kBwdDwDown || kind == kBwdDwGateUp; }
 
@@ -132,17 +134,26 @@ __host__ __device__ constexpr uint32_t bwd_idesc() {
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __expf(-z)); }
 
 // A warp's 32 x 32 fp32 chunk (lane i holds row i's 32 columns in a[]) written to rows
-// out + r * ld, r < n_rows, columns [0, 32): staged through shared memory so that each store
-// instruction writes 128 contiguous bytes of one row (instead of 32 lanes x 16 bytes in 32 rows).
+// out + r * ld, r < n_rows, columns [0, 32).  Staged through shared memory: each lane stores its row
+// as 8 float4 (with a pitch of 36 floats every 8-lane phase covers the 32 banks once), then lane l
+// writes columns 4(l % 8).. of rows l / 8 + 4i: one instruction stores 4 rows x 128 contiguous
+// bytes, and the 8 loads of a chunk are independent.
 __device__ __forceinline__ void store_chunk_rows(float* stg, const uint32_t (&a)[32], float* out, size_t ld,
                                                  int n_rows) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) stg[lane * kStagePitch + j] = __uint_as_float(a[j]);
+  for (int v = 0; v < 8; ++v)
+    *reinterpret_cast<float4*>(stg + lane * kStagePitch + 4 * v) =
+        make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]), __uint_as_float(a[4 * v + 2]),
+                    __uint_as_float(a[4 * v + 3]));
   __syncwarp();
-#pragma unroll 4
-  for (int r = 0; r < 32; ++r)
-    if (r < n_rows) out[(size_t)r * ld + lane] = stg[r * kStagePitch + lane];
+  const int c4 = (lane & 7) * 4, r0 = lane >> 3;
+  float4 vals[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) vals[i] = *reinterpret_cast<const float4*>(stg + (r0 + 4 * i) * kStagePitch + c4);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (r0 + 4 * i < n_rows) *reinterpret_cast<float4*>(out + (size_t)(r0 + 4 * i) * ld + c4) = vals[i];
   __syncwarp();
 }
 
@@ -156,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   int* tile_start = reinterpret_cast<int*>(smem + kStages * kStageBytes + kBarBytes);
-  float* stage_f = reinterpret_cast<float*>(tile_start + kMaxGroups + 1);  // [4 warps][32][33]
+  float* stage_f = reinterpret_cast<float*>(smem + kStages * kStageBytes + kBarBytes + kTileTableBytes);  // [4][32][36]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.n_groups[0] + (p.n_sets > 1 ? p.n_groups[1] : 0);
