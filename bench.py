@@ -42,11 +42,11 @@ _CSRC = "sparse_mixture_experts_16_b200/csrc/"
 _TRAFFIC = {
     # weights -> (kernel sources, their sha256, {workload: dram__bytes_read.sum + dram__bytes_write.sum})
     "bf16": ((_CSRC + "grouped_gemm_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
-             "636f5c796994e65aec9db9f1c91d3bba777c9551af9d012877e3d0879989a768",
-             {"mixtral": 1.946486e9 + 0.226486e9, "deepseek_decode": 5.876486e9 + 0.004078e9}),
+             "524599bd67b9b6b8deba6af1a7841ddec43f7e8250f30be76b353018d5a9bdf3",
+             {"mixtral": 1.947595e9 + 0.226813e9, "deepseek_decode": 5.876610e9 + 0.003743e9}),
     "fp8": ((_CSRC + "stream_fp8w_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
-            "d33af253c883b52c16557b50c8d3516c8200992db331ccc8d752899fff96ff3f",
-            {"deepseek_decode": 2.942076e9 + 0.005430e9, "gptoss_decode_T64": 0.556636e9 + 0.005026e9}),
+            "90184c605698454c7e2560af3fdb691544ae668cddf7910ea71752c9dc8e3252",
+            {"deepseek_decode": 2.942079e9 + 0.003725e9, "gptoss_decode_T64": 0.556999e9 + 0.004705e9}),
 }
 
 

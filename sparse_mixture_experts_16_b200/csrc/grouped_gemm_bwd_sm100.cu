@@ -138,19 +138,29 @@ __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __ex
 // as 8 float4 (with a pitch of 36 floats every 8-lane phase covers the 32 banks once), then lane l
 // writes columns 4(l % 8).. of rows l / 8 + 4i: one instruction stores 4 rows x 128 contiguous
 // bytes, and the 8 loads of a chunk are independent.
+__device__ __forceinline__ void st_shared_f4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void store_chunk_rows(float* stg, const uint32_t (&a)[32], float* out, size_t ld,
                                                  int n_rows) {
   const int lane = threadIdx.x & 31;
+  const uint32_t base = smem_u32(stg);
 #pragma unroll
   for (int v = 0; v < 8; ++v)
-    *reinterpret_cast<float4*>(stg + lane * kStagePitch + 4 * v) =
-        make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]), __uint_as_float(a[4 * v + 2]),
-                    __uint_as_float(a[4 * v + 3]));
+    st_shared_f4(base + (uint32_t)(lane * kStagePitch + 4 * v) * 4u, __uint_as_float(a[4 * v]),
+                 __uint_as_float(a[4 * v + 1]), __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
   __syncwarp();
   const int c4 = (lane & 7) * 4, r0 = lane >> 3;
   float4 vals[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) vals[i] = *reinterpret_cast<const float4*>(stg + (r0 + 4 * i) * kStagePitch + c4);
+  for (int i = 0; i < 8; ++i) vals[i] = ld_shared_f4(base + (uint32_t)((r0 + 4 * i) * kStagePitch + c4) * 4u);
 #pragma unroll
   for (int i = 0; i < 8; ++i)
     if (r0 + 4 * i < n_rows) *reinterpret_cast<float4*>(out + (size_t)(r0 + 4 * i) * ld + c4) = vals[i];
