@@ -41,19 +41,19 @@ constexpr int kStageBytes = kStageA + kStageB;
 constexpr int kStages = 4;
 constexpr int kAccCols = kBN;
 constexpr int kBarBytes = 256;
-constexpr int kStagePitch = 36;  // fp32 staging row pitch: 16-byte rows, conflict-free float4 phases
-constexpr int kStageFloats = 32 * kStagePitch;  // one epilogue warp's 32 x 32 chunk
+constexpr int kStageBytesOut = 32 * 128;  // one epilogue warp's 32 x 32 fp32 chunk, 128-byte swizzled rows
 constexpr int kTileTableBytes = (4 * (kMaxGroups + 1) + 127) / 128 * 128;  // keeps the staging 128-byte aligned
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kBarBytes + kTileTableBytes +
-                              4 * kStageFloats * sizeof(float);
+constexpr int kStageOffset = (kStages * kStageBytes + kBarBytes + kTileTableBytes + 1023) / 1024 * 1024;
+constexpr size_t kSmemBytes = 1024 + (size_t)kStageOffset + 4 * kStageBytesOut;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert((kStages * kStageBytes + kBarBytes + kTileTableBytes) % 128 == 0, "16-byte aligned staging");
+static_assert(kStageOffset % 1024 == 0, "swizzle-atom aligned output staging");
 
 __host__ __device__ constexpr bool is_dw(int kind) { return kind == kBwdDwDown || kind == kBwdDwGateUp; }
 
 struct alignas(64) BwdParams {
   CUtensorMap a_map[2];  // dx kinds: K-major A [rows, K], box {64, 128}; dw kinds: MN-major [rows, M], box {64, 64}
   CUtensorMap b_map[2];  // MN-major B [K rows, N cols], box {64, 64}
+  CUtensorMap o_map[2];  // fp32 outputs (dX, weight gradients) [rows, N], box {32, 32}, 128-byte swizzle
   const int32_t* offsets[2];      // per group: rows [offsets[g], offsets[g+1]) of the unpadded layout
   const int32_t* pad_offsets[2];  // the same groups in the 64-row padded layout (NULL: = offsets)
   int n_groups[2];
@@ -141,30 +141,39 @@ __device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + __ex
 __device__ __forceinline__ void st_shared_f4(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
-__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
-               : "memory");
-  return v;
-}
 
-__device__ __forceinline__ void store_chunk_rows(float* stg, const uint32_t (&a)[32], float* out, size_t ld,
-                                                 int n_rows) {
+// TMA bulk store of a box from shared memory (tracked in this thread's bulk group)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// A warp's 32 x 32 fp32 chunk (lane i holds row i's 32 columns in a[]) written to the output
+// tensor at (col x, row y) by one TMA bulk store.  The rows are staged with the 128-byte swizzle
+// the output map uses (16-byte chunk j of row r at position j ^ (r & 7)): every 8-lane phase of the
+// staging stores covers the 32 banks once.  Rows and columns past the tensor's extent are clipped
+// by TMA; callers never pass a box that reaches into another group's rows.
+__device__ __forceinline__ void store_chunk_tma(uint8_t* stg, const uint32_t (&a)[32], const CUtensorMap* map,
+                                                int x, int y) {
   const int lane = threadIdx.x & 31;
-  const uint32_t base = smem_u32(stg);
+  if (lane == 0) bulk_wait_read_all();  // the previous chunk's store has read the staging buffer
+  __syncwarp();
+  const uint32_t row = smem_u32(stg) + lane * 128;
 #pragma unroll
   for (int v = 0; v < 8; ++v)
-    st_shared_f4(base + (uint32_t)(lane * kStagePitch + 4 * v) * 4u, __uint_as_float(a[4 * v]),
-                 __uint_as_float(a[4 * v + 1]), __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
+    st_shared_f4(row + ((v ^ (lane & 7)) << 4), __uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
+                 __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic stores -> the TMA's reads
   __syncwarp();
-  const int c4 = (lane & 7) * 4, r0 = lane >> 3;
-  float4 vals[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) vals[i] = ld_shared_f4(base + (uint32_t)((r0 + 4 * i) * kStagePitch + c4) * 4u);
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (r0 + 4 * i < n_rows) *reinterpret_cast<float4*>(out + (size_t)(r0 + 4 * i) * ld + c4) = vals[i];
-  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, smem_u32(stg), x, y);
+    bulk_commit();
+  }
 }
 
 template <int KIND>
@@ -177,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   int* tile_start = reinterpret_cast<int*>(smem + kStages * kStageBytes + kBarBytes);
-  float* stage_f = reinterpret_cast<float*>(smem + kStages * kStageBytes + kBarBytes + kTileTableBytes);  // [4][32][36]
+  uint8_t* stage_o = smem + kStageOffset;  // [4 epilogue warps][32 rows][128 B], 128-byte swizzle
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.n_groups[0] + (p.n_sets > 1 ? p.n_groups[1] : 0);
@@ -331,11 +340,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
       const int s = ti.set;
       const int N = p.N_total[s];
       const int lrow = ti.m * kBM + q * 32 + lane;  // row of the tile in its group
-      float* stg = stage_f + (warp - 2) * kStageFloats;
+      uint8_t* stg = stage_o + (warp - 2) * kStageBytesOut;
       const int wrow0 = ti.m * kBM + q * 32;  // this warp's first tile row
       if constexpr (is_dw(KIND)) {
-        const int n_rows = min(32, p.M_total[s] - wrow0);
-        float* obase = p.out[s] + ((size_t)ti.g * p.M_total[s] + wrow0) * N;
+        const int n_rows = min(32, p.M_total[s] - wrow0);  // 32 or <= 0: M_total is a multiple of 64
+        const int orow = ti.g * p.M_total[s] + wrow0;
 #pragma unroll 1
         for (int c0 = 0; c0 < kBN; c0 += 32) {
           const int col = ti.n * kBN + c0;
@@ -348,15 +357,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
 #pragma unroll
             for (int j = 0; j < 32; ++j) a[j] = 0u;  // an expert without rows: zero gradient
           }
-          if (n_rows > 0) store_chunk_rows(stg, a, obase + col, N, n_rows);
+          if (n_rows > 0) store_chunk_tma(stg, a, &p.o_map[s], col, orow);
         }
       } else {
         const bool row_ok = lrow < ti.rows;
         const size_t prow = (size_t)ti.prow0 + lrow;  // padded row (A, dGU, dX)
         const size_t urow = (size_t)ti.row0 + lrow;   // unpadded row (p, saved g/u, dp)
         if constexpr (KIND == kBwdDxGateUp) {
+          // 32-row boxes stay inside the group's 64-row padded span (or the shared set's T rows, where
+          // TMA clips): wrow0 < rows, both wrow0 and the span are multiples of 32
           const int n_rows = min(32, ti.rows - wrow0);
-          float* obase = p.out[s] + ((size_t)ti.prow0 + wrow0) * N;
+          const int orow = ti.prow0 + wrow0;
 #pragma unroll 1
           for (int c0 = 0; c0 < kBN; c0 += 32) {
             const int col = ti.n * kBN + c0;
@@ -364,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
             uint32_t a[32];
             tmem_ld_32x32b_x32(tacc + c0, a);
             tmem_ld_wait();
-            if (n_rows > 0) store_chunk_rows(stg, a, obase + col, N, n_rows);
+            if (n_rows > 0) store_chunk_tma(stg, a, &p.o_map[s], col, orow);
           }
         } else {
           // kDxDown: SwiGLU backward.  N = F; saved g in columns [0, F), u in [F, 2F)
@@ -420,6 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
+    if (lane == 0) bulk_wait_all();  // every output store issued by this warp has been performed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -461,6 +474,19 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 row-major [rows, cols] output map for TMA stores: box 32 x 32, 128-byte swizzle
+bool make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -483,6 +509,12 @@ cudaError_t launch(const BwdSetHost* sets, int n_sets, int* err, cudaStream_t s)
     if (!make_map(&p.a_map[i], st.a, (uint64_t)st.a_rows, (uint64_t)st.a_cols, is_dw(KIND) ? 64 : 128))
       return cudaErrorInvalidValue;
     if (!make_map(&p.b_map[i], st.b, (uint64_t)st.b_rows, (uint64_t)st.b_cols, 64)) return cudaErrorInvalidValue;
+    if (is_dw(KIND) || KIND == kBwdDxGateUp) {
+      // weight gradients: [groups * M_total, N]; dX: [a_rows (padded rows, or T), N]
+      const uint64_t orows = is_dw(KIND) ? (uint64_t)st.n_groups * st.M_total : (uint64_t)st.a_rows;
+      if (st.out == nullptr || !make_out_map(&p.o_map[i], st.out, orows, (uint64_t)st.N_total))
+        return cudaErrorInvalidValue;
+    }
     p.offsets[i] = st.offsets;
     p.pad_offsets[i] = st.pad_offsets;
     p.n_groups[i] = st.n_groups;
