@@ -40,10 +40,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # valid only while that kernel's sources are unchanged, else reported as null.
 _CSRC = "sparse_mixture_experts_16_b200/csrc/"
 _TRAFFIC = {
-    # weights -> (kernel sources, their sha256, {workload: dram__bytes_read.sum + dram__bytes_write.sum})
+    # kernel variant -> (its sources, their sha256, {workload: dram__bytes_read.sum + dram__bytes_write.sum})
     "bf16": ((_CSRC + "grouped_gemm_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
              "524599bd67b9b6b8deba6af1a7841ddec43f7e8250f30be76b353018d5a9bdf3",
              {"mixtral": 1.947595e9 + 0.226813e9, "deepseek_decode": 5.876610e9 + 0.003743e9}),
+    "bf16_wide": ((_CSRC + "grouped_gemm_wide_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
+                  "", {}),
     "fp8": ((_CSRC + "stream_fp8w_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
             "90184c605698454c7e2560af3fdb691544ae668cddf7910ea71752c9dc8e3252",
             {"deepseek_decode": 2.942079e9 + 0.003725e9, "gptoss_decode_T64": 0.556999e9 + 0.004705e9}),
@@ -232,6 +234,12 @@ def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, max_experts: int = 4
 
 
 # ---------------------------------------------------------------------------------- GPU arm
+def tiling_flag(tiling: str) -> int:
+    import sparse_mixture_experts_16_b200 as moe
+
+    return {"auto": 0, "row": moe.MOE_FLAG_PREFILL_ROW_TILES, "wide": moe.MOE_FLAG_PREFILL_WIDE_TILES}[tiling]
+
+
 def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     import ctypes
 
@@ -257,7 +265,8 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         else:
             scales = None
         layer = moe.MoELayer(inp["wg"], inp["gate_up"], inp["down"], w.k, bias=inp["bias"],
-                             shared_gate_up=inp["shared_gate_up"], shared_down=inp["shared_down"], scales=scales)
+                             shared_gate_up=inp["shared_gate_up"], shared_down=inp["shared_down"], scales=scales,
+                             flags=0 if scales is not None else tiling_flag(args.tiling))
         x = inp["x"]
         y = torch.empty_like(x)
         ws = layer.workspace(w.T)
@@ -377,8 +386,10 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     else:
         achieved = gateup_flops(w) / (gate_ms / 1e3) / 1e12
         peak = pk["bf16_tflops_sustained"]
-        roof = {"kernel": "grouped_gemm_kernel<gate_up, tiled>", "bound": "tensor", "achieved": round(achieved, 1),
-                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name),
+        wide = layer.gemm_path(w.T) == "wide_tiles"
+        roof = {"kernel": "grouped_gemm_wide_kernel<gate_up>" if wide else "grouped_gemm_kernel<gate_up, tiled>",
+                "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name, "bf16_wide" if wide else "bf16"),
                 "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
                 "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4)}
     layer_tflops = w.flops / (ms_per_step / 1e3) / 1e12 * world
@@ -393,6 +404,7 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias,
                    "weights": ("E4M3 codes + per-row fp32 scales (f16 MMA, fp32 accumulation)"
                                if args.weights == "fp8" else "bf16"),
+                   "gemm_path": layer.gemm_path(w.T),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": ("L2 flushed (256 MB write) before every timed step" if flush is not None
                           else f"inputs larger than L2 (weights {weight_bytes / 1e9:.2f} GB), no flush"),
@@ -436,7 +448,7 @@ def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         inp = mi.device_inputs(w, device=dev)
         layer = moe.MoELayer(inp["wg"], inp["gate_up"], inp["down"], w.k, bias=inp["bias"],
                              shared_gate_up=inp["shared_gate_up"], shared_down=inp["shared_down"],
-                             flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD)
+                             flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD | tiling_flag(args.tiling))
         x = inp["x"]
         y = torch.empty_like(x)
         dy = torch.empty_like(x)
@@ -484,7 +496,7 @@ def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         "warmup": max(args.warmup, 3), "ms_per_step": round(step_ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; random-init weights)",
         "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias,
-                   "mode": "train", "parallelism": "single GPU",
+                   "mode": "train", "gemm_path": layer.gemm_path(w.T), "parallelism": "single GPU",
                    "l2": f"weights {sum(t.numel() * 2 for t in (inp['gate_up'], inp['down'])) / 1e9:.2f} GB, "
                          "larger than L2, no flush",
                    "timing": "two CUDA graphs (forward, backward) replayed back to back, events between them"},
@@ -537,6 +549,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--train", action="store_true",
                     help="time a training step (forward saving g|u + backward) instead of the forward")
+    ap.add_argument("--tiling", default="auto", choices=["auto", "row", "wide"],
+                    help="prefill tiling of the expert GEMMs (bf16): the layer's default rule, 128-row tiles, "
+                         "or token-wide tiles")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="expert weight format; fp8 (E4M3, per-row scales) runs the decode kernels, T <= 64")
     args = ap.parse_args()

@@ -170,6 +170,14 @@ moe_status_t moe_combine(const float* out_perm, const int32_t* inv_perm, const f
  * and the SwiGLU inputs g | u of the gate_up GEMMs, bf16).  Uses the tiled kernels at any T;
  * bf16 weights only. */
 #define MOE_FLAG_SAVE_FOR_BACKWARD 4
+/* Prefill tiling of the expert GEMMs (at most one of the two; neither with FORCE_DECODE):
+ *  ROW_TILES  128 permuted rows x 256 output columns per tile (tokens are the MMA's M);
+ *  WIDE_TILES 128 weight rows x up to 256 rows of one expert segment (tokens are N, so a
+ *             segment's last tile is padded to a multiple of 16 rows instead of 128).
+ * Without either, ROW_TILES.  Both give the same routing; outputs agree within fp32 rounding
+ * order. */
+#define MOE_FLAG_PREFILL_ROW_TILES 8
+#define MOE_FLAG_PREFILL_WIDE_TILES 16
 
 #define MOE_WEIGHTS_BF16 0     /* gate_up / down (and shared_*) hold bf16 weights            */
 #define MOE_WEIGHTS_FP8_E4M3 1 /* *_fp8 hold E4M3 codes with one fp32 scale per weight row  */
@@ -235,6 +243,15 @@ moe_status_t moe_layer_forward_timed(const moe_layer_desc_t* desc, const moe_bf1
 
 /* Number of kernels one moe_layer_forward launches for this descriptor (0 if invalid). */
 int moe_layer_kernel_count(const moe_layer_desc_t* desc);
+
+/* Which expert-GEMM kernels moe_layer_forward runs for this descriptor (host-only query; -1 if
+ * the descriptor is invalid): the weight-streaming decode kernels (bf16 or E4M3 weights), or the
+ * prefill tilings of MOE_FLAG_PREFILL_ROW_TILES / MOE_FLAG_PREFILL_WIDE_TILES. */
+#define MOE_PATH_STREAMING 0
+#define MOE_PATH_FP8_STREAMING 1
+#define MOE_PATH_ROW_TILES 2
+#define MOE_PATH_WIDE_TILES 3
+int moe_layer_gemm_path(const moe_layer_desc_t* desc);
 
 /* ----------------------------------------------------------------------------------------
  * Backward pass (training; keryc.com "Mixture of Experts optimiza...", section "Entrenamiento:

@@ -18,6 +18,9 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_FLAG_FORCE_PREFILL = 1
 MOE_FLAG_FORCE_DECODE = 2
 MOE_FLAG_SAVE_FOR_BACKWARD = 4
+MOE_FLAG_PREFILL_ROW_TILES = 8
+MOE_FLAG_PREFILL_WIDE_TILES = 16
+MOE_PATH_STREAMING, MOE_PATH_FP8_STREAMING, MOE_PATH_ROW_TILES, MOE_PATH_WIDE_TILES = 0, 1, 2, 3
 MOE_WEIGHTS_BF16 = 0
 MOE_WEIGHTS_FP8_E4M3 = 1
 
@@ -32,7 +35,7 @@ EXPORTS = (
     "moe_quantize_rows_fp8", "moe_router_topk_workspace_size", "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
     "moe_grouped_swiglu_ffn_workspace_size",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_layer_workspace_size", "moe_layer_forward",
-    "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_update_router_bias",
+    "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_layer_gemm_path", "moe_update_router_bias",
     "moe_layer_expert_counts", "moe_get_device_error", "moe_layer_backward_workspace_size", "moe_layer_backward",
     "moe_status_string",
 )
@@ -90,6 +93,7 @@ def lib():
             "moe_layer_forward_host": ([ctypes.POINTER(LayerDesc), P, P, P, Z, P], I),
             "moe_layer_forward_timed": ([ctypes.POINTER(LayerDesc), P, P, P, Z, P, ctypes.POINTER(P), I], I),
             "moe_layer_kernel_count": ([ctypes.POINTER(LayerDesc)], I),
+            "moe_layer_gemm_path": ([ctypes.POINTER(LayerDesc)], I),
             "moe_update_router_bias": ([P, I, ctypes.c_float, P, P], I),
             "moe_layer_expert_counts": ([ctypes.POINTER(LayerDesc), P, Z, ctypes.POINTER(P)], I),
             "moe_get_device_error": ([P, P], I),
@@ -301,6 +305,15 @@ class MoELayer:
     def kernel_count(self, T: int) -> int:
         d = self.desc(T)
         return lib().moe_layer_kernel_count(ctypes.byref(d))
+
+    def gemm_path(self, T: int) -> str:
+        """The expert-GEMM kernels a forward over T tokens runs: "streaming", "fp8_streaming",
+        "row_tiles" or "wide_tiles"."""
+        d = self.desc(T)
+        code = lib().moe_layer_gemm_path(ctypes.byref(d))
+        if code < 0:
+            raise MoeError(1, "moe_layer_gemm_path")
+        return ("streaming", "fp8_streaming", "row_tiles", "wide_tiles")[code]
 
     def forward(self, x, y=None, stream=None):
         import torch

@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstring>
 
+#include "grouped_gemm_wide.cuh"
 #include "moe_common.cuh"
 
 using namespace moe;
@@ -46,6 +47,12 @@ bool use_decode(const moe_layer_desc_t& d) {
 }
 
 int decode_tile(int max_seg) { return ((max_seg + 15) / 16) * 16; }
+
+// Prefill tiling: token-wide tiles (weights as the MMA's M, up to 256 rows of one segment as N)
+// pad each segment's last tile to 16 rows instead of 128 and need fewer MMA cycles, but measured
+// slower on every prefill shape here (their gate_up reaches lower tensor-pipe activity), so the
+// 128-row tiles are the default and the token-wide ones run only when asked for.
+bool wide_tiles(int flags) { return (flags & MOE_FLAG_PREFILL_WIDE_TILES) != 0; }
 
 struct LayerWs {
   size_t split_counters, split_partial, split_partial_bytes, gu_saved, gu_saved_sh, router, topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
@@ -122,8 +129,12 @@ moe_status_t validate_desc(const moe_layer_desc_t* d) {
   } else {
     return MOE_ERR_INVALID_ARG;
   }
-  if ((d->flags & ~(MOE_FLAG_FORCE_PREFILL | MOE_FLAG_FORCE_DECODE | MOE_FLAG_SAVE_FOR_BACKWARD)) != 0)
+  if ((d->flags & ~(MOE_FLAG_FORCE_PREFILL | MOE_FLAG_FORCE_DECODE | MOE_FLAG_SAVE_FOR_BACKWARD |
+                    MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES)) != 0)
     return MOE_ERR_INVALID_ARG;
+  const int tiling = d->flags & (MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES);
+  if (tiling == (MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES)) return MOE_ERR_INVALID_ARG;
+  if (tiling && ((d->flags & MOE_FLAG_FORCE_DECODE) || d->weight_format != MOE_WEIGHTS_BF16)) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && (d->flags & MOE_FLAG_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_FORCE_PREFILL) && (d->flags & MOE_FLAG_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_FORCE_DECODE) && d->T > kDecodeTMax) return MOE_ERR_INVALID_ARG;
@@ -146,7 +157,7 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
                      int F, const uint16_t* gate_up, const uint16_t* down, uint16_t* h, float* out_perm,
                      // optional shared expert over x[T, D]
                      const uint16_t* x, int T, int Fs, const uint16_t* sgu, const uint16_t* sdn, uint16_t* h_sh,
-                     float* out_sh, int decode_nt, int* err, cudaStream_t s, cudaEvent_t ev_mid,
+                     float* out_sh, int decode_nt, bool wide, int* err, cudaStream_t s, cudaEvent_t ev_mid,
                      unsigned ev_flags, uint16_t* save_gu = nullptr, uint16_t* save_gu_sh = nullptr) {
   GemmSetHost g[2];
   memset(g, 0, sizeof(g));
@@ -158,7 +169,10 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
     g[1].n_out = Fs, g[1].out = h_sh, g[1].save_gu = save_gu_sh;
     n_sets = 2;
   }
-  MOE_CUDA_TRY(launch_grouped_gemm(kGateUp, g, n_sets, decode_nt, err, s));
+  if (decode_nt == 0 && wide)
+    MOE_CUDA_TRY(launch_grouped_gemm_wide(kGateUp, g, n_sets, err, s));
+  else
+    MOE_CUDA_TRY(launch_grouped_gemm(kGateUp, g, n_sets, decode_nt, err, s));
   if (ev_mid) MOE_CUDA_TRY(cudaEventRecordWithFlags(ev_mid, s, ev_flags));
   GemmSetHost dn[2];
   memset(dn, 0, sizeof(dn));
@@ -168,7 +182,10 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
     dn[1].K = Fs, dn[1].a = h_sh, dn[1].a_rows = T, dn[1].w = sdn, dn[1].n_groups = 1, dn[1].m_rows = T;
     dn[1].n_out = D, dn[1].out = out_sh;
   }
-  MOE_CUDA_TRY(launch_grouped_gemm(kDown, dn, n_sets, decode_nt, err, s));
+  if (decode_nt == 0 && wide)
+    MOE_CUDA_TRY(launch_grouped_gemm_wide(kDown, dn, n_sets, err, s));
+  else
+    MOE_CUDA_TRY(launch_grouped_gemm(kDown, dn, n_sets, decode_nt, err, s));
   return MOE_OK;
 }
 
@@ -247,7 +264,8 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
     MOE_CUDA_TRY(launch_stream_fp8w(kDown, dn, ds, Fs > 0 ? 2 : 1, nt, split, err, s));
   } else {
   st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), Fp(w.out_perm), x,
-               T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, err, s, ev ? ev[3] : nullptr,
+               T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, wide_tiles(d->flags), err,
+               s, ev ? ev[3] : nullptr,
                rec_flags, (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) ? H(w.gu_saved) : nullptr,
                (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && Fs > 0 ? H(w.gu_saved_sh) : nullptr);
   if (st != MOE_OK) return st;
@@ -402,7 +420,8 @@ moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* off
   uint8_t* b = static_cast<uint8_t*>(ws);
   const int nt = max_seg <= kDecodeTMax ? decode_tile(max_seg < 1 ? 1 : max_seg) : 0;
   return run_ffn(x_perm, offsets, row_scale, M, E, D, F, gate_up, down, reinterpret_cast<uint16_t*>(b + kWsHeader),
-                 out_perm, nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr, nt, reinterpret_cast<int*>(b),
+                 out_perm, nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr, nt, wide_tiles(0),
+                 reinterpret_cast<int*>(b),
                  (cudaStream_t)stream, nullptr, cudaEventRecordDefault);
 }
 
@@ -465,6 +484,13 @@ int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   // above: hist, scan, scatter, gather
   const int dispatch = desc->T <= 256 ? 1 : 4;
   return 2 /*router GEMM, top-k*/ + dispatch + 2 /*grouped GEMMs*/ + 1 /*combine*/;
+}
+
+int moe_layer_gemm_path(const moe_layer_desc_t* desc) {
+  if (validate_desc(desc) != MOE_OK) return -1;
+  if (desc->weight_format == MOE_WEIGHTS_FP8_E4M3) return MOE_PATH_FP8_STREAMING;
+  if (use_decode(*desc)) return MOE_PATH_STREAMING;
+  return wide_tiles(desc->flags) ? MOE_PATH_WIDE_TILES : MOE_PATH_ROW_TILES;
 }
 
 moe_status_t moe_update_router_bias(const int32_t* counts, int E, float gamma, float* bias, moe_stream_t stream) {

@@ -67,6 +67,9 @@ def _desc(**kw):
     (dict(w_gate=0x1008), 3),     # misaligned
     (dict(flags=3), 1),           # both force flags
     (dict(flags=2, T=65), 1),     # decode forced above the decode range
+    (dict(flags=8 | 16), 1),      # both prefill tilings
+    (dict(flags=2 | 16), 1),      # a prefill tiling with decode forced
+    (dict(flags=32), 1),          # unknown flag
 ])
 def test_layer_forward_rejects_bad_descriptors(L, kw, status):
     d = _desc(**kw)
@@ -217,3 +220,24 @@ def test_backward_entry_validates_on_host(L):
     # FP8 weights cannot be trained here; decode forcing conflicts with saving
     assert L.moe_layer_workspace_size(ctypes.byref(_desc(**FP8, flags=SAVE))) == 0
     assert L.moe_layer_workspace_size(ctypes.byref(_desc(flags=SAVE | moe.MOE_FLAG_FORCE_DECODE))) == 0
+
+
+def test_gemm_path_query(L):
+    """The host-only path query follows the flags and the default rule: T <= 64 streams the weights,
+    larger T runs the 128-row tiles unless the token-wide tiles are asked for; E4M3 weights always
+    stream."""
+    P = lambda **kw: L.moe_layer_gemm_path(ctypes.byref(_desc(**kw)))
+    assert P() == moe.MOE_PATH_STREAMING                                     # T = 16
+    assert P(T=16, flags=moe.MOE_FLAG_FORCE_PREFILL) == moe.MOE_PATH_ROW_TILES
+    assert P(T=16, flags=moe.MOE_FLAG_FORCE_PREFILL | moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_WIDE_TILES
+    assert P(T=65) == moe.MOE_PATH_ROW_TILES
+    assert P(T=4096, E=8, k=2) == moe.MOE_PATH_ROW_TILES
+    assert P(T=4096, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_WIDE_TILES
+    assert P(T=16, flags=moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_STREAMING  # tiling flags leave decode
+    assert P(T=300, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_ROW_TILES) == moe.MOE_PATH_ROW_TILES
+    assert P(**FP8) == moe.MOE_PATH_FP8_STREAMING
+    assert P(**FP8, flags=moe.MOE_FLAG_PREFILL_WIDE_TILES) == -1             # E4M3 has no prefill path
+    assert P(k=9) == -1
+    # the training forward runs a prefill tiling at any T
+    assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD) == moe.MOE_PATH_ROW_TILES
+    assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD | moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_WIDE_TILES

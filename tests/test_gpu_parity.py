@@ -332,18 +332,25 @@ FULL = ["mixtral", "gptoss", "gptoss_decode_T1", "gptoss_decode_T8", "gptoss_dec
 SAMPLE = {"mixtral": 6, "gptoss": 8, "deepseek": 4, "deepseek_decode": 4}
 
 
+# the token-wide prefill tiling (the default is the 128-row tiling), at full size
+OTHER_TILING = [("mixtral", moe.MOE_FLAG_PREFILL_WIDE_TILES), ("gptoss", moe.MOE_FLAG_PREFILL_WIDE_TILES),
+                ("deepseek", moe.MOE_FLAG_PREFILL_WIDE_TILES)]
+
+
 @pytest.mark.slow
-@pytest.mark.parametrize("name", FULL)
-def test_full_size_workload_parity(name):
-    """Routing of every token bit-exact; layer outputs of sampled tokens within tolerance; the
-    layer is launched exactly as the benchmark launches it."""
+@pytest.mark.parametrize("name,flags", [(n, 0) for n in FULL] + OTHER_TILING,
+                         ids=[n for n in FULL] + [f"{n}-{'wide' if f == moe.MOE_FLAG_PREFILL_WIDE_TILES else 'row'}"
+                                                  for n, f in OTHER_TILING])
+def test_full_size_workload_parity(name, flags):
+    """Routing of every token bit-exact; layer outputs of sampled tokens within tolerance; with
+    flags = 0 the layer is launched exactly as the benchmark launches it."""
     import torch
 
     w = mi.WORKLOADS[name]
     rd = gap_redraw(w)
     d = mi.device_inputs(w, redraw=rd)
     L = moe.MoELayer(d["wg"], d["gate_up"], d["down"], w.k, bias=d["bias"], shared_gate_up=d["shared_gate_up"],
-                     shared_down=d["shared_down"])
+                     shared_down=d["shared_down"], flags=flags)
     y = L(d["x"])
     idx, _ = moe.moe_router_topk(d["x"], d["wg"], d["bias"], w.k)
     torch.cuda.synchronize()

@@ -1,0 +1,132 @@
+"""Both prefill tilings of the expert GEMMs against the fp64 oracle: 128-row tiles (permuted rows
+as the MMA's M) and token-wide tiles (128 weight rows as M, up to 256 rows of one expert segment
+as N).  Cases cover segments of one ragged token tile, of several token tiles, empty segments, a
+one-row segment, output columns that end mid-tile (D = 192: 1.5 column tiles of the down GEMM)
+and the shared expert; routing is bit-exact and the layer output within 2e-2 x RMS(y_oracle)."""
+import numpy as np
+import pytest
+
+import moe_inputs as mi
+import oracle
+import sparse_mixture_experts_16_b200 as moe
+from helpers import (REL_RMS_TOL, bf16_np_to_f64, gap_redraw, gap_violations, rel_rms_err, scores, to_np_bf16,
+                     to_torch_bf16)
+
+pytestmark = pytest.mark.gpu
+
+ROW, WIDE = moe.MOE_FLAG_PREFILL_ROW_TILES, moe.MOE_FLAG_PREFILL_WIDE_TILES
+PREFILL = moe.MOE_FLAG_FORCE_PREFILL
+
+
+def W(T, D, E, k, F, Fs=0, bias="none"):
+    return mi.Workload(f"wide_T{T}D{D}E{E}k{k}F{F}Fs{Fs}", T=T, D=D, E=E, k=k, F=F, Fs=Fs, bias=bias)
+
+
+def _case(w):
+    import torch
+
+    rd = gap_redraw(w)
+    h = mi.host_inputs(w, redraw=rd)
+    d = {n: None if a is None else (to_torch_bf16(a) if a.dtype == np.uint16 else torch.from_numpy(a).cuda())
+         for n, a in h.items()}
+    return h, d
+
+
+def _layer(d, k, flags):
+    return moe.MoELayer(d["wg"], d["gate_up"], d["down"], k, bias=d["bias"], shared_gate_up=d["shared_gate_up"],
+                        shared_down=d["shared_down"], flags=flags)
+
+
+def _oracle(h, k):
+    return oracle.layer(h["x"], h["wg"], h["bias"], h["gate_up"], h["down"], k, h["shared_gate_up"],
+                        h["shared_down"])[0]
+
+
+CASES = [
+    W(600, 256, 8, 2, 320),                               # ~150-row segments: one ragged token tile each
+    W(700, 192, 4, 2, 256, Fs=128, bias="zipf:1.1"),      # up to 3 token tiles; D = 1.5 down column tiles
+    W(300, 128, 64, 2, 128),                              # short and empty segments
+    W(520, 320, 2, 2, 192, Fs=64),                        # two long segments, shared expert of 3 token tiles
+    W(129, 128, 1, 1, 128),                               # one segment of 129 rows: N = 144
+]
+
+
+@pytest.mark.parametrize("tiling", [ROW, WIDE], ids=["row_tiles", "wide_tiles"])
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_layer_parity_both_tilings(cuda_device, w, tiling):
+    h, d = _case(w)
+    L = _layer(d, w.k, tiling | PREFILL)
+    assert L.gemm_path(w.T) == ("row_tiles" if tiling == ROW else "wide_tiles")
+    y = bf16_np_to_f64(to_np_bf16(L(d["x"])))
+    assert L.device_error() == 0
+    assert rel_rms_err(y, _oracle(h, w.k)) <= REL_RMS_TOL
+
+
+def test_wide_tiles_single_row_segments(cuda_device):
+    """One token, top-2 of 4: two segments of one row each (MMA N = 16, one 64-row token box)."""
+    w = W(1, 128, 4, 2, 64)
+    h, d = _case(w)
+    y = bf16_np_to_f64(to_np_bf16(_layer(d, w.k, WIDE | PREFILL)(d["x"])))
+    assert rel_rms_err(y, _oracle(h, w.k)) <= REL_RMS_TOL
+
+
+def test_wide_tiles_one_overloaded_expert(cuda_device):
+    """A large bias sends every token's first choice to expert 3: one segment of 600 rows (3 token
+    tiles, the last of 88 rows) and 63 short or empty ones.  On this input exact bf16 arithmetic
+    (h and y rounded to bf16, fp32 sums; emulated on the CPU) is already 2.22e-2 x RMS(y) off on
+    one token, so the bound here is normwise, like the backward tests': RMS(err) <= 5e-3 x RMS(y)
+    and max|err| <= 2e-2 x max|y|."""
+    w = W(600, 256, 64, 2, 192)
+    h, d = _case(w)
+    h["bias"] = np.zeros(64, np.float32)
+    h["bias"][3] = 1000.0
+    import torch
+
+    d["bias"] = torch.from_numpy(h["bias"]).cuda()
+    idx_ref = oracle.router(h["x"], h["wg"], h["bias"], w.k)[0]
+    assert (idx_ref[:, 0] == 3).all()
+    if gap_violations(scores(w, h["x"], h["wg"], h["bias"]), w.k).any():
+        pytest.skip("seeded inputs violate the gap under the changed bias")
+    y_ref = _oracle(h, w.k)
+    for tiling in (ROW, WIDE):
+        L = _layer(d, w.k, tiling | PREFILL)
+        err = bf16_np_to_f64(to_np_bf16(L(d["x"]))) - y_ref
+        assert L.device_error() == 0
+        assert np.sqrt(np.mean(err * err)) <= 5e-3 * np.sqrt(np.mean(y_ref * y_ref))
+        assert np.abs(err).max() <= 2e-2 * np.abs(y_ref).max()
+
+
+def test_wide_tiles_deterministic_and_close_to_row_tiles(cuda_device):
+    """Two runs give the same bits; the two tilings agree to fp32 accumulation-order rounding (both
+    round h to bf16, so a few h entries may differ by one bf16 ulp)."""
+    w = W(400, 256, 8, 2, 256, Fs=128, bias="normal:0.5")
+    h, d = _case(w)
+    Lw = _layer(d, w.k, WIDE | PREFILL)
+    y1, y2 = to_np_bf16(Lw(d["x"])), to_np_bf16(Lw(d["x"]))
+    assert (y1 == y2).all()
+    yr = bf16_np_to_f64(to_np_bf16(_layer(d, w.k, ROW | PREFILL)(d["x"])))
+    yw = bf16_np_to_f64(y1)
+    assert np.abs(yw - yr).max() <= 1e-2 * np.sqrt(np.mean(yr * yr))
+
+
+def test_standalone_ffn_entry_prefill_sizes(cuda_device):
+    """moe_grouped_swiglu_ffn (128-row tiles) on short and long segments matches the oracle's per-row
+    expert FFN."""
+    import torch
+
+    rng = np.random.default_rng(5)
+    for M, E in ((900, 4), (3000, 2)):
+        D, F = 128, 192
+        w = W(M, D, E, 1, F)
+        gu = mi.host_inputs(w)["gate_up"]
+        dn = mi.host_inputs(w)["down"]
+        counts = np.bincount(rng.integers(0, E, size=M), minlength=E)
+        offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        xp = mi.rows_bf16(mi.STREAM_X, np.arange(M), D, 1.0, seed=77)
+        scale = rng.uniform(0.1, 1.0, size=M).astype(np.float32)
+        out, _ = moe.moe_grouped_swiglu_ffn(to_torch_bf16(xp), torch.from_numpy(offsets).cuda(),
+                                            torch.from_numpy(scale).cuda(), to_torch_bf16(gu), to_torch_bf16(dn))
+        got = out.cpu().numpy().astype(np.float64)
+        ref = np.stack([scale[r] * oracle.expert_ffn(xp[r], gu[e], dn[e])
+                        for e in range(E) for r in range(offsets[e], offsets[e + 1])])
+        assert rel_rms_err(got, ref) <= REL_RMS_TOL
