@@ -550,8 +550,8 @@ def main():
     ap.add_argument("--train", action="store_true",
                     help="time a training step (forward saving g|u + backward) instead of the forward")
     ap.add_argument("--tiling", default="auto", choices=["auto", "row", "wide"],
-                    help="prefill tiling of the expert GEMMs (bf16): the layer's default rule, 128-row tiles, "
-                         "or token-wide tiles")
+                    help="prefill tiling of the expert GEMMs (bf16): the layer's default (gate_up on 128-row "
+                         "tiles, down on token-wide tiles), 128-row tiles for both, or token-wide tiles for both")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="expert weight format; fp8 (E4M3, per-row scales) runs the decode kernels, T <= 64")
     args = ap.parse_args()

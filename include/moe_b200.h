@@ -171,11 +171,12 @@ moe_status_t moe_combine(const float* out_perm, const int32_t* inv_perm, const f
  * bf16 weights only. */
 #define MOE_FLAG_SAVE_FOR_BACKWARD 4
 /* Prefill tiling of the expert GEMMs (at most one of the two; neither with FORCE_DECODE):
- *  ROW_TILES  128 permuted rows x 256 output columns per tile (tokens are the MMA's M);
- *  WIDE_TILES 128 weight rows x up to 256 rows of one expert segment (tokens are N, so a
+ *  ROW_TILES  both GEMMs on 128 permuted rows x 256 output columns per tile (tokens are the
+ *             MMA's M);
+ *  WIDE_TILES both on 128 weight rows x up to 256 rows of one expert segment (tokens are N, so a
  *             segment's last tile is padded to a multiple of 16 rows instead of 128).
- * Without either, ROW_TILES.  Both give the same routing; outputs agree within fp32 rounding
- * order. */
+ * Without either, gate_up runs ROW_TILES and down WIDE_TILES.  All give the same routing;
+ * outputs agree within fp32 rounding order. */
 #define MOE_FLAG_PREFILL_ROW_TILES 8
 #define MOE_FLAG_PREFILL_WIDE_TILES 16
 
@@ -251,6 +252,7 @@ int moe_layer_kernel_count(const moe_layer_desc_t* desc);
 #define MOE_PATH_FP8_STREAMING 1
 #define MOE_PATH_ROW_TILES 2
 #define MOE_PATH_WIDE_TILES 3
+#define MOE_PATH_MIXED_TILES 4 /* gate_up on 128-row tiles, down on token-wide tiles */
 int moe_layer_gemm_path(const moe_layer_desc_t* desc);
 
 /* ----------------------------------------------------------------------------------------

@@ -20,7 +20,7 @@ MOE_FLAG_FORCE_DECODE = 2
 MOE_FLAG_SAVE_FOR_BACKWARD = 4
 MOE_FLAG_PREFILL_ROW_TILES = 8
 MOE_FLAG_PREFILL_WIDE_TILES = 16
-MOE_PATH_STREAMING, MOE_PATH_FP8_STREAMING, MOE_PATH_ROW_TILES, MOE_PATH_WIDE_TILES = 0, 1, 2, 3
+MOE_PATH_STREAMING, MOE_PATH_FP8_STREAMING, MOE_PATH_ROW_TILES, MOE_PATH_WIDE_TILES, MOE_PATH_MIXED_TILES = 0, 1, 2, 3, 4
 MOE_WEIGHTS_BF16 = 0
 MOE_WEIGHTS_FP8_E4M3 = 1
 
@@ -308,12 +308,12 @@ class MoELayer:
 
     def gemm_path(self, T: int) -> str:
         """The expert-GEMM kernels a forward over T tokens runs: "streaming", "fp8_streaming",
-        "row_tiles" or "wide_tiles"."""
+        "row_tiles", "wide_tiles" or "mixed_tiles" (gate_up on row tiles, down on wide tiles)."""
         d = self.desc(T)
         code = lib().moe_layer_gemm_path(ctypes.byref(d))
         if code < 0:
             raise MoeError(1, "moe_layer_gemm_path")
-        return ("streaming", "fp8_streaming", "row_tiles", "wide_tiles")[code]
+        return ("streaming", "fp8_streaming", "row_tiles", "wide_tiles", "mixed_tiles")[code]
 
     def forward(self, x, y=None, stream=None):
         import torch

@@ -48,11 +48,17 @@ bool use_decode(const moe_layer_desc_t& d) {
 
 int decode_tile(int max_seg) { return ((max_seg + 15) / 16) * 16; }
 
-// Prefill tiling: token-wide tiles (weights as the MMA's M, up to 256 rows of one segment as N)
-// pad each segment's last tile to 16 rows instead of 128 and need fewer MMA cycles, but measured
-// slower on every prefill shape here (their gate_up reaches lower tensor-pipe activity), so the
-// 128-row tiles are the default and the token-wide ones run only when asked for.
-bool wide_tiles(int flags) { return (flags & MOE_FLAG_PREFILL_WIDE_TILES) != 0; }
+// Prefill tiling, as bits: 1 = gate_up on token-wide tiles (weights as the MMA's M, up to 256 rows
+// of one segment as N), 2 = down on token-wide tiles; clear bits mean 128-row tiles.  Token-wide
+// tiles pad a segment's last tile to 16 rows instead of 128, but their gate_up (SwiGLU epilogue
+// through a shared-memory transpose) measured slower than the 128-row one, while their down
+// measured faster; the default mixes the two.
+constexpr int kWideGateUp = 1, kWideDown = 2;
+int wide_tiles(int flags) {
+  if (flags & MOE_FLAG_PREFILL_WIDE_TILES) return kWideGateUp | kWideDown;
+  if (flags & MOE_FLAG_PREFILL_ROW_TILES) return 0;
+  return kWideDown;
+}
 
 struct LayerWs {
   size_t split_counters, split_partial, split_partial_bytes, gu_saved, gu_saved_sh, router, topk_idx, topk_w, scratch, counts, offsets, perm_token, inv_perm, p_perm, x_perm, h, h_sh, out_perm,
@@ -157,7 +163,7 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
                      int F, const uint16_t* gate_up, const uint16_t* down, uint16_t* h, float* out_perm,
                      // optional shared expert over x[T, D]
                      const uint16_t* x, int T, int Fs, const uint16_t* sgu, const uint16_t* sdn, uint16_t* h_sh,
-                     float* out_sh, int decode_nt, bool wide, int* err, cudaStream_t s, cudaEvent_t ev_mid,
+                     float* out_sh, int decode_nt, int wide, int* err, cudaStream_t s, cudaEvent_t ev_mid,
                      unsigned ev_flags, uint16_t* save_gu = nullptr, uint16_t* save_gu_sh = nullptr) {
   GemmSetHost g[2];
   memset(g, 0, sizeof(g));
@@ -169,7 +175,7 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
     g[1].n_out = Fs, g[1].out = h_sh, g[1].save_gu = save_gu_sh;
     n_sets = 2;
   }
-  if (decode_nt == 0 && wide)
+  if (decode_nt == 0 && (wide & kWideGateUp))
     MOE_CUDA_TRY(launch_grouped_gemm_wide(kGateUp, g, n_sets, err, s));
   else
     MOE_CUDA_TRY(launch_grouped_gemm(kGateUp, g, n_sets, decode_nt, err, s));
@@ -182,7 +188,7 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
     dn[1].K = Fs, dn[1].a = h_sh, dn[1].a_rows = T, dn[1].w = sdn, dn[1].n_groups = 1, dn[1].m_rows = T;
     dn[1].n_out = D, dn[1].out = out_sh;
   }
-  if (decode_nt == 0 && wide)
+  if (decode_nt == 0 && (wide & kWideDown))
     MOE_CUDA_TRY(launch_grouped_gemm_wide(kDown, dn, n_sets, err, s));
   else
     MOE_CUDA_TRY(launch_grouped_gemm(kDown, dn, n_sets, decode_nt, err, s));
@@ -490,7 +496,8 @@ int moe_layer_gemm_path(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK) return -1;
   if (desc->weight_format == MOE_WEIGHTS_FP8_E4M3) return MOE_PATH_FP8_STREAMING;
   if (use_decode(*desc)) return MOE_PATH_STREAMING;
-  return wide_tiles(desc->flags) ? MOE_PATH_WIDE_TILES : MOE_PATH_ROW_TILES;
+  const int wide = wide_tiles(desc->flags);
+  return wide == 0 ? MOE_PATH_ROW_TILES : wide == kWideDown ? MOE_PATH_MIXED_TILES : MOE_PATH_WIDE_TILES;
 }
 
 moe_status_t moe_update_router_bias(const int32_t* counts, int E, float gamma, float* bias, moe_stream_t stream) {

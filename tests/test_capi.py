@@ -223,15 +223,16 @@ def test_backward_entry_validates_on_host(L):
 
 
 def test_gemm_path_query(L):
-    """The host-only path query follows the flags and the default rule: T <= 64 streams the weights,
-    larger T runs the 128-row tiles unless the token-wide tiles are asked for; E4M3 weights always
-    stream."""
+    """The host-only path query follows the flags and the default rule: T <= 64 streams the weights;
+    larger T runs gate_up on 128-row tiles and down on token-wide tiles unless one tiling is asked
+    for; E4M3 weights always stream."""
     P = lambda **kw: L.moe_layer_gemm_path(ctypes.byref(_desc(**kw)))
     assert P() == moe.MOE_PATH_STREAMING                                     # T = 16
-    assert P(T=16, flags=moe.MOE_FLAG_FORCE_PREFILL) == moe.MOE_PATH_ROW_TILES
+    assert P(T=16, flags=moe.MOE_FLAG_FORCE_PREFILL) == moe.MOE_PATH_MIXED_TILES
     assert P(T=16, flags=moe.MOE_FLAG_FORCE_PREFILL | moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_WIDE_TILES
-    assert P(T=65) == moe.MOE_PATH_ROW_TILES
-    assert P(T=4096, E=8, k=2) == moe.MOE_PATH_ROW_TILES
+    assert P(T=16, flags=moe.MOE_FLAG_FORCE_PREFILL | moe.MOE_FLAG_PREFILL_ROW_TILES) == moe.MOE_PATH_ROW_TILES
+    assert P(T=65) == moe.MOE_PATH_MIXED_TILES
+    assert P(T=4096, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_ROW_TILES) == moe.MOE_PATH_ROW_TILES
     assert P(T=4096, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_WIDE_TILES
     assert P(T=16, flags=moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_STREAMING  # tiling flags leave decode
     assert P(T=300, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_ROW_TILES) == moe.MOE_PATH_ROW_TILES
@@ -239,5 +240,6 @@ def test_gemm_path_query(L):
     assert P(**FP8, flags=moe.MOE_FLAG_PREFILL_WIDE_TILES) == -1             # E4M3 has no prefill path
     assert P(k=9) == -1
     # the training forward runs a prefill tiling at any T
-    assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD) == moe.MOE_PATH_ROW_TILES
+    assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD) == moe.MOE_PATH_MIXED_TILES
+    assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD | moe.MOE_FLAG_PREFILL_ROW_TILES) == moe.MOE_PATH_ROW_TILES
     assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD | moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_WIDE_TILES

@@ -332,9 +332,9 @@ FULL = ["mixtral", "gptoss", "gptoss_decode_T1", "gptoss_decode_T8", "gptoss_dec
 SAMPLE = {"mixtral": 6, "gptoss": 8, "deepseek": 4, "deepseek_decode": 4}
 
 
-# the token-wide prefill tiling (the default is the 128-row tiling), at full size
-OTHER_TILING = [("mixtral", moe.MOE_FLAG_PREFILL_WIDE_TILES), ("gptoss", moe.MOE_FLAG_PREFILL_WIDE_TILES),
-                ("deepseek", moe.MOE_FLAG_PREFILL_WIDE_TILES)]
+# the prefill tilings other than the default mix, at full size
+OTHER_TILING = [("mixtral", moe.MOE_FLAG_PREFILL_ROW_TILES), ("gptoss", moe.MOE_FLAG_PREFILL_WIDE_TILES),
+                ("deepseek", moe.MOE_FLAG_PREFILL_ROW_TILES), ("deepseek", moe.MOE_FLAG_PREFILL_WIDE_TILES)]
 
 
 @pytest.mark.slow

@@ -1,6 +1,6 @@
-"""Both prefill tilings of the expert GEMMs against the fp64 oracle: 128-row tiles (permuted rows
-as the MMA's M) and token-wide tiles (128 weight rows as M, up to 256 rows of one expert segment
-as N).  Cases cover segments of one ragged token tile, of several token tiles, empty segments, a
+"""The prefill tilings of the expert GEMMs against the fp64 oracle: 128-row tiles (permuted rows
+as the MMA's M), token-wide tiles (128 weight rows as M, up to 256 rows of one expert segment as
+N), and the default mix of the two (gate_up on 128-row tiles, down on token-wide tiles).  Cases cover segments of one ragged token tile, of several token tiles, empty segments, a
 one-row segment, output columns that end mid-tile (D = 192: 1.5 column tiles of the down GEMM)
 and the shared expert; routing is bit-exact and the layer output within 2e-2 x RMS(y_oracle)."""
 import numpy as np
@@ -51,12 +51,15 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("tiling", [ROW, WIDE], ids=["row_tiles", "wide_tiles"])
+NAMES = {ROW: "row_tiles", WIDE: "wide_tiles", 0: "mixed_tiles"}
+
+
+@pytest.mark.parametrize("tiling", [ROW, WIDE, 0], ids=["row_tiles", "wide_tiles", "mixed_tiles"])
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
-def test_layer_parity_both_tilings(cuda_device, w, tiling):
+def test_layer_parity_all_tilings(cuda_device, w, tiling):
     h, d = _case(w)
     L = _layer(d, w.k, tiling | PREFILL)
-    assert L.gemm_path(w.T) == ("row_tiles" if tiling == ROW else "wide_tiles")
+    assert L.gemm_path(w.T) == NAMES[tiling]
     y = bf16_np_to_f64(to_np_bf16(L(d["x"])))
     assert L.device_error() == 0
     assert rel_rms_err(y, _oracle(h, w.k)) <= REL_RMS_TOL
