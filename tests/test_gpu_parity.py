@@ -90,6 +90,7 @@ ROUTER_CASES = [
     W(40, 256, 600, 16, 64, bias="zipf:1.1"),
     W(20, 128, 1024, 32, 64),
     W(33, 192, 6, 6, 64),
+    W(48, 1088, 256, 8, 64, bias="normal:0.5"),           # decode T with W_g > 256 Ki: tensor-core router
 ]
 
 
