@@ -15,7 +15,8 @@
 // (at N >= 96, where an MMA's time follows N) and reads each weight tile once per 256 tokens.
 //
 // Kernel layout (persistent, one CTA per SM, 192 threads):
-//   warp 0     TMA producer: per 64-wide K block, the weight tile (16 KB) and the token rows
+//   warp 0     TMA producer: per 64-wide K block, the weight tile (16 KB, one copy; gate_up's
+//              through a 4-D view that stacks the gate and up rows) and the token rows
 //              (one 256-row box for a full tile, else ceil(rows / 64) boxes of 64 rows, 8 KB
 //              each) into a 4-stage ring;
 //   warp 1     TMEM allocator and MMA issuer (one thread): 4 x tcgen05.mma M=128, N=round16(rows),
@@ -58,7 +59,9 @@ static_assert(kWStageBytes % 1024 == 0 && kWStagingBytes % 16 == 0, "alignment")
 struct alignas(64) WideParams {
   CUtensorMap t_map[2];     // token operand per set (x_perm / x / h), box 64 K x 64 rows
   CUtensorMap t_map256[2];  // the same tensor, box 64 K x 256 rows (full token tiles: one copy)
-  CUtensorMap w_map[2];  // weights per set, box 64 K x (64 rows gate_up | 128 rows down)
+  CUtensorMap w_map[2];  // weights per set: down [rows, K], box 64 K x 128 rows; gate_up viewed as
+                         // [groups][2 halves][F rows][K], box 64 K x 64 rows x 2 halves (the
+                         // gate and up rows of 64 output columns in one copy)
   const int32_t* offsets[2];
   void* out[2];          // gate_up: bf16 h [rows, F]; down: fp32 [rows, D]
   const float* row_scale[2];
@@ -153,6 +156,15 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ void tma_load_4d(const CUtensorMap* map, uint64_t* bar, void* dst, int32_t x, int32_t y,
+                                            int32_t z, int32_t w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
 template <int KIND>
 __global__ void __launch_bounds__(kWThreads, 1) grouped_gemm_wide_kernel(const __grid_constant__ WideParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -244,9 +256,7 @@ __global__ void __launch_bounds__(kWThreads, 1) grouped_gemm_wide_kernel(const _
           mbar_arrive_expect_tx(&full[stage], kWTileA + nb * kWBox);
           const int kx = kb * kWBK;
           if constexpr (KIND == kGateUp) {
-            const int F = p.n_out[ti.set];
-            tma_load_2d(&p.w_map[ti.set], &full[stage], sb, kx, wbase + ti.n * 64);               // gate rows
-            tma_load_2d(&p.w_map[ti.set], &full[stage], sb + kWTileA / 2, kx, wbase + F + ti.n * 64);  // up rows
+            tma_load_4d(&p.w_map[ti.set], &full[stage], sb, kx, ti.n * 64, 0, ti.gl);  // 64 gate rows, then 64 up
           } else {
             tma_load_2d(&p.w_map[ti.set], &full[stage], sb, kx, wbase + ti.n * 128);
           }
@@ -419,6 +429,20 @@ bool w_make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// gate_up weights [groups, 2F, K] bf16 as a 4-D tensor (K, F rows, 2 halves, groups); the box of
+// 64 K x 64 rows x 2 halves lands as 128 rows of 128 bytes: the 64 gate rows, then their 64 up rows.
+bool w_make_gate_up_map(CUtensorMap* m, const void* base, int groups, int F, int K) {
+  WEncodeFn enc = w_encode_fn();
+  if (enc == nullptr || groups <= 0 || F <= 0 || K <= 0) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)K, (cuuint64_t)F, 2, (cuuint64_t)groups};
+  cuuint64_t strides[3] = {(cuuint64_t)K * 2, (cuuint64_t)F * K * 2, (cuuint64_t)2 * F * K * 2};
+  cuuint32_t box[4] = {64, 64, 2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int w_num_sms() {
   static int n = 0;
   if (n == 0) {
@@ -445,8 +469,8 @@ cudaError_t launch_wide(const GemmSetHost* sets, int n_sets, int* err, cudaStrea
     if (!w_make_map(&p.t_map[i], st.a, (uint64_t)st.a_rows, (uint64_t)st.K, 64) ||
         !w_make_map(&p.t_map256[i], st.a, (uint64_t)st.a_rows, (uint64_t)st.K, kWT))
       return cudaErrorInvalidValue;
-    if (!w_make_map(&p.w_map[i], st.w, (uint64_t)st.n_groups * p.w_rows[i], (uint64_t)st.K,
-                    KIND == kGateUp ? 64 : 128))
+    if (KIND == kGateUp ? !w_make_gate_up_map(&p.w_map[i], st.w, st.n_groups, st.n_out, st.K)
+                        : !w_make_map(&p.w_map[i], st.w, (uint64_t)st.n_groups * p.w_rows[i], (uint64_t)st.K, 128))
       return cudaErrorInvalidValue;
     p.offsets[i] = st.offsets;
     p.out[i] = st.out;
