@@ -58,6 +58,7 @@ def _L():
         L.oracle_layer_f64.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64, P, i32]
         L.oracle_layer_backward_f64.argtypes = [P, P, P, P, P, P, P, P, i64, i64, i32, i32, i64, i64,
                                                 P, P, P, P, P, P, i32]
+        L.oracle_router_aux_loss_f64.argtypes = [P, P, P, i64, i64, i32, i32, ctypes.c_double, P, P, P, i32]
         _lib = L
     return _lib
 
@@ -304,6 +305,24 @@ def layer_backward(x, wg, bias, gate_up, down, k, dy, shared_gate_up=None, share
     if rc != 0:
         raise ValueError(f"oracle_layer_backward_f64 rc={rc}")
     return out
+
+
+def router_aux_loss(x, wg, bias, k, alpha):
+    """Load-balancing auxiliary loss L = alpha * E * sum_e f_e P_e of the router (the reading and its
+    gradient are stated at oracle_router_aux_loss_f64): (loss float, dw_gate [E, D], dx [T, D]),
+    float64; f counts the top-k of l + bias and carries no gradient."""
+    x, wg = _f64(x), _f64(wg)
+    T, D = x.shape
+    E = wg.shape[0]
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    loss = np.zeros(1)
+    dwg = np.empty((E, D))
+    dx = np.empty((T, D))
+    rc = _L().oracle_router_aux_loss_f64(x.ctypes.data, wg.ctypes.data, _ptr(b), T, D, E, k, float(alpha),
+                                         loss.ctypes.data, dwg.ctypes.data, dx.ctypes.data, _nthreads())
+    if rc != 0:
+        raise ValueError(f"oracle_router_aux_loss_f64 rc={rc}")
+    return float(loss[0]), dwg, dx
 
 
 # ----------------------------------------------------------------------------- gap-enforced inputs

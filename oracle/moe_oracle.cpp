@@ -547,4 +547,64 @@ int oracle_layer_backward_f64(const double* x, const double* wg, const float* bi
   return 0;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Load-balancing auxiliary loss of the router (training).  The pages say only that training adds
+// an auxiliary loss that penalises the router for spreading tokens unevenly and pushes it to use
+// all experts alike (josueisai.com, "El coste que la cifra bonita esconde"; dev.smart-guide.co.kr,
+// "Limitaciones y Cuidados": router collapse without a load-balancing loss).  They print no
+// formula; the reading taken is the product form of expert load and router probability:
+//   f_e = (number of the T*k routed slots that chose e) / (T*k)     (top-k of l + bias)
+//   P_e = (1/T) sum_t softmax(l_t)_e                               (all E, unbiased logits)
+//   L   = alpha * E * sum_e f_e P_e                                (= alpha when both are uniform)
+// f is piecewise constant in the parameters (it counts a selection), so only P carries a gradient:
+//   dL/dl_{t,e} = (alpha E / T) s_{t,e} (f_e - sum_j f_j s_{t,j}),   s_t = softmax(l_t),
+//   dW_g[e] = sum_t dL/dl_{t,e} x_t,   dx_t = sum_e dL/dl_{t,e} W_g[e].
+// fp64 parameters; outputs (overwritten): loss [1], dwg [E, D], dx [T, D].  Returns 0, or -1 on
+// invalid sizes.  T = 0 gives loss 0 and zero gradients.
+int oracle_router_aux_loss_f64(const double* x, const double* wg, const float* bias, int64_t T, int64_t D, int E,
+                               int k, double alpha, double* loss, double* dwg, double* dx, int nthreads) {
+  if (T < 0 || D < 1 || E < 1 || k < 1 || k > E) return -1;
+  std::fill(dwg, dwg + (int64_t)E * D, 0.0);
+  *loss = 0.0;
+  if (T == 0) return 0;
+  std::vector<double> l((size_t)T * E), s((size_t)T * E), dl((size_t)T * E);
+  std::vector<int32_t> idx((size_t)T * k);
+  for_tokens(T, nthreads, [&](int64_t t) {
+    std::vector<double> p(k);
+    router_logits_f64(x + t * D, wg, D, E, &l[t * E]);
+    select_and_weight(&l[t * E], bias, E, k, &idx[t * k], p.data());
+    double m = l[t * E];
+    for (int e = 1; e < E; ++e) m = std::max(m, l[t * E + e]);
+    double z = 0.0;
+    for (int e = 0; e < E; ++e) z += std::exp(l[t * E + e] - m);
+    for (int e = 0; e < E; ++e) s[t * E + e] = std::exp(l[t * E + e] - m) / z;
+  });
+  std::vector<double> f(E, 0.0), P(E, 0.0);
+  for (int64_t i = 0; i < T * k; ++i) f[idx[i]] += 1.0;
+  for (int e = 0; e < E; ++e) f[e] /= (double)(T * k);
+  for (int64_t t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) P[e] += s[t * E + e];
+  double acc = 0.0;
+  for (int e = 0; e < E; ++e) acc += f[e] * (P[e] / (double)T);
+  *loss = alpha * (double)E * acc;
+  const double scale = alpha * (double)E / (double)T;
+  for_tokens(T, nthreads, [&](int64_t t) {
+    double c = 0.0;
+    for (int e = 0; e < E; ++e) c += f[e] * s[t * E + e];
+    double* dxt = dx + t * D;
+    std::fill(dxt, dxt + D, 0.0);
+    for (int e = 0; e < E; ++e) {
+      const double g = scale * s[t * E + e] * (f[e] - c);
+      dl[t * E + e] = g;
+      for (int64_t d = 0; d < D; ++d) dxt[d] += g * wg[(int64_t)e * D + d];
+    }
+  });
+  for_tokens(E, nthreads, [&](int64_t e) {
+    double* dw = dwg + e * D;
+    for (int64_t t = 0; t < T; ++t)
+      for (int64_t d = 0; d < D; ++d) dw[d] += dl[t * E + e] * x[t * D + d];
+  });
+  return 0;
+}
+
 }  // extern "C"

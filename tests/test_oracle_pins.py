@@ -449,3 +449,54 @@ def test_f64_forward_is_the_bf16_forward():
     y64 = oracle.layer_f64(h["x"], h["wg"], h["bias"], h["gate_up"], h["down"], 2, h["shared_gate_up"],
                            h["shared_down"])
     np.testing.assert_allclose(y64, y16, rtol=1e-13, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- auxiliary loss
+def test_aux_loss_is_alpha_when_router_probabilities_are_uniform():
+    """W_g = 0 makes every softmax uniform (P_e = 1/E), so L = alpha * E * sum_e f_e / E = alpha for
+    any selection; the logit gradient is (alpha / T)(f_e - 1/E), so dW_g[e] = (alpha/T)(f_e - 1/E)
+    sum_t x_t and dx = 0.  With zero logits the selection is the top-k of the bias alone."""
+    rng = np.random.default_rng(11)
+    T, D, E, k, alpha = 7, 12, 6, 2, 0.03
+    x = rng.normal(size=(T, D))
+    wg = np.zeros((E, D))
+    bias = np.array([0.1, 0.5, -0.2, 0.4, 0.0, -0.3], np.float32)
+    loss, dwg, dx = oracle.router_aux_loss(x, wg, bias, k, alpha)
+    assert loss == pytest.approx(alpha, rel=1e-14)
+    f = np.zeros(E)
+    f[[1, 3]] = 1.0 / k  # the two largest biases
+    np.testing.assert_allclose(dwg, np.outer(alpha / T * (f - 1.0 / E), x.sum(axis=0)), rtol=1e-12, atol=1e-15)
+    assert not dx.any()
+
+
+def test_aux_loss_two_expert_closed_form():
+    """E = 2, k = 1, one token, D = 1 (x = [x0], W_g = [[a], [b]], a x0 > b x0): f = (1, 0) and
+    P_0 = sigmoid(l_0 - l_1), so L = 2 alpha sigmoid(l_0 - l_1) and dL/dl_0 = -dL/dl_1 =
+    2 alpha sig (1 - sig)."""
+    alpha, x0, a, b = 0.5, 1.5, 0.8, -0.4
+    loss, dwg, dx = oracle.router_aux_loss(np.array([[x0]]), np.array([[a], [b]]), None, 1, alpha)
+    sig = 1.0 / (1.0 + np.exp(-(a - b) * x0))
+    g = 2 * alpha * sig * (1 - sig)
+    assert loss == pytest.approx(2 * alpha * sig, rel=1e-14)
+    np.testing.assert_allclose(dwg[:, 0], [g * x0, -g * x0], rtol=1e-13)
+    assert dx[0, 0] == pytest.approx(g * a - g * b, rel=1e-13)
+
+
+def test_aux_loss_gradient_matches_finite_differences():
+    """<grad, V> equals the central difference of L along a random V, for x and W_g (the fp64 loss
+    is smooth while the selection stays fixed; top-k scores are 0.05 apart); and the logit gradient
+    of each token sums to zero (softmax shift invariance), so sum_e dW_g[e] = 0."""
+    for seed, k in ((1, 2), (2, 1), (3, 3)):
+        P = _bwd_problem(seed=seed, T=5, D=10, E=6, k=k)
+        loss, dwg, dx = oracle.router_aux_loss(P["x"], P["wg"], P["bias"], k, 0.1)
+        rng = np.random.default_rng(seed + 50)
+        eps = 1e-5
+        for name, g in (("x", dx), ("wg", dwg)):
+            V = rng.normal(size=P[name].shape)
+            q = dict(P)
+            q[name] = P[name] + eps * V
+            lp = oracle.router_aux_loss(q["x"], q["wg"], P["bias"], k, 0.1)[0]
+            q[name] = P[name] - eps * V
+            lm = oracle.router_aux_loss(q["x"], q["wg"], P["bias"], k, 0.1)[0]
+            assert float(np.sum(g * V)) == pytest.approx((lp - lm) / (2 * eps), rel=1e-6, abs=1e-11), (seed, name)
+        assert np.abs(dwg.sum(axis=0)).max() < 1e-12 * max(1.0, np.abs(dwg).max())
