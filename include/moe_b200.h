@@ -77,6 +77,29 @@ moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, cons
                              size_t ws_bytes, moe_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
+ * Router load-balancing auxiliary loss (training).  josueisai.com "Mixture of experts", section
+ * "El coste que la cifra bonita esconde": MoE training adds a loss that penalises the router for
+ * spreading tokens unevenly (dev.smart-guide.co.kr, "Limitaciones y Cuidados": without it the
+ * router collapses onto few experts).  The pages print no formula; the one computed here is the
+ * product of each expert's load and mean router probability:
+ *   L = alpha * E * sum_e f_e * P_e,
+ *   f_e = (slots of the top-k of l + bias that chose e) / (T * k)      -- a count, no gradient,
+ *   P_e = mean over tokens of softmax(l_t)_e over all E unbiased logits,
+ * so L = alpha when both are uniform.  Outputs (device, fp32, overwritten):
+ *   loss    [1]      L
+ *   dw_gate [E, D]   dL/dW_g      (add it to the layer backward's dw_gate)
+ *   dx      [T, D]   dL/dx        (add it to the layer backward's dx)
+ * Logits are computed as in moe_router_topk; every sum runs in a fixed order (deterministic).
+ * T = 0 writes loss = 0 and zeros dw_gate.  x, w_gate 16-byte aligned; bias, loss, dw_gate, dx
+ * 4-byte aligned.
+ *   ws: >= moe_router_aux_loss_workspace_size(T, D, E, k) bytes of device memory.
+ * ---------------------------------------------------------------------------------------- */
+size_t moe_router_aux_loss_workspace_size(int T, int D, int E, int k);
+moe_status_t moe_router_aux_loss(const moe_bf16_t* x, const moe_bf16_t* w_gate, const float* bias, int T,
+                                 int D, int E, int k, float alpha, float* loss, float* dw_gate, float* dx,
+                                 void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
  * Step 2: dispatch -- histogram, exclusive prefix sum and permutation into expert-contiguous
  * order (keryc.com "Mixture of Experts optimiza Transformers y LLMs", section "Ejecucion
  * eficiente: backends de expertos": the grouped backend sorts tokens by expert id).

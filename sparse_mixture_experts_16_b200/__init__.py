@@ -32,7 +32,8 @@ STATUS = {
 
 # every symbol include/moe_b200.h declares
 EXPORTS = (
-    "moe_quantize_rows_fp8", "moe_router_topk_workspace_size", "moe_router_topk", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
+    "moe_quantize_rows_fp8", "moe_router_topk_workspace_size", "moe_router_topk", "moe_router_aux_loss_workspace_size",
+    "moe_router_aux_loss", "moe_permute_workspace_size", "moe_permute", "moe_permute_noalloc",
     "moe_grouped_swiglu_ffn_workspace_size",
     "moe_grouped_swiglu_ffn", "moe_combine", "moe_layer_workspace_size", "moe_layer_forward",
     "moe_layer_forward_host", "moe_layer_forward_timed", "moe_layer_kernel_count", "moe_layer_gemm_path", "moe_update_router_bias",
@@ -82,6 +83,8 @@ def lib():
             "moe_quantize_rows_fp8": ([P, ctypes.c_int64, I, P, P, P], I),
             "moe_router_topk_workspace_size": ([I, I, I], Z),
             "moe_router_topk": ([P, P, P, I, I, I, I, P, P, P, Z, P], I),
+            "moe_router_aux_loss_workspace_size": ([I, I, I, I], Z),
+            "moe_router_aux_loss": ([P, P, P, I, I, I, I, ctypes.c_float, P, P, P, P, Z, P], I),
             "moe_permute_workspace_size": ([I, I, I], Z),
             "moe_permute": ([P, P, P, I, I, I, I, P, P, P, P, P, P, P, Z, P], I),
             "moe_permute_noalloc": ([P, P, P, I, I, I, I, P, P, P, P, P, P, P], I),
@@ -167,6 +170,32 @@ def moe_router_topk(x, w_gate, bias, k, topk_idx=None, topk_w=None, ws=None, str
     _check(lib().moe_router_topk(x.data_ptr(), w_gate.data_ptr(), _ptr(bias), T, D, E, k, topk_idx.data_ptr(),
                                  topk_w.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)), "moe_router_topk")
     return topk_idx, topk_w
+
+
+def moe_router_aux_loss(x, w_gate, bias, k, alpha, ws=None, stream=None):
+    """Router load-balancing auxiliary loss L = alpha * E * sum_e f_e P_e (training) and its
+    gradients -> (loss [1], dw_gate [E, D], dx [T, D]), all fp32 on x's device; add the gradients
+    to the layer backward's."""
+    import torch
+
+    T, D = x.shape
+    E = w_gate.shape[0]
+    _need(x, torch.bfloat16, None, "x")
+    _need(w_gate, torch.bfloat16, (E, D), "w_gate")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    loss = torch.empty(1, dtype=torch.float32, device=x.device)
+    dwg = torch.empty(E, D, dtype=torch.float32, device=x.device)
+    dx = torch.empty(T, D, dtype=torch.float32, device=x.device)
+    need = lib().moe_router_aux_loss_workspace_size(T, D, E, k)
+    if need == 0:
+        raise MoeError(1, "moe_router_aux_loss_workspace_size")
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    _check(lib().moe_router_aux_loss(x.data_ptr(), w_gate.data_ptr(), _ptr(bias), T, D, E, k, float(alpha),
+                                     loss.data_ptr(), dwg.data_ptr(), dx.data_ptr(), ws.data_ptr(), ws.numel(),
+                                     _stream(stream)), "moe_router_aux_loss")
+    return loss, dwg, dx
 
 
 def moe_permute(topk_idx, topk_w, x, E, stream=None, ws=None):

@@ -5,6 +5,7 @@
 #include <cstring>
 
 #include "grouped_gemm_wide.cuh"
+#include "router_aux.cuh"
 #include "moe_common.cuh"
 
 using namespace moe;
@@ -364,6 +365,65 @@ moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, cons
   cudaStream_t s = (cudaStream_t)stream;
   MOE_CUDA_TRY(launch_router_gemm(x, w_gate, T, D, E, part, router_ld(E), splits, reinterpret_cast<int*>(b), s));
   MOE_CUDA_TRY(launch_router_select(part, splits, T, router_ld(E), bias, E, k, topk_idx, topk_w, s));
+  return MOE_OK;
+}
+
+namespace {
+struct AuxWs {
+  size_t part, idx, w, counts, c, dl, total;
+};
+AuxWs aux_ws(int T, int D, int E, int k) {
+  AuxWs a;
+  size_t o = kWsHeader;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  a.part = take(router_scratch_bytes(T, D, E));
+  a.idx = take((size_t)T * k * 4);
+  a.w = take((size_t)T * k * 4);
+  a.counts = take((size_t)E * 4);
+  a.c = take((size_t)T * 4);
+  a.dl = take((size_t)T * E * 4);
+  a.total = o;
+  return a;
+}
+}  // namespace
+
+size_t moe_router_aux_loss_workspace_size(int T, int D, int E, int k) {
+  if (shape_status(T, D, E, k) != MOE_OK) return 0;
+  return aux_ws(T, D, E, k).total;
+}
+
+moe_status_t moe_router_aux_loss(const moe_bf16_t* x, const moe_bf16_t* w_gate, const float* bias, int T, int D,
+                                 int E, int k, float alpha, float* loss, float* dw_gate, float* dx, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t st = shape_status(T, D, E, k);
+  if (st != MOE_OK) return st;
+  if (!x || !w_gate || !loss || !dw_gate || !dx || !ws) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_gate, 16) || !aligned(bias, 4) || !aligned(loss, 4) || !aligned(dw_gate, 4) ||
+      !aligned(dx, 4) || !aligned(ws, 256))
+    return MOE_ERR_ALIGNMENT;
+  const AuxWs a = aux_ws(T, D, E, k);
+  if (ws_bytes < a.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = check_device()) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (T == 0) {
+    MOE_CUDA_TRY(cudaMemsetAsync(loss, 0, sizeof(float), s));
+    MOE_CUDA_TRY(cudaMemsetAsync(dw_gate, 0, (size_t)E * D * sizeof(float), s));
+    return MOE_OK;
+  }
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  auto Fp = [&](size_t off) { return reinterpret_cast<float*>(b + off); };
+  auto I = [&](size_t off) { return reinterpret_cast<int32_t*>(b + off); };
+  MOE_CUDA_TRY(cudaMemsetAsync(b, 0, kWsHeader, s));
+  MOE_CUDA_TRY(cudaMemsetAsync(b + a.counts, 0, (size_t)E * 4, s));
+  const int splits = router_k_splits(T, D, E);
+  MOE_CUDA_TRY(launch_router_gemm(x, w_gate, T, D, E, Fp(a.part), router_ld(E), splits, reinterpret_cast<int*>(b), s));
+  MOE_CUDA_TRY(launch_router_select(Fp(a.part), splits, T, router_ld(E), bias, E, k, I(a.idx), Fp(a.w), s));
+  MOE_CUDA_TRY(launch_router_aux(Fp(a.part), splits, router_ld(E), I(a.idx), x, w_gate, T, D, E, k, alpha, I(a.counts),
+                                 Fp(a.c), Fp(a.dl), loss, dw_gate, dx, s));
   return MOE_OK;
 }
 

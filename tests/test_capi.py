@@ -243,3 +243,25 @@ def test_gemm_path_query(L):
     assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD) == moe.MOE_PATH_MIXED_TILES
     assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD | moe.MOE_FLAG_PREFILL_ROW_TILES) == moe.MOE_PATH_ROW_TILES
     assert P(flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD | moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_WIDE_TILES
+
+
+def test_aux_loss_entry_validates_on_host(L):
+    """The auxiliary-loss entry checks shapes, pointers, alignment and the workspace before any
+    launch."""
+    need = L.moe_router_aux_loss_workspace_size(16, 128, 8, 2)
+    assert need > 256 and need % 256 == 0
+    assert L.moe_router_aux_loss_workspace_size(16, 96, 8, 2) == 0   # D not a multiple of 64
+    assert L.moe_router_aux_loss_workspace_size(16, 128, 8, 9) == 0  # k > E
+    args = dict(x=0x1000, wg=0x2000, bias=None, loss=0x3000, dwg=0x4000, dx=0x5000, ws=0x100000, ws_bytes=need)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return L.moe_router_aux_loss(a["x"], a["wg"], a["bias"], 16, 128, 8, 2, ctypes.c_float(0.01), a["loss"],
+                                     a["dwg"], a["dx"], a["ws"], a["ws_bytes"], None)
+
+    assert call(loss=None) == 1
+    assert call(dx=None) == 1
+    assert call(x=0x1008) == 3
+    assert call(dwg=0x4002) == 3
+    assert call(ws=0x100010) == 3
+    assert call(ws_bytes=need - 1) == 4
