@@ -370,7 +370,7 @@ moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, cons
 
 namespace {
 struct AuxWs {
-  size_t part, idx, w, counts, c, dl, total;
+  size_t part, idx, w, counts, c, dl, split, total;
 };
 AuxWs aux_ws(int T, int D, int E, int k) {
   AuxWs a;
@@ -386,6 +386,8 @@ AuxWs aux_ws(int T, int D, int E, int k) {
   a.counts = take((size_t)E * 4);
   a.c = take((size_t)T * 4);
   a.dl = take((size_t)T * E * 4);
+  const int S = T > 0 ? aux_token_splits(T, D, E) : 1;
+  a.split = take(S > 1 ? (size_t)S * E * D * 4 : 0);
   a.total = o;
   return a;
 }
@@ -423,7 +425,7 @@ moe_status_t moe_router_aux_loss(const moe_bf16_t* x, const moe_bf16_t* w_gate, 
   MOE_CUDA_TRY(launch_router_gemm(x, w_gate, T, D, E, Fp(a.part), router_ld(E), splits, reinterpret_cast<int*>(b), s));
   MOE_CUDA_TRY(launch_router_select(Fp(a.part), splits, T, router_ld(E), bias, E, k, I(a.idx), Fp(a.w), s));
   MOE_CUDA_TRY(launch_router_aux(Fp(a.part), splits, router_ld(E), I(a.idx), x, w_gate, T, D, E, k, alpha, I(a.counts),
-                                 Fp(a.c), Fp(a.dl), loss, dw_gate, dx, s));
+                                 Fp(a.c), Fp(a.dl), Fp(a.split), loss, dw_gate, dx, s));
   return MOE_OK;
 }
 

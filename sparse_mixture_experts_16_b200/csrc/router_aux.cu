@@ -15,9 +15,11 @@
 //                       full softmax, c_t, and the row dl[t, :];
 //   aux_loss_kernel     one block: sum_t c_t in a fixed tree, times alpha E / T;
 //   aux_dwg_kernel      dW_g[e, d] = sum_t dl[t, e] x[t, d], 16 experts x 256 columns per block,
-//                       tokens in order;
+//                       32-token chunks of x and dl staged in shared memory, tokens in order; when
+//                       that gives too few blocks, the tokens are split and aux_sum_splits_kernel
+//                       adds the partial sums in split order;
 //   aux_dx_kernel       dx[t, d] = sum_e dl[t, e] W_g[e, d], 16 tokens x 256 columns per block,
-//                       experts in order (dl staged in shared memory 256 experts at a time).
+//                       32-expert chunks of W_g and dl staged in shared memory, experts in order.
 #include <cfloat>
 
 #include "moe_common.cuh"
@@ -29,6 +31,8 @@ namespace {
 constexpr int kAuxThreads = 256;
 constexpr int kAuxRows = 16;   // experts (dW_g) or tokens (dx) per block
 constexpr int kAuxCols = 256;  // columns of D per block
+constexpr int kAuxChunk = 32;  // tokens (dW_g) or experts (dx) staged per step
+constexpr int kAuxMaxSplits = 16;
 
 __global__ void aux_count_kernel(const int32_t* __restrict__ idx, long long n, int E, int32_t* __restrict__ counts) {
   pdl_wait();
@@ -108,56 +112,94 @@ __global__ void __launch_bounds__(1024) aux_loss_kernel(const float* __restrict_
   pdl_trigger();
 }
 
+// dW_g over the tokens of split blockIdx.z: x [32 tokens][256 columns] and dl [32 tokens][16
+// experts] are staged in shared memory, then each thread adds 32 tokens x 16 experts for its
+// column.  With one split the block writes dW_g; otherwise partials [split][E][D].
 __global__ void __launch_bounds__(kAuxThreads) aux_dwg_kernel(const float* __restrict__ dl,
                                                               const uint16_t* __restrict__ x, int T, int D, int E,
-                                                              float* __restrict__ dwg) {
-  const int e0 = blockIdx.x * kAuxRows;
-  const int d = blockIdx.y * kAuxCols + threadIdx.x;
+                                                              int t_per, float* __restrict__ out) {
+  __shared__ __align__(16) uint16_t sx[kAuxChunk][kAuxCols];
+  __shared__ float sd[kAuxChunk][kAuxRows];
+  const int e0 = blockIdx.x * kAuxRows, d0 = blockIdx.y * kAuxCols;
+  const int d = d0 + threadIdx.x;
   const int ne = min(kAuxRows, E - e0);
+  const int tb = blockIdx.z * t_per, te = min(T, tb + t_per);
   pdl_wait();
   float acc[kAuxRows];
 #pragma unroll
   for (int j = 0; j < kAuxRows; ++j) acc[j] = 0.f;
-  if (d < D) {
-    for (int t = 0; t < T; ++t) {
-      const float xv = __uint_as_float((uint32_t)x[(size_t)t * D + d] << 16);
-      const float* drow = dl + (size_t)t * E + e0;
-#pragma unroll
-      for (int j = 0; j < kAuxRows; ++j)
-        if (j < ne) acc[j] = fmaf(__ldg(drow + j), xv, acc[j]);
+  for (int tc = tb; tc < te; tc += kAuxChunk) {
+    const int nt = min(kAuxChunk, te - tc);
+    __syncthreads();  // the previous chunk's readers are done
+    for (int i = threadIdx.x; i < kAuxChunk * (kAuxCols / 8); i += kAuxThreads) {
+      const int r = i / (kAuxCols / 8), c = (i % (kAuxCols / 8)) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (r < nt && d0 + c < D) v = *reinterpret_cast<const uint4*>(x + (size_t)(tc + r) * D + d0 + c);
+      *reinterpret_cast<uint4*>(&sx[r][c]) = v;
     }
+    for (int i = threadIdx.x; i < kAuxChunk * kAuxRows; i += kAuxThreads) {
+      const int r = i / kAuxRows, j = i % kAuxRows;
+      sd[r][j] = (r < nt && j < ne) ? dl[(size_t)(tc + r) * E + e0 + j] : 0.f;
+    }
+    __syncthreads();
+    for (int r = 0; r < nt; ++r) {
+      const float xv = __uint_as_float((uint32_t)sx[r][threadIdx.x] << 16);
+#pragma unroll
+      for (int j = 0; j < kAuxRows; ++j) acc[j] = fmaf(sd[r][j], xv, acc[j]);
+    }
+  }
+  if (d < D) {
+    float* o = out + (size_t)blockIdx.z * E * D;
 #pragma unroll
     for (int j = 0; j < kAuxRows; ++j)
-      if (j < ne) dwg[(size_t)(e0 + j) * D + d] = acc[j];
+      if (j < ne) o[(size_t)(e0 + j) * D + d] = acc[j];
   }
   pdl_trigger();
 }
 
+// out[i] = sum over splits s = 0, 1, ... of part[s][i], in that order
+__global__ void aux_sum_splits_kernel(const float* __restrict__ part, int S, long long n, float* __restrict__ out) {
+  pdl_wait();
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int sp = 0; sp < S; ++sp) acc += part[(size_t)sp * n + i];
+    out[i] = acc;
+  }
+  pdl_trigger();
+}
+
+// dx for 16 tokens x 256 columns: W_g [32 experts][256 columns] and dl [16 tokens][32 experts] are
+// staged in shared memory, experts in order.
 __global__ void __launch_bounds__(kAuxThreads) aux_dx_kernel(const float* __restrict__ dl,
                                                              const uint16_t* __restrict__ wg, int T, int D, int E,
                                                              float* __restrict__ dx) {
-  __shared__ float sdl[kAuxRows][kAuxCols];  // dl[t0 + j][ec + i]
-  const int t0 = blockIdx.x * kAuxRows;
-  const int d = blockIdx.y * kAuxCols + threadIdx.x;
+  __shared__ __align__(16) uint16_t sw[kAuxChunk][kAuxCols];
+  __shared__ float sdl[kAuxRows][kAuxChunk];
+  const int t0 = blockIdx.x * kAuxRows, d0 = blockIdx.y * kAuxCols;
+  const int d = d0 + threadIdx.x;
   const int nt = min(kAuxRows, T - t0);
   pdl_wait();
   float acc[kAuxRows];
 #pragma unroll
   for (int j = 0; j < kAuxRows; ++j) acc[j] = 0.f;
-  for (int ec = 0; ec < E; ec += kAuxCols) {
-    const int ne = min(kAuxCols, E - ec);
+  for (int ec = 0; ec < E; ec += kAuxChunk) {
+    const int ne = min(kAuxChunk, E - ec);
     __syncthreads();  // the previous chunk's readers are done
-    for (int i = threadIdx.x; i < kAuxRows * kAuxCols; i += kAuxThreads) {
-      const int j = i / kAuxCols, e = i % kAuxCols;
+    for (int i = threadIdx.x; i < kAuxChunk * (kAuxCols / 8); i += kAuxThreads) {
+      const int r = i / (kAuxCols / 8), c = (i % (kAuxCols / 8)) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (r < ne && d0 + c < D) v = *reinterpret_cast<const uint4*>(wg + (size_t)(ec + r) * D + d0 + c);
+      *reinterpret_cast<uint4*>(&sw[r][c]) = v;
+    }
+    for (int i = threadIdx.x; i < kAuxRows * kAuxChunk; i += kAuxThreads) {
+      const int j = i / kAuxChunk, e = i % kAuxChunk;
       sdl[j][e] = (j < nt && e < ne) ? dl[(size_t)(t0 + j) * E + ec + e] : 0.f;
     }
     __syncthreads();
-    if (d < D) {
-      for (int e = 0; e < ne; ++e) {
-        const float wv = __uint_as_float((uint32_t)wg[(size_t)(ec + e) * D + d] << 16);
+    for (int e = 0; e < ne; ++e) {
+      const float wv = __uint_as_float((uint32_t)sw[e][threadIdx.x] << 16);
 #pragma unroll
-        for (int j = 0; j < kAuxRows; ++j) acc[j] = fmaf(sdl[j][e], wv, acc[j]);
-      }
+      for (int j = 0; j < kAuxRows; ++j) acc[j] = fmaf(sdl[j][e], wv, acc[j]);
     }
   }
   if (d < D) {
@@ -179,9 +221,19 @@ cudaError_t launch_softmax(const float* part, int S, int T, int ld, const int32_
 
 }  // namespace
 
-cudaError_t launch_router_aux(const float* partials, int S, int ld, const int32_t* idx, const uint16_t* x,
+int aux_token_splits(int T, int D, int E) {
+  const long long tiles = (long long)((E + kAuxRows - 1) / kAuxRows) * ((D + kAuxCols - 1) / kAuxCols);
+  long long S = (2 * 148 + tiles - 1) / tiles;  // about two blocks per SM
+  const long long chunks = ((long long)T + kAuxChunk - 1) / kAuxChunk;
+  if (S > kAuxMaxSplits) S = kAuxMaxSplits;
+  if (S > chunks) S = chunks;
+  return S < 1 ? 1 : (int)S;
+}
+
+cudaError_t launch_router_aux(const float* partials, int S_router, int ld, const int32_t* idx, const uint16_t* x,
                               const uint16_t* w_gate, int T, int D, int E, int k, float alpha, int32_t* counts,
-                              float* c, float* dl, float* loss, float* dw_gate, float* dx, cudaStream_t s) {
+                              float* c, float* dl, float* split_part, float* loss, float* dw_gate, float* dx,
+                              cudaStream_t s) {
   if (T <= 0 || E <= 0 || E > 1024 || k <= 0) return cudaErrorInvalidValue;
   const long long slots = (long long)T * k;
   long long cb = (slots + 255) / 256;
@@ -189,19 +241,29 @@ cudaError_t launch_router_aux(const float* partials, int S, int ld, const int32_
   cudaError_t e = launch_pdl(aux_count_kernel, dim3((unsigned)cb), dim3(256), 0, s, idx, slots, E, counts);
   if (e != cudaSuccess) return e;
   const float scale = alpha * (float)E / (float)T;
-  if (E <= 32) e = launch_softmax<1>(partials, S, T, ld, counts, E, k, scale, c, dl, s);
-  else if (E <= 64) e = launch_softmax<2>(partials, S, T, ld, counts, E, k, scale, c, dl, s);
-  else if (E <= 128) e = launch_softmax<4>(partials, S, T, ld, counts, E, k, scale, c, dl, s);
-  else if (E <= 256) e = launch_softmax<8>(partials, S, T, ld, counts, E, k, scale, c, dl, s);
-  else if (E <= 512) e = launch_softmax<16>(partials, S, T, ld, counts, E, k, scale, c, dl, s);
-  else e = launch_softmax<32>(partials, S, T, ld, counts, E, k, scale, c, dl, s);
+  if (E <= 32) e = launch_softmax<1>(partials, S_router, T, ld, counts, E, k, scale, c, dl, s);
+  else if (E <= 64) e = launch_softmax<2>(partials, S_router, T, ld, counts, E, k, scale, c, dl, s);
+  else if (E <= 128) e = launch_softmax<4>(partials, S_router, T, ld, counts, E, k, scale, c, dl, s);
+  else if (E <= 256) e = launch_softmax<8>(partials, S_router, T, ld, counts, E, k, scale, c, dl, s);
+  else if (E <= 512) e = launch_softmax<16>(partials, S_router, T, ld, counts, E, k, scale, c, dl, s);
+  else e = launch_softmax<32>(partials, S_router, T, ld, counts, E, k, scale, c, dl, s);
   if (e != cudaSuccess) return e;
   e = launch_pdl(aux_loss_kernel, dim3(1), dim3(1024), 0, s, (const float*)c, T, scale, loss);
   if (e != cudaSuccess) return e;
   const unsigned dcols = (unsigned)((D + kAuxCols - 1) / kAuxCols);
-  e = launch_pdl(aux_dwg_kernel, dim3((unsigned)((E + kAuxRows - 1) / kAuxRows), dcols), dim3(kAuxThreads), 0, s,
-                 (const float*)dl, x, T, D, E, dw_gate);
+  const int S = aux_token_splits(T, D, E);
+  const int t_per = (T + S - 1) / S;
+  e = launch_pdl(aux_dwg_kernel, dim3((unsigned)((E + kAuxRows - 1) / kAuxRows), dcols, (unsigned)S),
+                 dim3(kAuxThreads), 0, s, (const float*)dl, x, T, D, E, t_per, S > 1 ? split_part : dw_gate);
   if (e != cudaSuccess) return e;
+  if (S > 1) {
+    const long long n = (long long)E * D;
+    long long blocks = (n + 255) / 256;
+    if (blocks > 148LL * 8) blocks = 148LL * 8;
+    e = launch_pdl(aux_sum_splits_kernel, dim3((unsigned)blocks), dim3(256), 0, s, (const float*)split_part, S, n,
+                   dw_gate);
+    if (e != cudaSuccess) return e;
+  }
   return launch_pdl(aux_dx_kernel, dim3((unsigned)((T + kAuxRows - 1) / kAuxRows), dcols), dim3(kAuxThreads), 0, s,
                     (const float*)dl, w_gate, T, D, E, dx);
 }
