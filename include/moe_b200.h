@@ -157,7 +157,9 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_idx, const float* topk_w, c
  *   offsets  [E+1]  int32      device; offsets[E] <= M
  *   row_scale [M]   fp32 or NULL (1.0): multiplies output row r (pass p_perm)
  *   max_seg:  an upper bound on any segment length (pass M if unknown).  max_seg <= 64
- *             selects the weight-streaming (decode) kernels, otherwise the tiled kernels.
+ *             selects the weight-streaming (decode) kernels, otherwise the tiled kernels with
+ *             the layer's default prefill tiling (gate_up on 128-row tiles, down on
+ *             token-wide tiles; see MOE_FLAG_PREFILL_*).
  *   gate_up  [E, 2F, D] bf16, down [E, D, F] bf16
  *   out_perm [M, D] fp32 out:   out_perm[r] = row_scale[r] * Expert_e(x_perm[r])
  *            (kept in fp32 so that y is rounded to bf16 once, in the combine)
