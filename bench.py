@@ -36,8 +36,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM bytes (read + write) of the dominant kernel (the gate_up launch) per launch, from one ncu
-# capture of the same bench command (profiles/grouped_gemm_kernels.md, profiles/stream_fp8w_kernel.md):
-# valid only while that kernel's sources are unchanged, else reported as null.
+# capture of the same bench command (the kernel summaries under profiles/): valid only while that
+# kernel's sources are unchanged, else reported as null.
 _CSRC = "sparse_mixture_experts_16_b200/csrc/"
 _TRAFFIC = {
     # kernel variant -> (its sources, their sha256, {workload: dram__bytes_read.sum + dram__bytes_write.sum})
@@ -158,6 +158,7 @@ class ClockSampler:
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         loaded = [r for r in rows if r["power"] > 300] or rows
+        capped = sum(1 for r in loaded if r["pcap"] == "Active")
         reasons = set()
         for r in loaded:
             if r["hw"] == "Active":
@@ -170,67 +171,94 @@ class ClockSampler:
                 reasons.add("sw_power_cap")
         return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["sm_max"] for r in rows),
                 "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded),
-                "power_w_max": max(r["power"] for r in rows)}
+                "samples_power_capped": capped, "power_w_max": max(r["power"] for r in rows)}
+
+
+def tensor_peak(pk: dict, clocks: dict, timed_s: float):
+    """The bf16 peak that matches the clocks of the timed region: the sustained figure (a
+    seconds-long loop at the 1 kW power cap) only for a region of >= 1 s in which the sampler saw
+    sw_power_cap under load; otherwise the burst figure (a GEMM timed alone at full clocks).
+    Returns (peak TFLOP/s, which)."""
+    if timed_s >= 1.0 and clocks.get("samples_power_capped", 0) > 0:
+        return pk["bf16_tflops_sustained"], "bf16_tflops_sustained"
+    return pk["bf16_tflops"], "bf16_tflops"
 
 
 # ---------------------------------------------------------------------------------- CPU oracle
-def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, max_experts: int = 40, weights: str = "bf16"):
+class OracleSample:
     """The fp64 oracle, as it stands, on a bounded sample of the workload's tokens (all host
-    cores; with fp8 weights the oracle's E4M3 layer on weights it quantised itself, outside the
-    timed calls).  Returns (tokens/s, cores, description)."""
-    import oracle
+    cores; with fp8 weights the oracle's E4M3 layer on weights it quantised itself).  Preparing the
+    sample (routing a prefix of the tokens, generating the weights of the experts the sample
+    needs, at most ``weight_budget`` bytes of them) happens once, outside any timed call."""
 
-    cores = host_cores()
-    x_all_rows = np.arange(w.T)
-    wg = mi.host_wg(w)
-    bias = mi.bias_f32(w)
-    # route a prefix of tokens to know which experts the sample needs (outside the timed region)
-    probe = x_all_rows[: min(w.T, 256)]
-    xp = mi.host_x(w, rows=probe)
-    idx, _ = oracle.router(xp, wg, bias, w.k)
-    chosen, experts = [], set()
-    for i, t in enumerate(probe):
-        e = set(idx[i].tolist())
-        if len(experts | e) > max_experts and chosen:
-            continue
-        experts |= e
-        chosen.append(i)
-    experts = sorted(experts)
-    gu = dict(zip(experts, mi.host_gate_up(w, experts)))
-    dn = dict(zip(experts, mi.host_down(w, experts)))
-    sgu, sdn = mi.host_shared(w)
-    if weights == "fp8":
-        q = dict(gu_q={}, gu_s={}, dn_q={}, dn_s={})
-        for e in experts:
-            q["gu_q"][e], q["gu_s"][e] = oracle.quantize_rows_fp8(gu[e])
-            q["dn_q"][e], q["dn_s"][e] = oracle.quantize_rows_fp8(dn[e])
-        shared_q = None
-        if w.Fs:
-            a, b = oracle.quantize_rows_fp8(sgu)
-            c, d = oracle.quantize_rows_fp8(sdn)
-            shared_q = dict(gu_q=a, gu_s=b, dn_q=c, dn_s=d)
-        run = lambda x: oracle.layer_fp8(x, wg, bias, w.k, q, shared_q)  # noqa: E731
-    else:
-        run = lambda x: oracle.layer(x, wg, bias, gu, dn, w.k, sgu, sdn, nthreads=cores)  # noqa: E731
-    chosen = np.array(chosen)
-    # time a growing number of tokens until the budget is reached
-    n, done, elapsed = min(len(chosen), cores), 0, 0.0
-    while True:
-        rows = chosen[np.arange(done, done + n) % len(chosen)]
-        x = xp[rows]
-        t0 = time.perf_counter()
-        run(x)
-        dt = time.perf_counter() - t0
-        done += n
-        elapsed += dt
-        if elapsed >= budget_s or done >= 64 * cores:
-            break
-        n = max(1, int(n * min(4.0, max(1.5, (budget_s - elapsed) / max(dt, 1e-3)))))
-    desc = (f"{done} tokens of workload {w.name} (full layer: routing over all E experts, top-{w.k} SwiGLU experts"
-            f"{', shared expert' if w.Fs else ''}{', E4M3 weights' if weights == 'fp8' else ''}) through the "
-            f"fp64 oracle on {cores} threads; tokens/s = "
-            f"{done} / {elapsed:.2f} s")
-    return done / elapsed, cores, desc
+    def __init__(self, w: mi.Workload, weights: str = "bf16", weight_budget: float = 3.0e9):
+        import oracle
+
+        self.w, self.weights, self.cores = w, weights, host_cores()
+        wg = mi.host_wg(w)
+        bias = mi.bias_f32(w)
+        expert_bytes = 3.0 * w.D * w.F * 2
+        max_experts = max(w.k, min(40, int(weight_budget // expert_bytes)))
+        # route a prefix of tokens to know which experts the sample needs
+        probe = np.arange(min(w.T, 256))
+        xp = mi.host_x(w, rows=probe)
+        idx, _ = oracle.router(xp, wg, bias, w.k)
+        chosen, experts = [], set()
+        for i in range(len(probe)):
+            e = set(idx[i].tolist())
+            if len(experts | e) > max_experts and chosen:
+                continue
+            experts |= e
+            chosen.append(i)
+        experts = sorted(experts)
+        gu = dict(zip(experts, mi.host_gate_up(w, experts)))
+        dn = dict(zip(experts, mi.host_down(w, experts)))
+        sgu, sdn = mi.host_shared(w)
+        if weights == "fp8":
+            q = dict(gu_q={}, gu_s={}, dn_q={}, dn_s={})
+            for e in experts:
+                q["gu_q"][e], q["gu_s"][e] = oracle.quantize_rows_fp8(gu[e])
+                q["dn_q"][e], q["dn_s"][e] = oracle.quantize_rows_fp8(dn[e])
+            shared_q = None
+            if w.Fs:
+                a, b = oracle.quantize_rows_fp8(sgu)
+                c, d = oracle.quantize_rows_fp8(sdn)
+                shared_q = dict(gu_q=a, gu_s=b, dn_q=c, dn_s=d)
+            self.run = lambda x: oracle.layer_fp8(x, wg, bias, w.k, q, shared_q)  # noqa: E731
+        else:
+            self.run = lambda x: oracle.layer(x, wg, bias, gu, dn, w.k, sgu, sdn, nthreads=self.cores)  # noqa: E731
+        self.x = xp[np.array(chosen)]
+        self.n_distinct = len(chosen)
+
+    def rate(self, budget_s: float = 12.0):
+        """Time growing batches of sampled tokens until about ``budget_s`` of oracle time has passed.
+        Returns (tokens/s, tokens timed, seconds)."""
+        n, done, elapsed = min(len(self.x), self.cores), 0, 0.0
+        while True:
+            x = self.x[np.arange(done, done + n) % len(self.x)]
+            t0 = time.perf_counter()
+            self.run(x)
+            dt = time.perf_counter() - t0
+            done += n
+            elapsed += dt
+            if elapsed >= budget_s or done >= 64 * self.cores:
+                break
+            n = max(1, int(n * min(4.0, max(1.5, (budget_s - elapsed) / max(dt, 1e-3)))))
+        return done / elapsed, done, elapsed
+
+    def describe(self, done: int, elapsed: float) -> str:
+        w = self.w
+        return (f"{done} tokens of workload {w.name} (drawn from {self.n_distinct} distinct tokens; full layer: "
+                f"routing over all E experts, top-{w.k} SwiGLU experts{', shared expert' if w.Fs else ''}"
+                f"{', E4M3 weights' if self.weights == 'fp8' else ''}) through the fp64 oracle on {self.cores} "
+                f"threads; tokens/s = {done} / {elapsed:.2f} s")
+
+
+def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, weights: str = "bf16"):
+    """(tokens/s, cores, description) of the oracle on a bounded sample of the workload."""
+    sample = OracleSample(w, weights)
+    v, done, elapsed = sample.rate(budget_s)
+    return v, sample.cores, sample.describe(done, elapsed)
 
 
 # ---------------------------------------------------------------------------------- GPU arm
@@ -370,6 +398,7 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     e2e_value = world * w.T * e2e_steps / (e2e_ms / 1e3)
 
     # ---- roofline of the dominant kernel (gate_up grouped GEMM: ~2/3 of the FLOPs / weight bytes)
+    clocks = clk.summary()
     gate_ms = statistics.mean(stage_ms[2])
     down_ms = statistics.mean(stage_ms[3])
     decode = w.T <= 64
@@ -385,13 +414,16 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
                 "peak_source": f"{pk_kind} hbm_gbs (copy bandwidth)"}
     else:
         achieved = gateup_flops(w) / (gate_ms / 1e3) / 1e12
-        peak = pk["bf16_tflops_sustained"]
+        peak, which = tensor_peak(pk, clocks, wall)
         wide = layer.gemm_path(w.T) == "wide_tiles"
         roof = {"kernel": "grouped_gemm_wide_kernel<gate_up>" if wide else "grouped_gemm_kernel<gate_up, tiled>",
                 "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name, "bf16_wide" if wide else "bf16"),
-                "peak_source": f"{pk_kind} bf16_tflops_sustained (kernel timed inside back-to-back steps)",
-                "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4)}
+                "peak_source": (f"{pk_kind} {which}: the sustained figure only for a timed region of >= 1 s "
+                                f"with power-capped samples (this one: {wall:.2f} s, "
+                                f"{clocks.get('samples_power_capped', 0)} capped samples)"),
+                "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4),
+                "frac_of_sustained_peak": round(achieved / pk["bf16_tflops_sustained"], 4)}
     layer_tflops = w.flops / (ms_per_step / 1e3) / 1e12 * world
     layer_gbs = active_weight_bytes(w, n_active, "all", args.weights) / (ms_per_step / 1e3) / 1e9
 
@@ -414,6 +446,8 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         "roofline": roof,
         "layer": {"tflops": round(layer_tflops, 1), "active_experts": n_active,
                   "active_weight_gbs": round(layer_gbs, 1),
+                  "frac_tensor": round(layer_tflops / world / tensor_peak(pk, clocks, wall)[0], 4),
+                  "frac_tensor_burst": round(layer_tflops / world / pk["bf16_tflops"], 4),
                   "frac_tensor_sustained": round(layer_tflops / world / pk["bf16_tflops_sustained"], 4),
                   "frac_hbm": round(layer_gbs / pk["hbm_gbs"], 4)},
         "stages_ms": {n: round(statistics.mean(v), 4) for n, v in
@@ -421,7 +455,7 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": w.T * w.D * 2,
                 "d2h_bytes_per_step": w.T * w.D * 2, "api": "moe_layer_forward_host (pinned host x, y)"},
         "gpu_launches": n_kernels * (len(plain_ms) + len(step_ms)),
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "wall_s_timed_region": round(wall, 3),
     }
     if rank == 0:
@@ -475,6 +509,7 @@ def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         pass
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     with ClockSampler(gpu_id) as clk, torch.cuda.stream(stream):
+        t_begin = time.perf_counter()
         for s in range(args.steps):
             evs[s][0].record(stream)
             g_fwd.replay()
@@ -482,12 +517,14 @@ def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
             g_bwd.replay()
             evs[s][2].record(stream)
         stream.synchronize()
+        wall = time.perf_counter() - t_begin
+    clocks = clk.summary()
     f_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in evs)
     b_ms = statistics.mean(b.elapsed_time(c) for _, b, c in evs)
     step_ms = f_ms + b_ms
     gemm_fwd = w.T * (6.0 * w.k * w.D * w.F + 6.0 * w.D * w.Fs)
     bwd_tflops = 2 * gemm_fwd / (b_ms / 1e3) / 1e12
-    peak = pk["bf16_tflops_sustained"]
+    peak, which = tensor_peak(pk, clocks, wall)
     n_fwd = layer.kernel_count(w.T)
     n_bwd = 9  # pad offsets, dy gather, 4 grouped GEMMs, router backward, dW_g, un-permute
     result = {
@@ -504,10 +541,11 @@ def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         "roofline": {"kernel": "backward pass (4 grouped GEMMs + 5 CUDA-core kernels)", "bound": "tensor",
                      "achieved": round(bwd_tflops, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(bwd_tflops / peak, 4), "traffic": None,
-                     "peak_source": f"{pk_kind} bf16_tflops_sustained",
+                     "peak_source": f"{pk_kind} {which} (timed region {wall:.2f} s)",
+                     "frac_of_sustained_peak": round(bwd_tflops / pk["bf16_tflops_sustained"], 4),
                      "flops": "2 x the forward's grouped-GEMM FLOPs: T(12kDF + 12DFs)"},
         "gpu_launches": (n_fwd + n_bwd) * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
     if rank == 0:
         print(json.dumps(result), flush=True)
@@ -515,26 +553,32 @@ def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
 
 
 def run_reference(args, w: mi.Workload, rank: int, world: int):
+    """The oracle on the host cores, each step a bounded sample of the workload (rank 0 only)."""
     if rank != 0:
         return
-    steps = []
-    cores = host_cores()
-    desc = None
+    sample = OracleSample(w, args.weights)
     budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    steps, done_all, secs_all = [], 0, 0.0
     for s in range(args.warmup + args.steps):
-        v, cores, desc = cpu_oracle_rate(w, budget_s=budget, weights=args.weights)
+        v, done, elapsed = sample.rate(budget)
         if s >= args.warmup:
             steps.append(v)
+            done_all += done
+            secs_all += elapsed
     value = statistics.mean(steps)
     ms = w.T / value * 1e3
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "ms_per_step_basis": (f"extrapolated: T = {w.T} tokens / the sampled rate; each timed step ran the oracle "
+                              f"on a sample of about {budget:.0f} s ({done_all} tokens in {secs_all:.1f} s over "
+                              f"{args.steps} steps), not on all T tokens"),
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; random-init weights)",
         "config": {"workload": w.name, "T": w.T, "D": w.D, "E": w.E, "k": w.k, "F": w.F, "Fs": w.Fs, "bias": w.bias,
                    "weights": "E4M3 codes + per-row fp32 scales" if args.weights == "fp8" else "bf16"},
-        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"per step: {desc}"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": sample.cores, "kind": "oracle",
+                         "sample": f"per step: {sample.describe(done_all // max(1, args.steps), secs_all / max(1, args.steps))}"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -544,7 +588,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="mixtral", choices=sorted(mi.WORKLOADS))
+    # the default is the largest single-GPU configuration: the DeepSeek-V3-shaped prefill layer
+    ap.add_argument("--workload", default="deepseek", choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--train", action="store_true",

@@ -135,8 +135,11 @@ moe_status_t moe_permute(const int32_t* topk_idx, const float* topk_w, const moe
  * GPU that loads the library until the process exits; it fits ceil(T/256) * E <= 131072
  * (e.g. T <= 32768 with E = 1024).  Larger sizes return MOE_ERR_WORKSPACE_TOO_SMALL and
  * launch nothing.
- * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
- * with that device current); make that first call before any stream capture.
+ * The array has one copy per CUDA context: each call looks up its address in the calling
+ * thread's current context (cudaGetSymbolAddress, a host-side lookup), so a caller that works
+ * in its own driver-API context, or after cudaDeviceReset, gets that context's copy.  The first
+ * call in a context loads the library's device code into it; make that first call before any
+ * stream capture.
  * All calls share the one array: calls whose kernels overlap on the GPU (e.g. on two streams
  * with no ordering between them) race and give wrong results.  Each call writes every scratch
  * entry it reads, so contents left by an earlier call do no harm.

@@ -35,6 +35,7 @@
 // own in-flight copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -526,10 +527,7 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int
   p.n_sets = n_sets;
   p.k_splits = k_splits;
   p.err = err;
-  // Fault-path test hook: with MOE_TEST_WITHHOLD_LOAD=1 the producer skips its first copies, so
-  // the consumers' bounded waits expire and the kernel reports MOE_ERR_TIMEOUT and returns.
-  const char* hold = getenv("MOE_TEST_WITHHOLD_LOAD");
-  p.withhold_first_load = (hold != nullptr && hold[0] == '1') ? 1 : 0;
+  p.withhold_first_load = (KIND != kRouter && test_withhold_this_launch()) ? 1 : 0;
   const uint32_t a_box = C::kTiled ? kBM : NT;
   const uint32_t w_box = (C::kTiled && KIND != kGateUp) ? 256 : 128;
   for (int i = 0; i < n_sets; ++i) {
@@ -560,6 +558,19 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int
 }
 
 }  // namespace
+
+bool test_withhold_this_launch() {
+  static std::atomic<int> remaining{0};
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const char* v = getenv("MOE_TEST_WITHHOLD_LOAD");
+    remaining.store(v != nullptr ? atoi(v) : 0);
+  });
+  int r = remaining.load();
+  while (r > 0 && !remaining.compare_exchange_weak(r, r - 1)) {
+  }
+  return r > 0;
+}
 
 cudaError_t launch_grouped_gemm(GemmKind kind, const GemmSetHost* sets, int n_sets, int decode_nt, int* err,
                                 cudaStream_t s) {

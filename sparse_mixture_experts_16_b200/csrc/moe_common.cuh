@@ -14,8 +14,17 @@ constexpr int kErrBadIndex = 1;  // an expert id outside [0, E)
 constexpr int kErrTimeout = 2;   // a bounded device-side wait gave up
 constexpr size_t kWsHeader = 256;
 
-// wall-time limit of every spin-wait inside a kernel
+// Wall-time limit of every spin-wait inside a kernel, measured on %globaltimer.  A context that
+// is descheduled for longer than this while a kernel waits (time-slicing with another process,
+// a debugger) can therefore report a spurious MOE_ERR_TIMEOUT.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
+
+// Fault-path test hook of the expert-GEMM launches (not of the router GEMM): the environment
+// variable MOE_TEST_WITHHOLD_LOAD=n, read once per process, makes the first n such launches
+// withhold the first stage's copies of every CTA.  The barriers are armed but the bytes never
+// arrive, so the bounded waits expire and the kernel reports MOE_ERR_TIMEOUT and returns.
+// Returns whether the launch being prepared is one of those n.
+bool test_withhold_this_launch();
 
 // ---- split-K of the weight-streaming (decode) GEMMs ---------------------------------------------
 // A decode step with fewer 128-row units than SMs splits each unit's K range.  Partial fp32

@@ -6,8 +6,6 @@
 // The only scratch the dispatch kernels need -- the per-block expert counts -- lives here in a
 // fixed file-scope device array instead of a caller workspace.  The kernels and their launcher
 // are the ones moe_permute uses; only where the scratch lives differs.
-#include <mutex>
-
 #include "moe_common.cuh"
 
 namespace {
@@ -17,36 +15,35 @@ constexpr long long kScratchInts = (long long)(kScratchBytes / 4);  // room for 
 constexpr int kTokPerBlock = 256;                                    // tokens per counting block (permute.cu)
 
 // The array's name is only a host-side stand-in in host code; its device address comes from
-// cudaGetSymbolAddress below, once per device.
+// cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_permute_scratch[kScratchBytes];
-
-std::mutex g_mu;
-void* g_scratch_addr[64];  // device address of g_permute_scratch, per device ordinal
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Device address of the scratch array on the current device (looked up on first use).
-moe_status_t scratch_for_current_device(int32_t** out) {
+// Device address of the scratch array in the calling thread's current context.  A __device__
+// array's address belongs to a CUDA context, not to a device ordinal: after cudaDeviceReset, or
+// when the caller runs in its own driver-API context on the same device, the array lives at
+// another address.  So the address is looked up on every call -- a host-side lookup in the
+// module's symbol table, with no allocation and no stream operation.  The first call in a
+// context loads the library's module into it (lazy loading), which is why that first call
+// should come before any stream capture.
+moe_status_t scratch_for_current_context(int32_t** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
     cudaGetLastError();
     return MOE_ERR_NO_DEVICE;
   }
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    int major = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
-      cudaGetLastError();
-      return MOE_ERR_NO_DEVICE;
-    }
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return MOE_ERR_CUDA;
-    }
-    g_scratch_addr[dev] = p;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
   }
-  *out = static_cast<int32_t*>(g_scratch_addr[dev]);
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  *out = static_cast<int32_t*>(p);
   return MOE_OK;
 }
 
@@ -67,7 +64,7 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_idx, const float
   const long long blocks = ((long long)T + kTokPerBlock - 1) / kTokPerBlock;
   if (blocks * E > kScratchInts) return MOE_ERR_WORKSPACE_TOO_SMALL;  // beyond the fixed scratch
   int32_t* scratch = nullptr;
-  moe_status_t st = scratch_for_current_device(&scratch);
+  moe_status_t st = scratch_for_current_context(&scratch);
   if (st != MOE_OK) return st;
   // Every entry the kernels read is written earlier in the same call, so the previous call's
   // contents need no clearing.  No error word: out-of-range ids are dropped but not reported.

@@ -480,8 +480,7 @@ cudaError_t launch_fp8(const GemmSetHost* sets, const float* const* scales, int 
     p.counters = counters;
     p.max_items = (int)std::min<size_t>(partial_bytes / item_bytes, (size_t)kMaxSplitItems);
   }
-  const char* hold = getenv("MOE_TEST_WITHHOLD_LOAD");
-  p.withhold_first_load = (hold != nullptr && hold[0] == '1') ? 1 : 0;
+  p.withhold_first_load = test_withhold_this_launch() ? 1 : 0;
   for (int i = 0; i < n_sets; ++i) {
     const GemmSetHost& st = sets[i];
     const int K = st.K;

@@ -74,3 +74,25 @@ def test_clock_summary_flags_throttling(bench):
     assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3 and out["samples_under_load"] == 2
     s.lines = ["0, 1000, 1965, 700.0, 0x8, Active, Not Active, Not Active, Not Active"]
     assert s.summary()["reasons"] == ["hw_slowdown"]
+
+
+def test_tensor_peak_matches_the_clocks_of_the_timed_region(bench):
+    pk = {"bf16_tflops": 1641.7, "bf16_tflops_sustained": 1368.0, "hbm_gbs": 6464.9}
+    capped = {"samples_power_capped": 4}
+    uncapped = {"samples_power_capped": 0}
+    # the sustained (power-capped, seconds-long) figure needs both a long region and capped samples
+    assert bench.tensor_peak(pk, capped, 2.5) == (1368.0, "bf16_tflops_sustained")
+    assert bench.tensor_peak(pk, capped, 0.2) == (1641.7, "bf16_tflops")
+    assert bench.tensor_peak(pk, uncapped, 5.0) == (1641.7, "bf16_tflops")
+    s = bench.ClockSampler("0")
+    s.lines = ["0, 1500, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active"]
+    assert s.summary()["samples_power_capped"] == 1
+
+
+def test_default_workload_is_the_largest_single_gpu_configuration(bench):
+    import moe_inputs as mi
+
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    assert 'ap.add_argument("--workload", default="deepseek"' in src
+    big = max((w for w in mi.WORKLOADS.values()), key=lambda w: w.flops)
+    assert big.name == "deepseek"

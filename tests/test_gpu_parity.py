@@ -12,8 +12,8 @@ import pytest
 import moe_inputs as mi
 import oracle
 import sparse_mixture_experts_16_b200 as moe
-from helpers import (GAP, P_ATOL, REL_RMS_TOL, bf16_np_to_f64, gap_redraw, gap_violations, rel_rms_err,
-                     scores, to_np_bf16, to_torch_bf16)
+from helpers import (GAP, P_ATOL, REL_RMS_TOL, bf16_np_to_f64, gap_redraw, gap_violations, oracle_rows_chunked,
+                     rel_rms_err, scores, segment_edge_tokens, to_np_bf16, to_torch_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -330,7 +330,6 @@ def test_layer_timed_records_six_events():
 # ----------------------------------------------------------------------------- full-size workloads
 FULL = ["mixtral", "gptoss", "gptoss_decode_T1", "gptoss_decode_T8", "gptoss_decode_T32", "gptoss_decode_T64",
         "deepseek", "deepseek_decode"]
-SAMPLE = {"mixtral": 6, "gptoss": 8, "deepseek": 4, "deepseek_decode": 4}
 
 
 # the prefill tilings other than the default mix, at full size
@@ -343,8 +342,10 @@ OTHER_TILING = [("mixtral", moe.MOE_FLAG_PREFILL_ROW_TILES), ("gptoss", moe.MOE_
                          ids=[n for n in FULL] + [f"{n}-{'wide' if f == moe.MOE_FLAG_PREFILL_WIDE_TILES else 'row'}"
                                                   for n, f in OTHER_TILING])
 def test_full_size_workload_parity(name, flags):
-    """Routing of every token bit-exact; layer outputs of sampled tokens within tolerance; with
-    flags = 0 the layer is launched exactly as the benchmark launches it."""
+    """Routing of every token and the whole dispatch (counts, offsets, perm_token, inv_perm)
+    bit-exact against the oracle; layer outputs within tolerance on every token that holds the
+    first or the last row of an expert segment (so every segment's ragged last tile is checked).
+    With flags = 0 the layer is launched exactly as the benchmark launches it."""
     import torch
 
     w = mi.WORKLOADS[name]
@@ -353,20 +354,22 @@ def test_full_size_workload_parity(name, flags):
     L = moe.MoELayer(d["wg"], d["gate_up"], d["down"], w.k, bias=d["bias"], shared_gate_up=d["shared_gate_up"],
                      shared_down=d["shared_down"], flags=flags)
     y = L(d["x"])
-    idx, _ = moe.moe_router_topk(d["x"], d["wg"], d["bias"], w.k)
+    idx, topk_w = moe.moe_router_topk(d["x"], d["wg"], d["bias"], w.k)
+    disp = moe.moe_permute(idx, topk_w, None, w.E)
     torch.cuda.synchronize()
     assert L.device_error() == 0
     x_h = mi.host_x(w, redraw=rd)
     wg_h = mi.host_wg(w)
     bias_h = mi.bias_f32(w)
-    o_idx, _ = oracle.router(x_h, wg_h, bias_h, w.k)
+    o_idx, o_p = oracle.router(x_h, wg_h, bias_h, w.k)
     assert (idx.cpu().numpy() == o_idx).all()
-    n = min(w.T, SAMPLE.get(name, w.T))
-    rows = np.random.default_rng(1).choice(w.T, size=n, replace=False)
-    used = sorted(set(o_idx[rows].reshape(-1).tolist()))
-    gu = dict(zip(used, mi.host_gate_up(w, used)))
-    dn = dict(zip(used, mi.host_down(w, used)))
-    sgu, sdn = mi.host_shared(w)
-    y_ref, _, _ = oracle.layer(x_h[rows], wg_h, bias_h, gu, dn, w.k, sgu, sdn)
+    assert np.abs(topk_w.cpu().numpy() - o_p).max() <= P_ATOL
+    counts, offsets, pt, ps, inv = oracle.permute(o_idx, w.E)
+    assert (disp["counts"].cpu().numpy() == counts).all()
+    assert (disp["offsets"].cpu().numpy() == offsets).all()
+    assert (disp["perm_token"].cpu().numpy() == pt).all()
+    assert (disp["inv_perm"].cpu().numpy() == inv).all()
+    rows = segment_edge_tokens(pt, offsets)
+    y_ref = oracle_rows_chunked(w, x_h[rows], o_idx[rows], o_p[rows])
     got = bf16_np_to_f64(to_np_bf16(y[torch.from_numpy(rows).cuda()]))
     assert rel_rms_err(got, y_ref) <= REL_RMS_TOL

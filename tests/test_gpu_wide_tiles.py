@@ -75,10 +75,15 @@ def test_wide_tiles_single_row_segments(cuda_device):
 
 def test_wide_tiles_one_overloaded_expert(cuda_device):
     """A large bias sends every token's first choice to expert 3: one segment of 600 rows (3 token
-    tiles, the last of 88 rows) and 63 short or empty ones.  On this input exact bf16 arithmetic
-    (h and y rounded to bf16, fp32 sums; emulated on the CPU) is already 2.22e-2 x RMS(y) off on
-    one token, so the bound here is normwise, like the backward tests': RMS(err) <= 5e-3 x RMS(y)
-    and max|err| <= 2e-2 x max|y|."""
+    tiles, the last of 88 rows) and 63 short or empty ones.  On this input the path's own
+    roundings (h and y rounded to bf16, fp32 sums; tests/rounding_emulation.py) already put exact
+    arithmetic 2.22e-2 x RMS(y) off the oracle on one token, so no bf16 implementation meets
+    max|err| <= 2e-2 x RMS here.  The test therefore checks (1) that the GPU is that emulation up
+    to fp32 accumulation order -- one bf16 ulp of y per element -- and (2) a normwise bound
+    against the oracle, like the backward tests': RMS(err) <= 5e-3 x RMS(y), max|err| <= 2e-2 x
+    max|y|."""
+    from rounding_emulation import emulate_layer
+
     w = W(600, 256, 64, 2, 192)
     h, d = _case(w)
     h["bias"] = np.zeros(64, np.float32)
@@ -91,11 +96,19 @@ def test_wide_tiles_one_overloaded_expert(cuda_device):
     if gap_violations(scores(w, h["x"], h["wg"], h["bias"]), w.k).any():
         pytest.skip("seeded inputs violate the gap under the changed bias")
     y_ref = _oracle(h, w.k)
-    for tiling in (ROW, WIDE):
+    y_emu = emulate_layer(h["x"], h["wg"], h["bias"], h["gate_up"], h["down"], w.k)
+    rms = np.sqrt(np.mean(y_ref * y_ref))
+    assert rel_rms_err(y_emu, y_ref) > REL_RMS_TOL  # why this case is bounded normwise
+    for tiling in (ROW, WIDE, 0):
         L = _layer(d, w.k, tiling | PREFILL)
-        err = bf16_np_to_f64(to_np_bf16(L(d["x"]))) - y_ref
+        y = bf16_np_to_f64(to_np_bf16(L(d["x"])))
         assert L.device_error() == 0
-        assert np.sqrt(np.mean(err * err)) <= 5e-3 * np.sqrt(np.mean(y_ref * y_ref))
+        # (1) the emulated rounding points: within one bf16 ulp of y (2^-7 relative) per element
+        assert (np.abs(y - y_emu) <= 2.0 ** -7 * np.abs(y_emu) + 1e-4 * rms).all()
+        assert np.sqrt(np.mean((y - y_emu) ** 2)) <= 1e-3 * rms
+        # (2) normwise against the oracle
+        err = y - y_ref
+        assert np.sqrt(np.mean(err * err)) <= 5e-3 * rms
         assert np.abs(err).max() <= 2e-2 * np.abs(y_ref).max()
 
 

@@ -371,6 +371,53 @@ def test_fp8_ffn_equals_bf16_ffn_on_exactly_representable_weights():
     np.testing.assert_array_equal(oracle.expert_ffn_fp8(x, gq, gs, dq, ds), oracle.expert_ffn(x, gu, dn))
 
 
+def _e4m3_exact_bf16(rng, shape, exp):
+    """bf16 weights that are E4M3 values times 2^exp, every row reaching 448 * 2^exp, so that the
+    per-row quantiser reproduces them exactly (scale = 2^exp, codes = the drawn codes)."""
+    codes = rng.integers(0, 0x7E, shape).astype(np.uint8)
+    codes |= rng.integers(0, 2, shape).astype(np.uint8) << 7
+    codes[..., 0] = 0x7E
+    vals = np.vectorize(oracle.e4m3_value)(codes) * 2.0 ** exp
+    w = _bf16(vals)
+    assert (f64(w) == vals).all()
+    return w
+
+
+@pytest.mark.parametrize("k", [2, 3])
+def test_fp8_layer_equals_bf16_layer_on_exactly_representable_weights(k):
+    """The E4M3 layer (routing, FP8 experts weighted by p, shared expert at weight 1) on weights the
+    quantiser reproduces exactly is the bf16 layer: a p taken from the wrong slot, a shared expert
+    weighted by p, or a dropped term fails this (keryc.com, "Resultados practicos": per-expert
+    quantisation leaves the layer's definition unchanged; gotburnout.io glossary "MoE", section 2)."""
+    rng = np.random.default_rng(22 + k)
+    T, D, E, F, Fs = 9, 32, 6, 16, 16
+    gu = _e4m3_exact_bf16(rng, (E, 2 * F, D), -12)
+    dn = _e4m3_exact_bf16(rng, (E, D, F), -11)
+    sgu = _e4m3_exact_bf16(rng, (2 * Fs, D), -12)
+    sdn = _e4m3_exact_bf16(rng, (D, Fs), -11)
+    x = _bf16(rng.standard_normal((T, D)))
+    wg = _bf16(rng.standard_normal((E, D)) * 0.3)
+    bias = (rng.standard_normal(E) * 0.2).astype(np.float32)
+    q = dict(gu_q={}, gu_s={}, dn_q={}, dn_s={})
+    for e in range(E):
+        q["gu_q"][e], q["gu_s"][e] = oracle.quantize_rows_fp8(gu[e])
+        q["dn_q"][e], q["dn_s"][e] = oracle.quantize_rows_fp8(dn[e])
+    a, b = oracle.quantize_rows_fp8(sgu)
+    c, d = oracle.quantize_rows_fp8(sdn)
+    shared_q = dict(gu_q=a, gu_s=b, dn_q=c, dn_s=d)
+    y8, idx8, p8 = oracle.layer_fp8(x, wg, bias, k, q, shared_q)
+    y, idx, p = oracle.layer(x, wg, bias, gu, dn, k, sgu, sdn)
+    np.testing.assert_array_equal(idx8, idx)
+    np.testing.assert_array_equal(p8, p)
+    # the same terms in the same order up to the summation order of the C and numpy loops
+    assert np.abs(y8 - y).max() <= 1e-13 * np.abs(y).max()
+    # the weights in the p vector differ from one another, so a p from the wrong slot would show
+    assert (np.abs(np.diff(p, axis=1)) > 1e-3).any()
+    # and the shared expert's term is large enough that weighting it by p would show
+    ys, _, _ = oracle.layer(x, wg, bias, gu, dn, k)
+    assert np.abs(y - ys).max() > 1e-3 * np.abs(y).max()
+
+
 # ----------------------------------------------------------------------------- backward pass
 def _bwd_problem(seed=0, T=6, D=16, E=6, k=2, F=8, Fs=8, bias=True):
     """A small fp64 problem whose top-k choices are separated by at least 0.05 in score, so that the
@@ -500,3 +547,22 @@ def test_aux_loss_gradient_matches_finite_differences():
             lm = oracle.router_aux_loss(q["x"], q["wg"], P["bias"], k, 0.1)[0]
             assert float(np.sum(g * V)) == pytest.approx((lp - lm) / (2 * eps), rel=1e-6, abs=1e-11), (seed, name)
         assert np.abs(dwg.sum(axis=0)).max() < 1e-12 * max(1.0, np.abs(dwg).max())
+
+
+# ----------------------------------------------------------------------------- full-size sampling helpers
+def test_chunked_oracle_rows_equal_the_layer():
+    """The sampled full-size check builds y from oracle expert FFNs, experts generated in chunks;
+    on a small workload that must be the oracle's layer (up to summation order)."""
+    from helpers import oracle_rows_chunked, segment_edge_tokens
+
+    w = mi.Workload("chunk", T=40, D=64, E=6, k=3, F=64, Fs=64, bias="normal:0.5")
+    h = mi.host_inputs(w)
+    y, idx, p = oracle.layer(h["x"], h["wg"], h["bias"], h["gate_up"], h["down"], w.k, h["shared_gate_up"],
+                             h["shared_down"])
+    counts, offsets, pt, _, _ = oracle.permute(idx, w.E)
+    rows = segment_edge_tokens(pt, offsets)
+    for e in range(w.E):  # every non-empty segment's first and last token is among the rows
+        if counts[e]:
+            assert pt[offsets[e]] in rows and pt[offsets[e + 1] - 1] in rows
+    got = oracle_rows_chunked(w, h["x"][rows], idx[rows], p[rows], chunk=4)
+    assert np.abs(got - y[rows]).max() <= 1e-12 * np.abs(y).max()

@@ -4,8 +4,9 @@ Such callers (whose device memory is owned by an engine's own pools, or a plugin
 to its host program's allocator) cannot hand moe_permute a workspace; this entry point keeps its
 scratch in a fixed array inside the library instead.  Its outputs must equal moe_permute's bit
 for bit (integer and copy work), on two calls in a row -- the second call sees the array as the
-first call left it.  This file runs last so that a stop-at-first-failure run has already run
-every other test; it also passes on its own in a fresh process.
+first call left it -- and equal the oracle's stable counting sort, so that a mistake the two GPU
+entry points share cannot pass.  This file runs last so that a stop-at-first-failure run has
+already run every other test; it also passes on its own in a fresh process.
 """
 import ctypes
 
@@ -13,6 +14,7 @@ import numpy as np
 import pytest
 
 import moe_inputs as mi
+import oracle
 import sparse_mixture_experts_16_b200 as moe
 
 pytestmark = pytest.mark.gpu
@@ -57,11 +59,31 @@ def _noalloc(L, idx, wts, x, E):
     return out
 
 
+def _check_against_oracle(got, idx, wts, x, E):
+    """counts, offsets, perm_token, inv_perm bit-exact against the oracle's stable counting sort;
+    p_perm and x_perm are the routed weight and token row of each permuted slot."""
+    import torch
+
+    idx_h, w_h = idx.cpu().numpy(), wts.cpu().numpy()
+    counts, offsets, pt, ps, inv = oracle.permute(idx_h, E)
+    assert (got["counts"].cpu().numpy() == counts).all()
+    assert (got["offsets"].cpu().numpy() == offsets).all()
+    assert (got["perm_token"].cpu().numpy() == pt).all()
+    assert (got["inv_perm"].cpu().numpy() == inv).all()
+    assert (got["p_perm"].cpu().numpy() == w_h[pt, ps]).all()
+    x_h = x.view(torch.int16).cpu().numpy()
+    assert (got["x_perm"].view(torch.int16).cpu().numpy() == x_h[pt]).all()
+
+
+# (T, E, k, D, seed): multi-block counting (T > 256) first, filling more of the shared array than
+# the calls after it read; then the one-kernel dispatch of T <= 256 and a single token
+CASES = [(3000, 64, 4, 128, 1), (777, 33, 3, 192, 2), (200, 16, 4, 128, 3), (1, 8, 2, 64, 4)]
+
+
 def test_noalloc_permute_matches_workspace_permute_on_two_calls_in_a_row(L):
     import torch
 
-    # the first call fills more of the shared array than the second one reads
-    for (T, E, k, D, seed) in [(3000, 64, 4, 128, 1), (777, 33, 3, 192, 2)]:
+    for (T, E, k, D, seed) in CASES:
         idx, wts, x = _inputs(T, E, k, D, seed)
         ref = moe.moe_permute(idx, wts, x, E)
         got = _noalloc(L, idx, wts, x, E)
@@ -69,6 +91,16 @@ def test_noalloc_permute_matches_workspace_permute_on_two_calls_in_a_row(L):
         for name in ("counts", "offsets", "perm_token", "inv_perm", "p_perm"):
             assert torch.equal(got[name], ref[name]), name
         assert torch.equal(got["x_perm"].view(torch.int16), ref["x_perm"].view(torch.int16))
+
+
+def test_noalloc_permute_matches_the_oracle(L):
+    import torch
+
+    for (T, E, k, D, seed) in CASES:
+        idx, wts, x = _inputs(T, E, k, D, seed)
+        got = _noalloc(L, idx, wts, x, E)
+        torch.cuda.synchronize()
+        _check_against_oracle(got, idx, wts, x, E)
 
 
 def test_noalloc_permute_rejects_sizes_beyond_its_fixed_scratch(L):
