@@ -46,6 +46,8 @@ _TRAFFIC = {
              {"mixtral": 1.947595e9 + 0.226813e9, "deepseek_decode": 5.876610e9 + 0.003743e9}),
     "bf16_wide": ((_CSRC + "grouped_gemm_wide_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
                   "", {}),
+    "bf16_pair": ((_CSRC + "grouped_gemm_pair_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
+                  "", {}),
     "fp8": ((_CSRC + "stream_fp8w_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
             "90184c605698454c7e2560af3fdb691544ae668cddf7910ea71752c9dc8e3252",
             {"deepseek_decode": 2.942079e9 + 0.003725e9, "gptoss_decode_T64": 0.556999e9 + 0.004705e9}),
@@ -265,7 +267,8 @@ def cpu_oracle_rate(w: mi.Workload, budget_s: float = 12.0, weights: str = "bf16
 def tiling_flag(tiling: str) -> int:
     import sparse_mixture_experts_16_b200 as moe
 
-    return {"auto": 0, "row": moe.MOE_FLAG_PREFILL_ROW_TILES, "wide": moe.MOE_FLAG_PREFILL_WIDE_TILES}[tiling]
+    return {"auto": 0, "row": moe.MOE_FLAG_PREFILL_ROW_TILES, "wide": moe.MOE_FLAG_PREFILL_WIDE_TILES,
+            "pair": moe.MOE_FLAG_PREFILL_PAIR_TILES}[tiling]
 
 
 def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
@@ -415,10 +418,11 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     else:
         achieved = gateup_flops(w) / (gate_ms / 1e3) / 1e12
         peak, which = tensor_peak(pk, clocks, wall)
-        wide = layer.gemm_path(w.T) == "wide_tiles"
-        roof = {"kernel": "grouped_gemm_wide_kernel<gate_up>" if wide else "grouped_gemm_kernel<gate_up, tiled>",
+        gu_kernel = {"wide_tiles": "grouped_gemm_wide_kernel<gate_up>", "pair_tiles": "grouped_gemm_pair_kernel<gate_up>"}
+        path = layer.gemm_path(w.T)
+        roof = {"kernel": gu_kernel.get(path, "grouped_gemm_kernel<gate_up, tiled>"),
                 "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name, "bf16_wide" if wide else "bf16"),
+                "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name, {"wide_tiles": "bf16_wide", "pair_tiles": "bf16_pair"}.get(path, "bf16")),
                 "peak_source": (f"{pk_kind} {which}: the sustained figure only for a timed region of >= 1 s "
                                 f"with power-capped samples (this one: {wall:.2f} s, "
                                 f"{clocks.get('samples_power_capped', 0)} capped samples)"),
@@ -594,9 +598,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--train", action="store_true",
                     help="time a training step (forward saving g|u + backward) instead of the forward")
-    ap.add_argument("--tiling", default="auto", choices=["auto", "row", "wide"],
-                    help="prefill tiling of the expert GEMMs (bf16): the layer's default (gate_up on 128-row "
-                         "tiles, down on token-wide tiles), 128-row tiles for both, or token-wide tiles for both")
+    ap.add_argument("--tiling", default="auto", choices=["auto", "row", "wide", "pair"],
+                    help="prefill tiling of the expert GEMMs (bf16): the layer's default, 128-row tiles for both, "
+                         "token-wide tiles for both, or token-wide tiles on CTA pairs for both")
     ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
                     help="expert weight format; fp8 (E4M3, per-row scales) runs the decode kernels, T <= 64")
     args = ap.parse_args()

@@ -160,9 +160,10 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_idx, const float* topk_w, c
  *   offsets  [E+1]  int32      device; offsets[E] <= M
  *   row_scale [M]   fp32 or NULL (1.0): multiplies output row r (pass p_perm)
  *   max_seg:  an upper bound on any segment length (pass M if unknown).  max_seg <= 64
- *             selects the weight-streaming (decode) kernels, otherwise the tiled kernels with
- *             the layer's default prefill tiling (gate_up on 128-row tiles, down on
- *             token-wide tiles; see MOE_FLAG_PREFILL_*).
+ *             selects the weight-streaming (decode) kernels, otherwise the tiled kernels.
+ *   flags:    0 for the layer's default prefill tiling, or one of MOE_FLAG_PREFILL_ROW_TILES /
+ *             _WIDE_TILES / _PAIR_TILES (defined with moe_layer_desc_t below); ignored when the
+ *             streaming kernels run.  Any other bit is MOE_ERR_INVALID_ARG.
  *   gate_up  [E, 2F, D] bf16, down [E, D, F] bf16
  *   out_perm [M, D] fp32 out:   out_perm[r] = row_scale[r] * Expert_e(x_perm[r])
  *            (kept in fp32 so that y is rounded to bf16 once, in the combine)
@@ -171,7 +172,7 @@ moe_status_t moe_permute_noalloc(const int32_t* topk_idx, const float* topk_w, c
  * ---------------------------------------------------------------------------------------- */
 size_t moe_grouped_swiglu_ffn_workspace_size(int M, int F);
 moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* offsets,
-                                    const float* row_scale, int M, int max_seg, int E, int D, int F,
+                                    const float* row_scale, int M, int max_seg, int flags, int E, int D, int F,
                                     const moe_bf16_t* gate_up, const moe_bf16_t* down,
                                     float* out_perm, void* ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -198,15 +199,19 @@ moe_status_t moe_combine(const float* out_perm, const int32_t* inv_perm, const f
  * and the SwiGLU inputs g | u of the gate_up GEMMs, bf16).  Uses the tiled kernels at any T;
  * bf16 weights only. */
 #define MOE_FLAG_SAVE_FOR_BACKWARD 4
-/* Prefill tiling of the expert GEMMs (at most one of the two; neither with FORCE_DECODE):
+/* Prefill tiling of the expert GEMMs (at most one of the three; none with FORCE_DECODE):
  *  ROW_TILES  both GEMMs on 128 permuted rows x 256 output columns per tile (tokens are the
  *             MMA's M);
  *  WIDE_TILES both on 128 weight rows x up to 256 rows of one expert segment (tokens are N, so a
- *             segment's last tile is padded to a multiple of 16 rows instead of 128).
- * Without either, gate_up runs ROW_TILES and down WIDE_TILES.  All give the same routing;
+ *             segment's last tile is padded to a multiple of 16 rows instead of 128);
+ *  PAIR_TILES both on the WIDE orientation computed by a cluster of two CTAs: 256 weight rows x
+ *             up to 256 tokens per tcgen05.mma.cta_group::2, each CTA loading its own half of both
+ *             operands (no multicast).
+ * Without any, gate_up runs ROW_TILES and down WIDE_TILES.  All give the same routing;
  * outputs agree within fp32 rounding order. */
 #define MOE_FLAG_PREFILL_ROW_TILES 8
 #define MOE_FLAG_PREFILL_WIDE_TILES 16
+#define MOE_FLAG_PREFILL_PAIR_TILES 32
 
 #define MOE_WEIGHTS_BF16 0     /* gate_up / down (and shared_*) hold bf16 weights            */
 #define MOE_WEIGHTS_FP8_E4M3 1 /* *_fp8 hold E4M3 codes with one fp32 scale per weight row  */
@@ -275,12 +280,13 @@ int moe_layer_kernel_count(const moe_layer_desc_t* desc);
 
 /* Which expert-GEMM kernels moe_layer_forward runs for this descriptor (host-only query; -1 if
  * the descriptor is invalid): the weight-streaming decode kernels (bf16 or E4M3 weights), or the
- * prefill tilings of MOE_FLAG_PREFILL_ROW_TILES / MOE_FLAG_PREFILL_WIDE_TILES. */
+ * prefill tilings of MOE_FLAG_PREFILL_ROW_TILES / _WIDE_TILES / _PAIR_TILES. */
 #define MOE_PATH_STREAMING 0
 #define MOE_PATH_FP8_STREAMING 1
 #define MOE_PATH_ROW_TILES 2
 #define MOE_PATH_WIDE_TILES 3
 #define MOE_PATH_MIXED_TILES 4 /* gate_up on 128-row tiles, down on token-wide tiles */
+#define MOE_PATH_PAIR_TILES 5  /* both on token-wide tiles of CTA pairs */
 int moe_layer_gemm_path(const moe_layer_desc_t* desc);
 
 /* ----------------------------------------------------------------------------------------

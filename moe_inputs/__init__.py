@@ -75,6 +75,10 @@ WORKLOADS = {
 }
 for _t in (1, 8, 32, 64):
     WORKLOADS[f"gptoss_decode_T{_t}"] = replace(WORKLOADS["gptoss"], name=f"gptoss_decode_T{_t}", T=_t)
+# the DeepSeek-V3-shaped layer cut to 32 experts and 1024 tokens: the same per-expert GEMM shapes
+# (~256 rows per expert segment, D = 7168, F = Fs = 2048) with 2.9 GB of weights instead of 22.6 GB,
+# small enough for kernel profiling captures
+WORKLOADS["deepseek_e32"] = replace(WORKLOADS["deepseek"], name="deepseek_e32", T=1024, E=32)
 
 
 def build(force: bool = False) -> str:

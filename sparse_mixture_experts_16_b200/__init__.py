@@ -20,7 +20,9 @@ MOE_FLAG_FORCE_DECODE = 2
 MOE_FLAG_SAVE_FOR_BACKWARD = 4
 MOE_FLAG_PREFILL_ROW_TILES = 8
 MOE_FLAG_PREFILL_WIDE_TILES = 16
+MOE_FLAG_PREFILL_PAIR_TILES = 32
 MOE_PATH_STREAMING, MOE_PATH_FP8_STREAMING, MOE_PATH_ROW_TILES, MOE_PATH_WIDE_TILES, MOE_PATH_MIXED_TILES = 0, 1, 2, 3, 4
+MOE_PATH_PAIR_TILES = 5
 MOE_WEIGHTS_BF16 = 0
 MOE_WEIGHTS_FP8_E4M3 = 1
 
@@ -89,7 +91,7 @@ def lib():
             "moe_permute": ([P, P, P, I, I, I, I, P, P, P, P, P, P, P, Z, P], I),
             "moe_permute_noalloc": ([P, P, P, I, I, I, I, P, P, P, P, P, P, P], I),
             "moe_grouped_swiglu_ffn_workspace_size": ([I, I], Z),
-            "moe_grouped_swiglu_ffn": ([P, P, P, I, I, I, I, I, P, P, P, P, Z, P], I),
+            "moe_grouped_swiglu_ffn": ([P, P, P, I, I, I, I, I, I, P, P, P, P, Z, P], I),
             "moe_combine": ([P, P, P, I, I, I, P, P], I),
             "moe_layer_workspace_size": ([ctypes.POINTER(LayerDesc)], Z),
             "moe_layer_forward": ([ctypes.POINTER(LayerDesc), P, P, P, Z, P], I),
@@ -254,8 +256,9 @@ def moe_permute_noalloc(topk_idx, topk_w, x, E, out=None, stream=None):
 
 
 def moe_grouped_swiglu_ffn(x_perm, offsets, row_scale, gate_up, down, max_seg=None, out_perm=None, ws=None,
-                           stream=None):
-    """out_perm[r] = row_scale[r] * Expert_e(x_perm[r]) for the rows r of each expert segment e."""
+                           stream=None, tiling=0):
+    """out_perm[r] = row_scale[r] * Expert_e(x_perm[r]) for the rows r of each expert segment e.
+    ``tiling``: 0 (the layer's default) or one MOE_FLAG_PREFILL_* flag."""
     import torch
 
     M, D = x_perm.shape
@@ -268,7 +271,7 @@ def moe_grouped_swiglu_ffn(x_perm, offsets, row_scale, gate_up, down, max_seg=No
     if ws is None or ws.numel() < need:
         ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=x_perm.device)
     _check(lib().moe_grouped_swiglu_ffn(x_perm.data_ptr(), offsets.data_ptr(), _ptr(row_scale), M,
-                                        M if max_seg is None else max_seg, E, D, F, gate_up.data_ptr(),
+                                        M if max_seg is None else max_seg, tiling, E, D, F, gate_up.data_ptr(),
                                         down.data_ptr(), out_perm.data_ptr(), ws.data_ptr(), ws.numel(),
                                         _stream(stream)), "moe_grouped_swiglu_ffn")
     return out_perm, ws
@@ -337,12 +340,13 @@ class MoELayer:
 
     def gemm_path(self, T: int) -> str:
         """The expert-GEMM kernels a forward over T tokens runs: "streaming", "fp8_streaming",
-        "row_tiles", "wide_tiles" or "mixed_tiles" (gate_up on row tiles, down on wide tiles)."""
+        "row_tiles", "wide_tiles", "mixed_tiles" (gate_up on row tiles, down on wide tiles) or
+        "pair_tiles" (both on token-wide tiles of CTA pairs)."""
         d = self.desc(T)
         code = lib().moe_layer_gemm_path(ctypes.byref(d))
         if code < 0:
             raise MoeError(1, "moe_layer_gemm_path")
-        return ("streaming", "fp8_streaming", "row_tiles", "wide_tiles", "mixed_tiles")[code]
+        return ("streaming", "fp8_streaming", "row_tiles", "wide_tiles", "mixed_tiles", "pair_tiles")[code]
 
     def forward(self, x, y=None, stream=None):
         import torch

@@ -14,4 +14,8 @@ namespace moe {
 // of 64, down's n_out (D) a multiple of 32.
 cudaError_t launch_grouped_gemm_wide(GemmKind kind, const GemmSetHost* sets, int n_sets, int* err, cudaStream_t s);
 
+// The same products on token-wide tiles computed by clusters of two CTAs (one M = 256 MMA per
+// tile, each CTA loading half of each operand): grouped_gemm_pair_sm100.cu.  Same contract.
+cudaError_t launch_grouped_gemm_pair(GemmKind kind, const GemmSetHost* sets, int n_sets, int* err, cudaStream_t s);
+
 }  // namespace moe

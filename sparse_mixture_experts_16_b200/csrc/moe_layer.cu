@@ -49,16 +49,26 @@ bool use_decode(const moe_layer_desc_t& d) {
 
 int decode_tile(int max_seg) { return ((max_seg + 15) / 16) * 16; }
 
-// Prefill tiling, as bits: 1 = gate_up on token-wide tiles (weights as the MMA's M, up to 256 rows
-// of one segment as N), 2 = down on token-wide tiles; clear bits mean 128-row tiles.  Token-wide
-// tiles pad a segment's last tile to 16 rows instead of 128, but their gate_up (SwiGLU epilogue
-// through a shared-memory transpose) measured slower than the 128-row one, while their down
-// measured faster; the default mixes the two.
-constexpr int kWideGateUp = 1, kWideDown = 2;
-int wide_tiles(int flags) {
-  if (flags & MOE_FLAG_PREFILL_WIDE_TILES) return kWideGateUp | kWideDown;
-  if (flags & MOE_FLAG_PREFILL_ROW_TILES) return 0;
-  return kWideDown;
+// Prefill tiling: which kernel runs each expert GEMM.  Row tiles: 128 permuted rows x 256 output
+// columns (tokens are the MMA's M).  Wide tiles: 128 weight rows x up to 256 rows of one expert
+// segment (tokens are N, so a segment's last tile pads to 16 rows instead of 128).  Pair tiles: the
+// wide orientation on a cluster of two CTAs, 256 weight rows x up to 256 tokens per MMA (each SM
+// loads a third fewer operand bytes per FLOP).  The default mixes the measured best per GEMM.
+enum TileKind { kRowT = 0, kWideT = 1, kPairT = 2 };
+struct Tiling {
+  int gu, dn;
+};
+Tiling prefill_tiling(int flags) {
+  if (flags & MOE_FLAG_PREFILL_WIDE_TILES) return {kWideT, kWideT};
+  if (flags & MOE_FLAG_PREFILL_ROW_TILES) return {kRowT, kRowT};
+  if (flags & MOE_FLAG_PREFILL_PAIR_TILES) return {kPairT, kPairT};
+  return {kRowT, kWideT};
+}
+
+cudaError_t launch_tiled(TileKind t, GemmKind kind, const GemmSetHost* sets, int n_sets, int* err, cudaStream_t s) {
+  if (t == kPairT) return launch_grouped_gemm_pair(kind, sets, n_sets, err, s);
+  if (t == kWideT) return launch_grouped_gemm_wide(kind, sets, n_sets, err, s);
+  return launch_grouped_gemm(kind, sets, n_sets, 0, err, s);
 }
 
 struct LayerWs {
@@ -137,10 +147,10 @@ moe_status_t validate_desc(const moe_layer_desc_t* d) {
     return MOE_ERR_INVALID_ARG;
   }
   if ((d->flags & ~(MOE_FLAG_FORCE_PREFILL | MOE_FLAG_FORCE_DECODE | MOE_FLAG_SAVE_FOR_BACKWARD |
-                    MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES)) != 0)
+                    MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES | MOE_FLAG_PREFILL_PAIR_TILES)) != 0)
     return MOE_ERR_INVALID_ARG;
-  const int tiling = d->flags & (MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES);
-  if (tiling == (MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES)) return MOE_ERR_INVALID_ARG;
+  const int tiling = d->flags & (MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES | MOE_FLAG_PREFILL_PAIR_TILES);
+  if (tiling & (tiling - 1)) return MOE_ERR_INVALID_ARG;  // at most one tiling flag
   if (tiling && ((d->flags & MOE_FLAG_FORCE_DECODE) || d->weight_format != MOE_WEIGHTS_BF16)) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && (d->flags & MOE_FLAG_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
   if ((d->flags & MOE_FLAG_FORCE_PREFILL) && (d->flags & MOE_FLAG_FORCE_DECODE)) return MOE_ERR_INVALID_ARG;
@@ -164,33 +174,40 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
                      int F, const uint16_t* gate_up, const uint16_t* down, uint16_t* h, float* out_perm,
                      // optional shared expert over x[T, D]
                      const uint16_t* x, int T, int Fs, const uint16_t* sgu, const uint16_t* sdn, uint16_t* h_sh,
-                     float* out_sh, int decode_nt, int wide, int* err, cudaStream_t s, cudaEvent_t ev_mid,
-                     unsigned ev_flags, uint16_t* save_gu = nullptr, uint16_t* save_gu_sh = nullptr) {
-  GemmSetHost g[2];
-  memset(g, 0, sizeof(g));
-  g[0].K = D, g[0].a = x_perm, g[0].a_rows = M, g[0].w = gate_up, g[0].n_groups = E, g[0].offsets = offsets;
-  g[0].n_out = F, g[0].out = h, g[0].save_gu = save_gu;
+                     float* out_sh, int decode_nt, Tiling tiling, int* err, cudaStream_t s, cudaEvent_t ev_mid,
+                     unsigned ev_flags, uint16_t* save_gu = nullptr, uint16_t* save_gu_sh = nullptr,
+                     const int32_t* perm_token = nullptr) {
+  // perm_token (streaming only): the gate_up launch gathers its token rows from x by the
+  // permutation (x_perm is not read) and prefetches the active experts' down weights into L2
+  GemmSetHost g[2] = {};
+  const bool gather = decode_nt > 0 && perm_token != nullptr;
+  g[0].K = D, g[0].a = gather ? x : x_perm, g[0].a_rows = gather ? T : M, g[0].w = gate_up, g[0].n_groups = E;
+  g[0].offsets = offsets, g[0].n_out = F, g[0].out = h, g[0].save_gu = save_gu;
+  if (gather) {
+    g[0].gather_rows = perm_token, g[0].gather_src = x;
+    g[0].prefetch_w = down, g[0].prefetch_bytes = (long long)D * F * 2;
+  }
   int n_sets = 1;
   if (Fs > 0) {
     g[1].K = D, g[1].a = x, g[1].a_rows = T, g[1].w = sgu, g[1].n_groups = 1, g[1].m_rows = T;
     g[1].n_out = Fs, g[1].out = h_sh, g[1].save_gu = save_gu_sh;
+    if (gather) g[1].prefetch_w = sdn, g[1].prefetch_bytes = (long long)D * Fs * 2;
     n_sets = 2;
   }
-  if (decode_nt == 0 && (wide & kWideGateUp))
-    MOE_CUDA_TRY(launch_grouped_gemm_wide(kGateUp, g, n_sets, err, s));
+  if (decode_nt == 0)
+    MOE_CUDA_TRY(launch_tiled((TileKind)tiling.gu, kGateUp, g, n_sets, err, s));
   else
     MOE_CUDA_TRY(launch_grouped_gemm(kGateUp, g, n_sets, decode_nt, err, s));
   if (ev_mid) MOE_CUDA_TRY(cudaEventRecordWithFlags(ev_mid, s, ev_flags));
-  GemmSetHost dn[2];
-  memset(dn, 0, sizeof(dn));
+  GemmSetHost dn[2] = {};
   dn[0].K = F, dn[0].a = h, dn[0].a_rows = M, dn[0].w = down, dn[0].n_groups = E, dn[0].offsets = offsets;
   dn[0].n_out = D, dn[0].out = out_perm, dn[0].row_scale = row_scale;
   if (Fs > 0) {
     dn[1].K = Fs, dn[1].a = h_sh, dn[1].a_rows = T, dn[1].w = sdn, dn[1].n_groups = 1, dn[1].m_rows = T;
     dn[1].n_out = D, dn[1].out = out_sh;
   }
-  if (decode_nt == 0 && (wide & kWideDown))
-    MOE_CUDA_TRY(launch_grouped_gemm_wide(kDown, dn, n_sets, err, s));
+  if (decode_nt == 0)
+    MOE_CUDA_TRY(launch_tiled((TileKind)tiling.dn, kDown, dn, n_sets, err, s));
   else
     MOE_CUDA_TRY(launch_grouped_gemm(kDown, dn, n_sets, decode_nt, err, s));
   return MOE_OK;
@@ -228,18 +245,33 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
   // a fresh error word and zeroed split-K counters (they follow the header) for this forward
   MOE_CUDA_TRY(cudaMemsetAsync(err, 0, w.split_counters + kSplitCounterBytes, s));
   const int splits = router_k_splits(T, D, E);
-  MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s));
-  MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
-                                    Fp(w.topk_w), s));
-  if (ev) MOE_CUDA_TRY(record(ev[1]));
   const bool fp8 = d->weight_format == MOE_WEIGHTS_FP8_E4M3;
-  // dispatch + gather (one kernel for T <= 256); the FP8 path gathers f16 rows and, for the
-  // shared expert, an f16 copy of x
-  MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), x, T, D, E, k, I(w.counts), I(w.offsets), I(w.perm_token),
-                              I(w.inv_perm), Fp(w.p_perm), H(w.x_perm), fp8, (fp8 && Fs > 0) ? H(w.x16) : nullptr,
-                              I(w.scratch), err, s, nullptr));
-  if (ev) MOE_CUDA_TRY(record(ev[2]));
   const int nt = use_decode(*d) ? decode_tile(T) : 0;
+  // bf16 decode: the router GEMM's last CTA also selects and dispatches (no top-k or dispatch
+  // launch), and the gate_up launch gathers token rows from x itself (no x_perm)
+  const bool fused_decode = nt > 0 && !fp8 && router_tail_fits(T, E, splits);
+  if (fused_decode) {
+    RouterTail tail = {};
+    tail.counter = reinterpret_cast<int*>(b + kRouterTailCounter);
+    tail.bias = d->bias, tail.T = T, tail.E = E, tail.k = k;
+    tail.topk_idx = I(w.topk_idx), tail.topk_w = Fp(w.topk_w), tail.counts = I(w.counts);
+    tail.offsets = I(w.offsets), tail.perm_token = I(w.perm_token), tail.inv_perm = I(w.inv_perm);
+    tail.p_perm = Fp(w.p_perm);
+    MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s, &tail));
+    if (ev) MOE_CUDA_TRY(record(ev[1]));
+    if (ev) MOE_CUDA_TRY(record(ev[2]));
+  } else {
+    MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s));
+    MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
+                                      Fp(w.topk_w), s));
+    if (ev) MOE_CUDA_TRY(record(ev[1]));
+    // dispatch + gather (one kernel for T <= 256); the FP8 path gathers f16 rows and, for the
+    // shared expert, an f16 copy of x
+    MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), x, T, D, E, k, I(w.counts), I(w.offsets),
+                                I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), H(w.x_perm), fp8,
+                                (fp8 && Fs > 0) ? H(w.x16) : nullptr, I(w.scratch), err, s, nullptr));
+    if (ev) MOE_CUDA_TRY(record(ev[2]));
+  }
   SplitBuf split;  // split-K buffers of the FP8 weight-streaming GEMMs
   if (w.split_partial_bytes > 0) {
     split.partial = Fp(w.split_partial);
@@ -271,10 +303,11 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
     MOE_CUDA_TRY(launch_stream_fp8w(kDown, dn, ds, Fs > 0 ? 2 : 1, nt, split, err, s));
   } else {
   st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), Fp(w.out_perm), x,
-               T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, wide_tiles(d->flags), err,
+               T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, prefill_tiling(d->flags), err,
                s, ev ? ev[3] : nullptr,
                rec_flags, (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) ? H(w.gu_saved) : nullptr,
-               (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && Fs > 0 ? H(w.gu_saved_sh) : nullptr);
+               (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && Fs > 0 ? H(w.gu_saved_sh) : nullptr,
+               fused_decode ? I(w.perm_token) : nullptr);
   if (st != MOE_OK) return st;
   }
   if (ev) MOE_CUDA_TRY(record(ev[4]));
@@ -472,10 +505,12 @@ size_t moe_grouped_swiglu_ffn_workspace_size(int M, int F) {
 }
 
 moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* offsets, const float* row_scale, int M,
-                                    int max_seg, int E, int D, int F, const moe_bf16_t* gate_up,
+                                    int max_seg, int flags, int E, int D, int F, const moe_bf16_t* gate_up,
                                     const moe_bf16_t* down, float* out_perm, void* ws, size_t ws_bytes,
                                     moe_stream_t stream) {
   if (M < 0 || E <= 0 || D <= 0 || F <= 0 || max_seg < 0 || max_seg > M) return MOE_ERR_INVALID_ARG;
+  const int tiling_flags = MOE_FLAG_PREFILL_ROW_TILES | MOE_FLAG_PREFILL_WIDE_TILES | MOE_FLAG_PREFILL_PAIR_TILES;
+  if ((flags & ~tiling_flags) != 0 || (flags & (flags - 1)) != 0) return MOE_ERR_INVALID_ARG;
   if (D % 64 != 0 || F % 64 != 0 || E > 1024) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!x_perm || !offsets || !gate_up || !down || !out_perm || !ws) return MOE_ERR_INVALID_ARG;
   if (!aligned(x_perm, 16) || !aligned(gate_up, 16) || !aligned(down, 16) || !aligned(out_perm, 16) ||
@@ -488,7 +523,7 @@ moe_status_t moe_grouped_swiglu_ffn(const moe_bf16_t* x_perm, const int32_t* off
   uint8_t* b = static_cast<uint8_t*>(ws);
   const int nt = max_seg <= kDecodeTMax ? decode_tile(max_seg < 1 ? 1 : max_seg) : 0;
   return run_ffn(x_perm, offsets, row_scale, M, E, D, F, gate_up, down, reinterpret_cast<uint16_t*>(b + kWsHeader),
-                 out_perm, nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr, nt, wide_tiles(0),
+                 out_perm, nullptr, 0, 0, nullptr, nullptr, nullptr, nullptr, nt, prefill_tiling(flags),
                  reinterpret_cast<int*>(b),
                  (cudaStream_t)stream, nullptr, cudaEventRecordDefault);
 }
@@ -548,6 +583,10 @@ moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16
 
 int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK || desc->T == 0) return 0;
+  // bf16 decode: the router GEMM also selects and dispatches, gate_up gathers its rows itself
+  if (use_decode(*desc) && desc->weight_format == MOE_WEIGHTS_BF16 &&
+      router_tail_fits(desc->T, desc->E, router_k_splits(desc->T, desc->D, desc->E)))
+    return 1 /*router*/ + 2 /*GEMMs*/ + 1;
   // T <= 256: one kernel sorts and gathers (and casts x for the FP8 path's shared expert, T <= 64);
   // above: hist, scan, scatter, gather
   const int dispatch = desc->T <= 256 ? 1 : 4;
@@ -558,8 +597,12 @@ int moe_layer_gemm_path(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK) return -1;
   if (desc->weight_format == MOE_WEIGHTS_FP8_E4M3) return MOE_PATH_FP8_STREAMING;
   if (use_decode(*desc)) return MOE_PATH_STREAMING;
-  const int wide = wide_tiles(desc->flags);
-  return wide == 0 ? MOE_PATH_ROW_TILES : wide == kWideDown ? MOE_PATH_MIXED_TILES : MOE_PATH_WIDE_TILES;
+  const Tiling t = prefill_tiling(desc->flags);
+  if (t.gu == kRowT && t.dn == kRowT) return MOE_PATH_ROW_TILES;
+  if (t.gu == kWideT && t.dn == kWideT) return MOE_PATH_WIDE_TILES;
+  if (t.gu == kPairT && t.dn == kPairT) return MOE_PATH_PAIR_TILES;
+  if (t.gu == kRowT && t.dn == kWideT) return MOE_PATH_MIXED_TILES;
+  return -1;
 }
 
 moe_status_t moe_update_router_bias(const int32_t* counts, int E, float gamma, float* bias, moe_stream_t stream) {

@@ -62,6 +62,7 @@ def test_tiling_option_maps_to_the_layer_flags(bench):
     assert bench.tiling_flag("auto") == 0
     assert bench.tiling_flag("row") == moe.MOE_FLAG_PREFILL_ROW_TILES
     assert bench.tiling_flag("wide") == moe.MOE_FLAG_PREFILL_WIDE_TILES
+    assert bench.tiling_flag("pair") == moe.MOE_FLAG_PREFILL_PAIR_TILES
 
 
 def test_clock_summary_flags_throttling(bench):

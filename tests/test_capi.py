@@ -1,5 +1,6 @@
 """The C-ABI library on the host (no GPU needed): it loads, exports every symbol the header
-declares, and rejects bad arguments before touching the device."""
+declares, and rejects bad arguments before touching the device.  The pointers here are made up,
+so no call in this file may pass validation and launch when a GPU is present."""
 import ctypes
 import os
 import re
@@ -69,7 +70,9 @@ def _desc(**kw):
     (dict(flags=2, T=65), 1),     # decode forced above the decode range
     (dict(flags=8 | 16), 1),      # both prefill tilings
     (dict(flags=2 | 16), 1),      # a prefill tiling with decode forced
-    (dict(flags=32), 1),          # unknown flag
+    (dict(flags=16 | 32), 1),     # token-wide and pair tiles
+    (dict(flags=2 | 32), 1),      # pair tiles with decode forced
+    (dict(flags=64), 1),          # unknown flag
 ])
 def test_layer_forward_rejects_bad_descriptors(L, kw, status):
     d = _desc(**kw)
@@ -85,7 +88,10 @@ def test_layer_workspace_size_and_small_workspace(L):
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, need - 1, None) == 4
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100010, need, None) == 3  # ws not 256-aligned
     assert L.moe_layer_forward(ctypes.byref(d), 0x4008, 0x5000, 0x100000, need, None) == 3
-    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 6  # T=16: one kernel sorts and gathers
+    # T=16 (bf16 decode): the router GEMM also selects and dispatches; gate_up gathers its rows
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 4
+    # forced prefill at T=16: router GEMM, top-k, one kernel that sorts and gathers, 2 GEMMs, combine
+    assert L.moe_layer_kernel_count(ctypes.byref(_desc(flags=1))) == 6
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(T=300))) == 9
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(k=9))) == 0
     # shared expert grows the workspace
@@ -110,11 +116,15 @@ def test_step_entry_points_validate_on_host(L):
     args_bad = list(args)
     args_bad[-1] = None  # x given, x_perm missing
     assert L.moe_permute(*args_bad, 0x100000, need, None) == 1
-    # grouped ffn: max_seg > M, F not multiple of 64
-    assert L.moe_grouped_swiglu_ffn(0x1000, 0x2000, None, 10, 11, 4, 128, 128, 0x3000, 0x4000, 0x5000, 0x100000,
+    # grouped ffn: max_seg > M, F not multiple of 64, two tiling flags, an unknown flag
+    assert L.moe_grouped_swiglu_ffn(0x1000, 0x2000, None, 10, 11, 0, 4, 128, 128, 0x3000, 0x4000, 0x5000, 0x100000,
                                     1 << 20, None) == 1
-    assert L.moe_grouped_swiglu_ffn(0x1000, 0x2000, None, 10, 10, 4, 128, 100, 0x3000, 0x4000, 0x5000, 0x100000,
+    assert L.moe_grouped_swiglu_ffn(0x1000, 0x2000, None, 10, 10, 0, 4, 128, 100, 0x3000, 0x4000, 0x5000, 0x100000,
                                     1 << 20, None) == 2
+    assert L.moe_grouped_swiglu_ffn(0x1000, 0x2000, None, 10, 10, 8 | 32, 4, 128, 128, 0x3000, 0x4000, 0x5000,
+                                    0x100000, 1 << 20, None) == 1
+    assert L.moe_grouped_swiglu_ffn(0x1000, 0x2000, None, 10, 10, 2, 4, 128, 128, 0x3000, 0x4000, 0x5000,
+                                    0x100000, 1 << 20, None) == 1
     assert L.moe_grouped_swiglu_ffn_workspace_size(10, 128) == 256 + 2560 + (256 - 2560 % 256) % 256
     # combine: k > 32, misaligned y
     assert L.moe_combine(0x1000, 0x2000, None, 4, 128, 33, 0x3000, None) == 2
@@ -172,11 +182,16 @@ FP8 = dict(weight_format=1, gate_up=None, down=None, gate_up_fp8=0x8000, gate_up
     (dict(down_scale=0xB002), 3),
 ])
 def test_fp8_descriptor_validation(L, kw, status):
+    import torch
+
     d = _desc(**{**FP8, **kw})
-    st = L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, 1 << 30, None)
     if status == 0:
-        assert st in (0, 8) and L.moe_layer_workspace_size(ctypes.byref(d)) > 0
+        assert L.moe_layer_workspace_size(ctypes.byref(d)) > 0
+        if torch.cuda.is_available():
+            return  # a valid descriptor would launch kernels on the made-up pointers: host checks only
+        assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, 1 << 30, None) == 8
     else:
+        st = L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, 1 << 30, None)
         assert st == status, moe.STATUS.get(st)
 
 
@@ -234,6 +249,7 @@ def test_gemm_path_query(L):
     assert P(T=65) == moe.MOE_PATH_MIXED_TILES
     assert P(T=4096, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_ROW_TILES) == moe.MOE_PATH_ROW_TILES
     assert P(T=4096, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_WIDE_TILES
+    assert P(T=4096, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_PAIR_TILES) == moe.MOE_PATH_PAIR_TILES
     assert P(T=16, flags=moe.MOE_FLAG_PREFILL_WIDE_TILES) == moe.MOE_PATH_STREAMING  # tiling flags leave decode
     assert P(T=300, E=8, k=2, flags=moe.MOE_FLAG_PREFILL_ROW_TILES) == moe.MOE_PATH_ROW_TILES
     assert P(**FP8) == moe.MOE_PATH_FP8_STREAMING

@@ -82,13 +82,16 @@ def test_backward_matches_oracle(cuda_device, w):
     _check(w, h, dy_h, dx, g)
 
 
-@pytest.mark.parametrize("tiling", [moe.MOE_FLAG_PREFILL_ROW_TILES, moe.MOE_FLAG_PREFILL_WIDE_TILES],
-                         ids=["row_tiles", "wide_tiles"])
-def test_backward_after_either_forward_tiling(cuda_device, tiling):
-    """Both prefill tilings save the same g | u layout for the backward pass."""
+TILINGS = {moe.MOE_FLAG_PREFILL_ROW_TILES: "row_tiles", moe.MOE_FLAG_PREFILL_WIDE_TILES: "wide_tiles",
+           moe.MOE_FLAG_PREFILL_PAIR_TILES: "pair_tiles"}
+
+
+@pytest.mark.parametrize("tiling", list(TILINGS), ids=list(TILINGS.values()))
+def test_backward_after_every_forward_tiling(cuda_device, tiling):
+    """Every prefill tiling saves the same g | u layout for the backward pass."""
     w = W(300, 256, 4, 2, 192, Fs=128, bias="normal:0.5")
     h, d, dy_h, L, y, dx, g = _run(w, flags=moe.MOE_FLAG_SAVE_FOR_BACKWARD | tiling)
-    assert L.gemm_path(w.T) == ("row_tiles" if tiling == moe.MOE_FLAG_PREFILL_ROW_TILES else "wide_tiles")
+    assert L.gemm_path(w.T) == TILINGS[tiling]
     _check(w, h, dy_h, dx, g)
 
 

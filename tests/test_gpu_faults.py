@@ -6,7 +6,8 @@ Nothing else changes: the consumers' waits are bounded (1 s of wall time), so th
 MOE_ERR_TIMEOUT in the workspace's error word, drains its own copies, frees TMEM and returns.
 Each case runs in a child process started with n = 1: its first forward's gate_up launch times
 out, the host reads the status, and the next forward on the same context must match the oracle.
-The three expert-GEMM kernels are covered: 128-row tiles, token-wide tiles and weight streaming.
+The expert-GEMM kernels are covered: 128-row tiles, token-wide tiles (one CTA and CTA pairs) and
+weight streaming.
 """
 import json
 import os
@@ -52,7 +53,7 @@ print("RESULT " + json.dumps(dict(first=first, second=second, elapsed=elapsed, e
 """
 
 CASES = [(100, moe.MOE_FLAG_PREFILL_ROW_TILES, "row_tiles"), (100, moe.MOE_FLAG_PREFILL_WIDE_TILES, "wide_tiles"),
-         (24, 0, "streaming")]
+         (100, moe.MOE_FLAG_PREFILL_PAIR_TILES, "pair_tiles"), (24, 0, "streaming")]
 
 
 @pytest.mark.parametrize("T,flags,path", CASES, ids=[c[2] for c in CASES])

@@ -275,22 +275,42 @@ def test_decode_path_is_deterministic_and_matches_oracle():
     assert L.device_error() == 0
 
 
-def test_decode_layer_equals_the_step_by_step_path_bit_for_bit():
-    """The layer forward and the step-by-step entry points (router, permute, grouped FFN with the
-    same 16-token tile, combine) are the same computation and must give the same bits."""
-    w = W(16, 256, 32, 4, 384, bias="normal:0.5")
+DECODE_STEP_CASES = [
+    W(16, 256, 32, 4, 384, bias="normal:0.5"),
+    W(1, 256, 32, 4, 384, bias="zipf:1.1"),
+    W(64, 256, 64, 8, 128, Fs=128, bias="normal:0.5"),
+    W(3, 128, 256, 8, 64, Fs=64, bias="normal:0.5"),
+]
+
+
+@pytest.mark.parametrize("w", DECODE_STEP_CASES, ids=lambda w: w.name)
+def test_decode_layer_equals_the_step_by_step_path_bit_for_bit(w):
+    """The decode layer forward (router GEMM whose last CTA selects and dispatches, gate_up that
+    gathers its token rows from x) and the step-by-step entry points (router + top-k kernel,
+    permute with x_perm, grouped FFN with the same token tile, combine) are the same computation
+    and must give the same bits; the layer's counts equal the oracle's."""
+    import torch
+
     inp, _ = host_case(w)
     d = device_from_host(inp)
     L = layer_from(d, w.k)
+    assert L.kernel_count(w.T) == 4
     y_layer = to_np_bf16(L(d["x"]))
     assert L.device_error() == 0
+    o_idx, _ = oracle.router(inp["x"], inp["wg"], inp["bias"], w.k)
+    counts, _, _, _, _ = oracle.permute(o_idx, w.E)
+    assert (L.expert_counts(w.T).cpu().numpy() == counts).all()
     idx, p = moe.moe_router_topk(d["x"], d["wg"], d["bias"], w.k)
+    assert (idx.cpu().numpy() == o_idx).all()
     pm = moe.moe_permute(idx, p, d["x"], w.E)
-    max_seg = int(pm["counts"].max().item())
-    assert 0 < max_seg <= 16
     out_perm, _ = moe.moe_grouped_swiglu_ffn(pm["x_perm"], pm["offsets"], pm["p_perm"], d["gate_up"], d["down"],
-                                             max_seg=max_seg)
-    y_steps = to_np_bf16(moe.moe_combine(out_perm, pm["inv_perm"], None, w.T, w.k))
+                                             max_seg=w.T)
+    shared = None
+    if w.Fs:
+        off = torch.tensor([0, w.T], dtype=torch.int32, device="cuda")
+        shared, _ = moe.moe_grouped_swiglu_ffn(d["x"], off, None, d["shared_gate_up"][None], d["shared_down"][None],
+                                               max_seg=w.T)
+    y_steps = to_np_bf16(moe.moe_combine(out_perm, pm["inv_perm"], shared, w.T, w.k))
     assert (y_layer == y_steps).all()
 
 
@@ -334,13 +354,16 @@ FULL = ["mixtral", "gptoss", "gptoss_decode_T1", "gptoss_decode_T8", "gptoss_dec
 
 # the prefill tilings other than the default mix, at full size
 OTHER_TILING = [("mixtral", moe.MOE_FLAG_PREFILL_ROW_TILES), ("gptoss", moe.MOE_FLAG_PREFILL_WIDE_TILES),
-                ("deepseek", moe.MOE_FLAG_PREFILL_ROW_TILES), ("deepseek", moe.MOE_FLAG_PREFILL_WIDE_TILES)]
+                ("deepseek", moe.MOE_FLAG_PREFILL_ROW_TILES), ("deepseek", moe.MOE_FLAG_PREFILL_WIDE_TILES),
+                ("mixtral", moe.MOE_FLAG_PREFILL_PAIR_TILES), ("gptoss", moe.MOE_FLAG_PREFILL_PAIR_TILES),
+                ("deepseek", moe.MOE_FLAG_PREFILL_PAIR_TILES)]
+_TILING_ID = {moe.MOE_FLAG_PREFILL_ROW_TILES: "row", moe.MOE_FLAG_PREFILL_WIDE_TILES: "wide",
+              moe.MOE_FLAG_PREFILL_PAIR_TILES: "pair"}
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name,flags", [(n, 0) for n in FULL] + OTHER_TILING,
-                         ids=[n for n in FULL] + [f"{n}-{'wide' if f == moe.MOE_FLAG_PREFILL_WIDE_TILES else 'row'}"
-                                                  for n, f in OTHER_TILING])
+                         ids=[n for n in FULL] + [f"{n}-{_TILING_ID[f]}" for n, f in OTHER_TILING])
 def test_full_size_workload_parity(name, flags):
     """Routing of every token and the whole dispatch (counts, offsets, perm_token, inv_perm)
     bit-exact against the oracle; layer outputs within tolerance on every token that holds the
