@@ -207,8 +207,8 @@ moe_status_t moe_combine(const float* out_perm, const int32_t* inv_perm, const f
  *  PAIR_TILES both on the WIDE orientation computed by a cluster of two CTAs: 256 weight rows x
  *             up to 256 tokens per tcgen05.mma.cta_group::2, each CTA loading its own half of both
  *             operands (no multicast).
- * Without any, gate_up runs ROW_TILES and down WIDE_TILES.  All give the same routing;
- * outputs agree within fp32 rounding order. */
+ * Without any, gate_up runs ROW_TILES and down PAIR_TILES (the measured best per GEMM).  All
+ * give the same routing; outputs agree within fp32 rounding order. */
 #define MOE_FLAG_PREFILL_ROW_TILES 8
 #define MOE_FLAG_PREFILL_WIDE_TILES 16
 #define MOE_FLAG_PREFILL_PAIR_TILES 32
@@ -285,7 +285,7 @@ int moe_layer_kernel_count(const moe_layer_desc_t* desc);
 #define MOE_PATH_FP8_STREAMING 1
 #define MOE_PATH_ROW_TILES 2
 #define MOE_PATH_WIDE_TILES 3
-#define MOE_PATH_MIXED_TILES 4 /* gate_up on 128-row tiles, down on token-wide tiles */
+#define MOE_PATH_MIXED_TILES 4 /* gate_up on 128-row tiles, down on token-wide tiles of CTA pairs */
 #define MOE_PATH_PAIR_TILES 5  /* both on token-wide tiles of CTA pairs */
 int moe_layer_gemm_path(const moe_layer_desc_t* desc);
 

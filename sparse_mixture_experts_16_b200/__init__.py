@@ -340,7 +340,7 @@ class MoELayer:
 
     def gemm_path(self, T: int) -> str:
         """The expert-GEMM kernels a forward over T tokens runs: "streaming", "fp8_streaming",
-        "row_tiles", "wide_tiles", "mixed_tiles" (gate_up on row tiles, down on wide tiles) or
+        "row_tiles", "wide_tiles", "mixed_tiles" (gate_up on row tiles, down on pair tiles) or
         "pair_tiles" (both on token-wide tiles of CTA pairs)."""
         d = self.desc(T)
         code = lib().moe_layer_gemm_path(ctypes.byref(d))

@@ -263,6 +263,7 @@ __global__ void __launch_bounds__(kPThreads, 1) grouped_gemm_pair_kernel(const _
           } else {
             tma_load_2d_pair(&p.w_map[ti.set], bar, sb, kx, wrow);
           }
+
           if (half == 128) {
             tma_load_2d_pair(&p.t_map128[ti.set], bar, sb + kPTileW, kx, trow);
           } else {

@@ -73,11 +73,6 @@ struct alignas(64) GemmParams {
   // gather_rows[row] (the permutation), instead of read from a permuted copy (NULL: TMA rows of a)
   const int32_t* gather_rows[2];
   const uint16_t* gather_src[2];
-  // streaming kGateUp: CTAs without a unit prefetch into L2 the down weights of the active groups
-  // (prefetch_w[s] + group * prefetch_bytes[s]) when they total at most prefetch_limit bytes
-  const uint8_t* prefetch_w[2];
-  long long prefetch_bytes[2];
-  long long prefetch_limit;
   RouterTail tail;  // streaming kRouter: fused top-k selection and dispatch (tail.counter NULL: off)
   int n_sets;
   int withhold_first_load;  // test only: never issue the first stage's copies (its wait then times out)
@@ -309,43 +304,13 @@ __device__ void router_tail(const GemmParams& p, uint8_t* scratch) {
   if (tid == 0) *rt.counter = 0;  // ready for the next launch
 }
 
-// Streaming gate_up: CTAs without a unit prefetch the active groups' down weights into L2, split
-// into 64 KB pieces over those CTAs' lanes, so the down launch that follows reads them from L2
-// while this launch still streams gate_up weights from HBM.
-template <int KIND, int NT>
-__device__ void prefetch_down_weights(const GemmParams& p, const int* tile_start, int G, int total, int lane) {
-  constexpr long long kPiece = 64 * 1024;
-  long long bytes = 0;
-  int n_active = 0;
-  for (int g = 0; g < G; ++g) {
-    const int s = g < p.n_groups[0] ? 0 : 1;
-    if (tile_start[g + 1] > tile_start[g] && p.prefetch_w[s] != nullptr) bytes += p.prefetch_bytes[s], ++n_active;
-  }
-  if (n_active == 0 || bytes > p.prefetch_limit) return;
-  const long long workers = (long long)(gridDim.x - total) * 32;
-  const long long me = (long long)(blockIdx.x - total) * 32 + lane;
-  long long base = 0;  // running piece index of the active groups
-  for (int g = 0; g < G; ++g) {
-    const int s = g < p.n_groups[0] ? 0 : 1;
-    if (!(tile_start[g + 1] > tile_start[g] && p.prefetch_w[s] != nullptr)) continue;
-    const int gl = s == 0 ? g : g - p.n_groups[0];
-    const long long gbytes = p.prefetch_bytes[s];
-    const long long pieces = (gbytes + kPiece - 1) / kPiece;
-    const uint8_t* w = p.prefetch_w[s] + (long long)gl * gbytes;
-    for (long long pc = ((me - base) % workers + workers) % workers; pc < pieces; pc += workers) {
-      const long long off = pc * kPiece;
-      prefetch_l2_bulk(w + off, (uint32_t)min(kPiece, gbytes - off));
-    }
-    base += pieces;
-  }
-}
-
 template <int KIND, int NT>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<KIND, NT>;
   // streaming gate_up: the whole producer warp fills stages (lane 0 the weight copies, all lanes
-  // the gathered token rows), so each full barrier also counts the 32 lanes' cp.async arrivals
+  // the gathered token rows), so each full barrier also counts the 32 lanes' arrivals
   constexpr bool kWarpProducer = (NT > 0 && KIND == kGateUp);
+  constexpr int kGatherRows = NT > 0 ? NT : 4;  // token rows of one stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
@@ -419,9 +384,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if constexpr (KIND == kGateUp && NT > 0) {
-      if ((int)blockIdx.x >= total && total > 0) prefetch_down_weights<KIND, NT>(p, tile_start, G, total, lane);
-    }
     if (kWarpProducer || lane == 0) {
       uint32_t it = 0;
       bool ok = true;
@@ -432,16 +394,18 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const CUtensorMap* wmap = &p.w_map[ti.set];
         const int wbase = ti.gl * p.w_rows[ti.set];
         // gathered token rows: this lane copies 16-byte chunk (lane & 7) of rows (lane >> 3) + 4 i
+        // of the segment's <= NT rows
         const bool gather = kWarpProducer && p.gather_rows[ti.set] != nullptr;
-        int tok[NT > 0 ? NT / 4 : 1];
+        int tok[kGatherRows / 4];
         if constexpr (kWarpProducer) {
 #pragma unroll
-          for (int i = 0; i < NT / 4; ++i) {
+          for (int i = 0; i < kGatherRows / 4; ++i) {
             const int j = (lane >> 3) + 4 * i;
             tok[i] = (gather && j < ti.rows) ? p.gather_rows[ti.set][ti.row0 + j] : -1;
           }
         }
-        const uint32_t stage_bytes = gather ? (uint32_t)(C::kStageBytes - NT * kBK * 2) : (uint32_t)C::kStageBytes;
+        const uint32_t stage_bytes =
+            gather ? (uint32_t)(C::kStageBytes - kGatherRows * kBK * 2) : (uint32_t)C::kStageBytes;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++it) {
           const int stage = it % C::kStages;
           bool got = lane != 0 || mbar_wait(&empty[stage], ((it / C::kStages) & 1) ^ 1, kWaitLimitNs);
@@ -485,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
               const uint16_t* src0 = p.gather_src[ti.set];
               const int K = p.k_blocks[ti.set] * kBK;
 #pragma unroll
-              for (int i = 0; i < NT / 4; ++i) {
+              for (int i = 0; i < kGatherRows / 4; ++i) {
                 const int j = (lane >> 3) + 4 * i;
                 const uint32_t dst = tbase + (uint32_t)(j * 128 + ((c ^ (j & 7)) << 4));
                 const uint16_t* src = tok[i] >= 0 ? src0 + (size_t)tok[i] * K + kx + c * 8 : src0;
@@ -756,10 +720,6 @@ int num_sms() {
   return n;
 }
 
-// Down weights of the active experts are prefetched into L2 during a streaming gate_up launch only
-// while they fit comfortably next to the streamed gate_up weights (which are marked evict-first).
-constexpr long long kPrefetchLimit = 64ll << 20;
-
 template <int KIND, int NT>
 cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int* err, cudaStream_t s,
                           const RouterTail* tail = nullptr) {
@@ -769,7 +729,6 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int
   p.n_sets = n_sets;
   p.k_splits = k_splits;
   p.err = err;
-  p.prefetch_limit = kPrefetchLimit;
   if (KIND == kRouter && NT > 0 && tail != nullptr) p.tail = *tail;
   p.withhold_first_load = (KIND != kRouter && test_withhold_this_launch()) ? 1 : 0;
   const uint32_t a_box = C::kTiled ? kBM : NT;
@@ -790,11 +749,7 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int
     if (KIND == kGateUp && NT > 0) {
       p.gather_rows[i] = st.gather_rows;
       p.gather_src[i] = st.gather_src;
-      p.prefetch_w[i] = static_cast<const uint8_t*>(st.prefetch_w);
-      p.prefetch_bytes[i] = st.prefetch_bytes;
       if ((st.gather_rows != nullptr) != (st.gather_src != nullptr)) return cudaErrorInvalidValue;
-      if (st.prefetch_w != nullptr && (st.prefetch_bytes <= 0 || st.prefetch_bytes % 16 != 0))
-        return cudaErrorInvalidValue;
     }
     p.n_groups[i] = st.n_groups;
     p.m_rows[i] = st.m_rows;

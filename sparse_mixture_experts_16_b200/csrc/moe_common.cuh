@@ -167,10 +167,6 @@ struct GemmSetHost {
   // permutation) instead of reading a (NULL: read a)
   const int32_t* gather_rows = nullptr;
   const uint16_t* gather_src = nullptr;
-  // streaming gate_up: prefetch into L2 the down weights of the active groups (group g at
-  // prefetch_w + g * prefetch_bytes) from the CTAs that have no unit (NULL: no prefetch)
-  const void* prefetch_w = nullptr;
-  long long prefetch_bytes = 0;
 };
 
 enum GemmKind { kGateUp = 0, kDown = 1, kRouter = 2 };

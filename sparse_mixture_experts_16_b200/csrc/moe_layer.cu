@@ -62,7 +62,7 @@ Tiling prefill_tiling(int flags) {
   if (flags & MOE_FLAG_PREFILL_WIDE_TILES) return {kWideT, kWideT};
   if (flags & MOE_FLAG_PREFILL_ROW_TILES) return {kRowT, kRowT};
   if (flags & MOE_FLAG_PREFILL_PAIR_TILES) return {kPairT, kPairT};
-  return {kRowT, kWideT};
+  return {kRowT, kPairT};
 }
 
 cudaError_t launch_tiled(TileKind t, GemmKind kind, const GemmSetHost* sets, int n_sets, int* err, cudaStream_t s) {
@@ -178,20 +178,16 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
                      unsigned ev_flags, uint16_t* save_gu = nullptr, uint16_t* save_gu_sh = nullptr,
                      const int32_t* perm_token = nullptr) {
   // perm_token (streaming only): the gate_up launch gathers its token rows from x by the
-  // permutation (x_perm is not read) and prefetches the active experts' down weights into L2
+  // permutation (x_perm is not read)
   GemmSetHost g[2] = {};
   const bool gather = decode_nt > 0 && perm_token != nullptr;
   g[0].K = D, g[0].a = gather ? x : x_perm, g[0].a_rows = gather ? T : M, g[0].w = gate_up, g[0].n_groups = E;
   g[0].offsets = offsets, g[0].n_out = F, g[0].out = h, g[0].save_gu = save_gu;
-  if (gather) {
-    g[0].gather_rows = perm_token, g[0].gather_src = x;
-    g[0].prefetch_w = down, g[0].prefetch_bytes = (long long)D * F * 2;
-  }
+  if (gather) g[0].gather_rows = perm_token, g[0].gather_src = x;
   int n_sets = 1;
   if (Fs > 0) {
     g[1].K = D, g[1].a = x, g[1].a_rows = T, g[1].w = sgu, g[1].n_groups = 1, g[1].m_rows = T;
     g[1].n_out = Fs, g[1].out = h_sh, g[1].save_gu = save_gu_sh;
-    if (gather) g[1].prefetch_w = sdn, g[1].prefetch_bytes = (long long)D * Fs * 2;
     n_sets = 2;
   }
   if (decode_nt == 0)
@@ -601,7 +597,7 @@ int moe_layer_gemm_path(const moe_layer_desc_t* desc) {
   if (t.gu == kRowT && t.dn == kRowT) return MOE_PATH_ROW_TILES;
   if (t.gu == kWideT && t.dn == kWideT) return MOE_PATH_WIDE_TILES;
   if (t.gu == kPairT && t.dn == kPairT) return MOE_PATH_PAIR_TILES;
-  if (t.gu == kRowT && t.dn == kWideT) return MOE_PATH_MIXED_TILES;
+  if (t.gu == kRowT && t.dn == kPairT) return MOE_PATH_MIXED_TILES;
   return -1;
 }
 

@@ -99,7 +99,7 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// ------------------------------------------------------------------------------ LSU copies and prefetch
+// ------------------------------------------------------------------------------ LSU copies
 // 16-byte global -> shared copy (L2 only, not L1); src_bytes < 16 zero-fills the rest (0: no read).
 __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes) : "memory");
@@ -113,10 +113,6 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
 // stores) before later async-proxy reads (tcgen05.mma operands).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-// Fire-and-forget prefetch of [addr, addr + bytes) into L2 (addr and bytes multiples of 16).
-__device__ __forceinline__ void prefetch_l2_bulk(const void* addr, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(addr), "r"(bytes) : "memory");
 }
 
 // ------------------------------------------------------------------------------ tcgen05

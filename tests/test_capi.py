@@ -92,6 +92,7 @@ def test_layer_workspace_size_and_small_workspace(L):
     assert L.moe_layer_kernel_count(ctypes.byref(d)) == 4
     # forced prefill at T=16: router GEMM, top-k, one kernel that sorts and gathers, 2 GEMMs, combine
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(flags=1))) == 6
+    # T=300 prefill: router GEMM, top-k, hist, scan, scatter, gather, 2 GEMMs, combine
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(T=300))) == 9
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(k=9))) == 0
     # shared expert grows the workspace
@@ -239,7 +240,7 @@ def test_backward_entry_validates_on_host(L):
 
 def test_gemm_path_query(L):
     """The host-only path query follows the flags and the default rule: T <= 64 streams the weights;
-    larger T runs gate_up on 128-row tiles and down on token-wide tiles unless one tiling is asked
+    larger T runs gate_up on 128-row tiles and down on token-wide tiles of CTA pairs unless one tiling is asked
     for; E4M3 weights always stream."""
     P = lambda **kw: L.moe_layer_gemm_path(ctypes.byref(_desc(**kw)))
     assert P() == moe.MOE_PATH_STREAMING                                     # T = 16

@@ -283,7 +283,7 @@ DECODE_STEP_CASES = [
 ]
 
 
-@pytest.mark.parametrize("w", DECODE_STEP_CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("w", DECODE_STEP_CASES + [W(16, 128, 1024, 32, 64)], ids=lambda w: w.name)
 def test_decode_layer_equals_the_step_by_step_path_bit_for_bit(w):
     """The decode layer forward (router GEMM whose last CTA selects and dispatches, gate_up that
     gathers its token rows from x) and the step-by-step entry points (router + top-k kernel,
@@ -291,7 +291,9 @@ def test_decode_layer_equals_the_step_by_step_path_bit_for_bit(w):
     and must give the same bits; the layer's counts equal the oracle's."""
     import torch
 
-    inp, _ = host_case(w)
+    # E = 1024, k = 32, T = 16: the fused tail's logit table is exactly its 64 KB; D = 128 logits
+    # are accurate to ~1e-6 in fp32, so a 2e-4 score gap keeps the selection exact
+    inp, _ = host_case(w, delta=2e-4 if w.E > 256 else None)
     d = device_from_host(inp)
     L = layer_from(d, w.k)
     assert L.kernel_count(w.T) == 4

@@ -188,3 +188,4 @@ def test_standalone_ffn_entry_prefill_sizes(cuda_device):
         ref = np.stack([scale[r] * oracle.expert_ffn(xp[r], gu[e], dn[e])
                         for e in range(E) for r in range(offsets[e], offsets[e + 1])])
         assert rel_rms_err(got, ref) <= REL_RMS_TOL
+
