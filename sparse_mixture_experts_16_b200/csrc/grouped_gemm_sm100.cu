@@ -387,7 +387,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     if (kWarpProducer || lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      const uint64_t w_policy = policy_evict_first();  // streaming weights are read once per step
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile ti = decode_tile<KIND, NT>(p, tile_start, G, t);
         const CUtensorMap* amap = &p.a_map[ti.set];
@@ -431,8 +430,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
               } else {
                 if constexpr (KIND == kGateUp) {
                   const int F = p.n_out[ti.set];
-                  tma_load_2d_hint(wmap, &full[stage], sb, kx, wbase + ti.n * 128, w_policy);
-                  tma_load_2d_hint(wmap, &full[stage], sb + kTileBytesA, kx, wbase + F + ti.n * 128, w_policy);
+                  tma_load_2d(wmap, &full[stage], sb, kx, wbase + ti.n * 128);
+                  tma_load_2d(wmap, &full[stage], sb + kTileBytesA, kx, wbase + F + ti.n * 128);
                   if (!gather) tma_load_2d(amap, &full[stage], sb + 2 * kTileBytesA, kx, ti.row0);
                 } else {
                   tma_load_2d(wmap, &full[stage], sb, kx, wbase + ti.n * 128);

@@ -136,6 +136,12 @@ cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wg, int T, int
                                int k_splits, int* err, cudaStream_t s, const RouterTail* tail = nullptr);
 cudaError_t launch_router_select(const float* partials, int k_splits, int T, int ld, const float* bias, int E, int k,
                                  int32_t* idx, float* w, cudaStream_t s);
+// One-CTA routing for a few tokens when x and W_g fit in shared memory (router_topk.cu): logits on
+// the CUDA cores, top-k and weights, and (counts != NULL) the dispatch metadata.
+bool router_small_fits(int T, int D, int E, int k);
+cudaError_t launch_router_small(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int D, int E, int k,
+                                int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                                int32_t* perm_token, int32_t* inv_perm, float* p_perm, int* err, cudaStream_t s);
 
 cudaError_t launch_update_bias(const int32_t* counts, int E, float gamma, float* bias, cudaStream_t s);
 

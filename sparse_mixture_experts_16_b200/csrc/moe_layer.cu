@@ -245,8 +245,16 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
   const int nt = use_decode(*d) ? decode_tile(T) : 0;
   // bf16 decode: the router GEMM's last CTA also selects and dispatches (no top-k or dispatch
   // launch), and the gate_up launch gathers token rows from x itself (no x_perm)
-  const bool fused_decode = nt > 0 && !fp8 && router_tail_fits(T, E, splits);
-  if (fused_decode) {
+  // a few decode tokens whose x and W_g fit in shared memory: one CTA routes (and, for bf16,
+  // dispatches) on the CUDA cores
+  const bool small_router = nt > 0 && router_small_fits(T, D, E, k);
+  const bool fused_decode = nt > 0 && !fp8 && (small_router || router_tail_fits(T, E, splits));
+  if (fused_decode && small_router) {
+    MOE_CUDA_TRY(launch_router_small(x, d->w_gate, d->bias, T, D, E, k, I(w.topk_idx), Fp(w.topk_w), I(w.counts),
+                                     I(w.offsets), I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), err, s));
+    if (ev) MOE_CUDA_TRY(record(ev[1]));
+    if (ev) MOE_CUDA_TRY(record(ev[2]));
+  } else if (fused_decode) {
     RouterTail tail = {};
     tail.counter = reinterpret_cast<int*>(b + kRouterTailCounter);
     tail.bias = d->bias, tail.T = T, tail.E = E, tail.k = k;
@@ -257,9 +265,14 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
     if (ev) MOE_CUDA_TRY(record(ev[1]));
     if (ev) MOE_CUDA_TRY(record(ev[2]));
   } else {
-    MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s));
-    MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
-                                      Fp(w.topk_w), s));
+    if (small_router) {
+      MOE_CUDA_TRY(launch_router_small(x, d->w_gate, d->bias, T, D, E, k, I(w.topk_idx), Fp(w.topk_w), nullptr,
+                                       nullptr, nullptr, nullptr, nullptr, err, s));
+    } else {
+      MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s));
+      MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
+                                        Fp(w.topk_w), s));
+    }
     if (ev) MOE_CUDA_TRY(record(ev[1]));
     // dispatch + gather (one kernel for T <= 256); the FP8 path gathers f16 rows and, for the
     // shared expert, an f16 copy of x
@@ -392,6 +405,11 @@ moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, cons
   float* part = reinterpret_cast<float*>(b + kWsHeader);
   const int splits = router_k_splits(T, D, E);
   cudaStream_t s = (cudaStream_t)stream;
+  if (router_small_fits(T, D, E, k)) {  // the layer's decode router, so both give the same bits
+    MOE_CUDA_TRY(launch_router_small(x, w_gate, bias, T, D, E, k, topk_idx, topk_w, nullptr, nullptr, nullptr,
+                                     nullptr, nullptr, reinterpret_cast<int*>(b), s));
+    return MOE_OK;
+  }
   MOE_CUDA_TRY(launch_router_gemm(x, w_gate, T, D, E, part, router_ld(E), splits, reinterpret_cast<int*>(b), s));
   MOE_CUDA_TRY(launch_router_select(part, splits, T, router_ld(E), bias, E, k, topk_idx, topk_w, s));
   return MOE_OK;
@@ -579,10 +597,13 @@ moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16
 
 int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  // bf16 decode: the router GEMM also selects and dispatches, gate_up gathers its rows itself
-  if (use_decode(*desc) && desc->weight_format == MOE_WEIGHTS_BF16 &&
-      router_tail_fits(desc->T, desc->E, router_k_splits(desc->T, desc->D, desc->E)))
+  const bool decode = use_decode(*desc);
+  const bool small = decode && router_small_fits(desc->T, desc->D, desc->E, desc->k);
+  // bf16 decode: one router kernel also selects and dispatches, gate_up gathers its rows itself
+  if (decode && desc->weight_format == MOE_WEIGHTS_BF16 &&
+      (small || router_tail_fits(desc->T, desc->E, router_k_splits(desc->T, desc->D, desc->E))))
     return 1 /*router*/ + 2 /*GEMMs*/ + 1;
+  if (small) return 1 /*router*/ + 1 /*dispatch*/ + 2 + 1;  // E4M3 decode
   // T <= 256: one kernel sorts and gathers (and casts x for the FP8 path's shared expert, T <= 64);
   // above: hist, scan, scatter, gather
   const int dispatch = desc->T <= 256 ? 1 : 4;

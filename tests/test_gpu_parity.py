@@ -278,6 +278,7 @@ def test_decode_path_is_deterministic_and_matches_oracle():
 DECODE_STEP_CASES = [
     W(16, 256, 32, 4, 384, bias="normal:0.5"),
     W(1, 256, 32, 4, 384, bias="zipf:1.1"),
+    W(2, 2880, 32, 4, 128, bias="zipf:1.1"),  # the gpt-oss-shaped router: W_g in 7 bulk copies, one CTA
     W(64, 256, 64, 8, 128, Fs=128, bias="normal:0.5"),
     W(3, 128, 256, 8, 64, Fs=64, bias="normal:0.5"),
 ]
@@ -285,8 +286,9 @@ DECODE_STEP_CASES = [
 
 @pytest.mark.parametrize("w", DECODE_STEP_CASES + [W(16, 128, 1024, 32, 64)], ids=lambda w: w.name)
 def test_decode_layer_equals_the_step_by_step_path_bit_for_bit(w):
-    """The decode layer forward (router GEMM whose last CTA selects and dispatches, gate_up that
-    gathers its token rows from x) and the step-by-step entry points (router + top-k kernel,
+    """The decode layer forward (one router kernel that also selects and dispatches -- the one-CTA
+    router for T <= 4 when W_g fits in shared memory, else the router GEMM whose last CTA does it
+    -- and a gate_up that gathers its token rows from x) and the step-by-step entry points (router,
     permute with x_perm, grouped FFN with the same token tile, combine) are the same computation
     and must give the same bits; the layer's counts equal the oracle's."""
     import torch
