@@ -36,8 +36,6 @@
 #include <cuda.h>
 
 #include <atomic>
-#include <cfloat>
-#include <climits>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -69,11 +67,6 @@ struct alignas(64) GemmParams {
   int ld_out[2];    // row stride of the output (elements)
   int k_splits;     // kRouter: K is split into this many contiguous k-block ranges
   uint16_t* save_gu[2];  // tiled kGateUp in a training forward: g | u [rows, 2F] bf16, or NULL
-  // streaming kGateUp: the token rows of set s are gathered straight from gather_src [*, K] by
-  // gather_rows[row] (the permutation), instead of read from a permuted copy (NULL: TMA rows of a)
-  const int32_t* gather_rows[2];
-  const uint16_t* gather_src[2];
-  RouterTail tail;  // streaming kRouter: fused top-k selection and dispatch (tail.counter NULL: off)
   int n_sets;
   int withhold_first_load;  // test only: never issue the first stage's copies (its wait then times out)
   int* err;
@@ -158,159 +151,9 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, const int* tile
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
 
-// ------------------------------------------------------------------------------ fused router tail
-// Decode router (streaming kRouter): once every CTA has written its split-K partial logits, the
-// last CTA to finish (a device-wide counter) selects each token's top k and sorts the T*k slots by
-// expert, so the layer needs neither a top-k nor a dispatch launch.  It computes exactly what
-// router_topk.cu and the one-kernel dispatch of permute.cu compute:
-//   l[t][e]  = sum of the partials over the splits, in split order (fp32);
-//   selection: k rounds of the highest l + bias (ties -> lower expert id);
-//   weights  : softmax of the chosen unbiased logits (fp32 expf, butterfly sums);
-//   dispatch : counts, offsets (exclusive scan), and the stable order (experts ascending, tokens
-//              ascending within an expert) as perm_token / inv_perm / p_perm.
-// All 192 threads first reduce the partials into a [T][ld] logit table in shared memory with
-// 16-byte loads, all splits of one item in flight at once; the warps then select token by token.
-// Scratch lives in the (now idle) pipeline stages of shared memory: T * ld * 4 <= kTailTableBytes.
-constexpr int kTailWarps = kThreads / 32;
-constexpr int kTailTableBytes = 64 * 1024;
-// flag + table + taken flags (E <= 1024 per warp) + slot ids and weights (T*k <= 2048) + counts
-static_assert(256 + kTailTableBytes + kTailWarps * 1024 + 2 * 2048 * 4 + 2 * 1024 * 4 + 64 <=
-                  Cfg<kRouter, 16>::kStages * Cfg<kRouter, 16>::kStageBytes,
-              "the router tail's scratch fits in the smallest router kernel's stages");
-
-__device__ void router_tail(const GemmParams& p, uint8_t* scratch) {
-  const RouterTail& rt = p.tail;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int* flag = reinterpret_cast<int*>(scratch);
-  __threadfence();  // this thread's partials are visible device-wide before the count below
-  __syncthreads();
-  if (tid == 0) *flag = (atomicAdd(rt.counter, 1) == (int)gridDim.x - 1) ? 1 : 0;
-  __syncthreads();
-  if (*flag == 0) return;
-  __threadfence();
-  const int T = rt.T, E = rt.E, k = rt.k, S = p.k_splits, ld = p.ld_out[0];
-  const int n_items = T * k;
-  const float* part = static_cast<const float*>(p.out[0]);
-  float* table = reinterpret_cast<float*>(scratch + 256);                        // [T][ld] logits
-  uint8_t* taken_all = reinterpret_cast<uint8_t*>(scratch + 256 + kTailTableBytes);  // [warps][E]
-  int* idx_s = reinterpret_cast<int*>(taken_all + ((kTailWarps * E + 15) & ~15));  // [T*k]
-  float* w_s = reinterpret_cast<float*>(idx_s + n_items);                        // [T*k]
-  int* cnt = reinterpret_cast<int*>(w_s + n_items);                              // [E]
-  int* run = cnt + E;                                                            // [E]
-  int* warp_tot = run + E;                                                       // [warps]
-  // (1) logits: item (t, 4 experts) sums its kMaxSplits-bounded partials in split order
-  const int quads = ld / 4;
-  for (int item = tid; item < T * quads; item += kThreads) {
-    const int t = item / quads, e4 = (item - t * quads) * 4;
-    const float4* src = reinterpret_cast<const float4*>(part + (size_t)t * ld + e4);
-    const size_t stride4 = (size_t)T * ld / 4;
-    float4 v[kMaxSplits];
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp)
-      if (sp < S) v[sp] = __ldcg(src + sp * stride4);
-    float4 l = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp)
-      if (sp < S) l.x += v[sp].x, l.y += v[sp].y, l.z += v[sp].z, l.w += v[sp].w;
-    *reinterpret_cast<float4*>(table + (size_t)t * ld + e4) = l;
-  }
-  __syncthreads();
-  // (2) selection, one warp per token
-  uint8_t* taken = taken_all + warp * E;
-  for (int t = warp; t < T; t += kTailWarps) {
-    const float* lrow = table + (size_t)t * ld;
-    for (int e = lane; e < E; e += 32) taken[e] = 0;
-    __syncwarp();
-    int my_idx = -1;
-    float my_l = 0.f;
-    for (int j = 0; j < k; ++j) {
-      float bv = -FLT_MAX;
-      int be = INT_MAX;
-      for (int e = lane; e < E; e += 32) {
-        const float sv = lrow[e] + (rt.bias != nullptr ? rt.bias[e] : 0.f);
-        if (!taken[e] && (be == INT_MAX || sv > bv)) bv = sv, be = e;
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) bv = ov, be = oe;
-      }
-      if (lane == 0) taken[be] = 1;
-      if (lane == j) my_idx = be, my_l = lrow[be];
-      __syncwarp();
-    }
-    float m = lane < k ? my_l : -FLT_MAX;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float ex = lane < k ? expf(my_l - m) : 0.f;
-    float z = ex;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-    if (lane < k) {
-      const float wv = ex / z;
-      rt.topk_idx[(size_t)t * k + lane] = my_idx;
-      rt.topk_w[(size_t)t * k + lane] = wv;
-      idx_s[t * k + lane] = my_idx;
-      w_s[t * k + lane] = wv;
-    }
-    __syncwarp();
-  }
-  // (3) dispatch: histogram, exclusive scan over experts, order-preserving scatter
-  for (int e = tid; e < E; e += kThreads) cnt[e] = 0;
-  __syncthreads();
-  for (int i = tid; i < n_items; i += kThreads) atomicAdd(&cnt[idx_s[i]], 1);
-  __syncthreads();
-  const int per = (E + kThreads - 1) / kThreads;  // thread tid owns experts [tid*per, tid*per + per)
-  const int lo = min(E, tid * per), hi = min(E, lo + per);
-  int sum = 0;
-  for (int e = lo; e < hi; ++e) sum += cnt[e];
-  int incl = sum;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  int before = 0;
-  for (int q = 0; q < warp; ++q) before += warp_tot[q];
-  int r0 = before + incl - sum;
-  for (int e = lo; e < hi; ++e) {
-    rt.counts[e] = cnt[e];
-    rt.offsets[e] = r0;
-    run[e] = r0;
-    r0 += cnt[e];
-  }
-  if (tid == kThreads - 1) rt.offsets[E] = before + incl;
-  __syncthreads();
-  if (warp == 0) {  // slots in (token, slot) order; equal experts ranked by lane
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int i0 = 0; i0 < n_items; i0 += 32) {
-      const int i = i0 + lane;
-      const int e = i < n_items ? idx_s[i] : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      if (e >= 0) {
-        const int r = run[e] + __popc(peers & lt_mask);
-        rt.perm_token[r] = i / k;
-        rt.inv_perm[i] = r;
-        rt.p_perm[r] = w_s[i];
-      }
-      __syncwarp();
-      if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
-      __syncwarp();
-    }
-  }
-  if (tid == 0) *rt.counter = 0;  // ready for the next launch
-}
-
 template <int KIND, int NT>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<KIND, NT>;
-  // streaming gate_up: the whole producer warp fills stages (lane 0 the weight copies, all lanes
-  // the gathered token rows), so each full barrier also counts the 32 lanes' arrivals
-  constexpr bool kWarpProducer = (NT > 0 && KIND == kGateUp);
-  constexpr int kGatherRows = NT > 0 ? NT : 4;  // token rows of one stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
@@ -325,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], kWarpProducer ? 33 : 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -384,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (kWarpProducer || lane == 0) {
+    if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -392,84 +235,45 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         const CUtensorMap* amap = &p.a_map[ti.set];
         const CUtensorMap* wmap = &p.w_map[ti.set];
         const int wbase = ti.gl * p.w_rows[ti.set];
-        // gathered token rows: this lane copies 16-byte chunk (lane & 7) of rows (lane >> 3) + 4 i
-        // of the segment's <= NT rows
-        const bool gather = kWarpProducer && p.gather_rows[ti.set] != nullptr;
-        int tok[kGatherRows / 4];
-        if constexpr (kWarpProducer) {
-#pragma unroll
-          for (int i = 0; i < kGatherRows / 4; ++i) {
-            const int j = (lane >> 3) + 4 * i;
-            tok[i] = (gather && j < ti.rows) ? p.gather_rows[ti.set][ti.row0 + j] : -1;
-          }
-        }
-        const uint32_t stage_bytes =
-            gather ? (uint32_t)(C::kStageBytes - kGatherRows * kBK * 2) : (uint32_t)C::kStageBytes;
         for (int kb = ti.kb0; kb < ti.kb1; ++kb, ++it) {
           const int stage = it % C::kStages;
-          bool got = lane != 0 || mbar_wait(&empty[stage], ((it / C::kStages) & 1) ^ 1, kWaitLimitNs);
-          if constexpr (kWarpProducer) got = __shfl_sync(0xffffffffu, got, 0);
-          if (!got) {
+          if (!mbar_wait(&empty[stage], ((it / C::kStages) & 1) ^ 1, kWaitLimitNs)) {
             ok = false;
             break;
           }
           uint8_t* sb = smem + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          if (p.withhold_first_load && it == 0) continue;  // the bytes never arrive
           const int kx = kb * kBK;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[stage], stage_bytes);
-            if (!(p.withhold_first_load && it == 0)) {  // withheld: the bytes never arrive
-              if constexpr (C::kTiled) {
-                tma_load_2d(amap, &full[stage], sb, kx, ti.row0 + ti.m * kBM);
-                if constexpr (KIND == kGateUp) {
-                  const int F = p.n_out[ti.set];
-                  tma_load_2d(wmap, &full[stage], sb + kTileBytesA, kx, wbase + ti.n * 128);
-                  tma_load_2d(wmap, &full[stage], sb + 2 * kTileBytesA, kx, wbase + F + ti.n * 128);
-                } else {
-                  tma_load_2d(wmap, &full[stage], sb + kTileBytesA, kx, wbase + ti.n * 256);
-                }
-              } else {
-                if constexpr (KIND == kGateUp) {
-                  const int F = p.n_out[ti.set];
-                  tma_load_2d(wmap, &full[stage], sb, kx, wbase + ti.n * 128);
-                  tma_load_2d(wmap, &full[stage], sb + kTileBytesA, kx, wbase + F + ti.n * 128);
-                  if (!gather) tma_load_2d(amap, &full[stage], sb + 2 * kTileBytesA, kx, ti.row0);
-                } else {
-                  tma_load_2d(wmap, &full[stage], sb, kx, wbase + ti.n * 128);
-                  tma_load_2d(amap, &full[stage], sb + kTileBytesA, kx, ti.row0);
-                }
-              }
-            }
-          }
-          if constexpr (kWarpProducer) {
-            if (gather) {
-              // rows past the segment are zero-filled (nothing is read for them)
-              const uint32_t tbase = smem_u32(sb + 2 * kTileBytesA);
-              const int c = lane & 7;
-              const uint16_t* src0 = p.gather_src[ti.set];
-              const int K = p.k_blocks[ti.set] * kBK;
-#pragma unroll
-              for (int i = 0; i < kGatherRows / 4; ++i) {
-                const int j = (lane >> 3) + 4 * i;
-                const uint32_t dst = tbase + (uint32_t)(j * 128 + ((c ^ (j & 7)) << 4));
-                const uint16_t* src = tok[i] >= 0 ? src0 + (size_t)tok[i] * K + kx + c * 8 : src0;
-                cp_async_16(dst, src, tok[i] >= 0 ? 16u : 0u);
-              }
-              cp_async_mbar_arrive_noinc(&full[stage]);
+          if constexpr (C::kTiled) {
+            tma_load_2d(amap, &full[stage], sb, kx, ti.row0 + ti.m * kBM);
+            if constexpr (KIND == kGateUp) {
+              const int F = p.n_out[ti.set];
+              tma_load_2d(wmap, &full[stage], sb + kTileBytesA, kx, wbase + ti.n * 128);
+              tma_load_2d(wmap, &full[stage], sb + 2 * kTileBytesA, kx, wbase + F + ti.n * 128);
             } else {
-              mbar_arrive(&full[stage]);
+              tma_load_2d(wmap, &full[stage], sb + kTileBytesA, kx, wbase + ti.n * 256);
+            }
+          } else {
+            if constexpr (KIND == kGateUp) {
+              const int F = p.n_out[ti.set];
+              tma_load_2d(wmap, &full[stage], sb, kx, wbase + ti.n * 128);
+              tma_load_2d(wmap, &full[stage], sb + kTileBytesA, kx, wbase + F + ti.n * 128);
+              tma_load_2d(amap, &full[stage], sb + 2 * kTileBytesA, kx, ti.row0);
+            } else {
+              tma_load_2d(wmap, &full[stage], sb, kx, wbase + ti.n * 128);
+              tma_load_2d(amap, &full[stage], sb + kTileBytesA, kx, ti.row0);
             }
           }
         }
       }
-      if (lane == 0) {
-        if (!ok) set_error(p.err, kErrTimeout);
-        // drain: every issued stage load must have landed before shared memory is released
-        const uint32_t issued = it;
-        for (int s = 0; s < C::kStages; ++s) {
-          if ((uint32_t)s >= issued) break;
-          const uint32_t last = issued - 1 - ((issued - 1 - s) % C::kStages);  // last index with it % S == s
-          if (!mbar_wait(&full[s], (last / C::kStages) & 1, kWaitLimitNs)) set_error(p.err, kErrTimeout);
-        }
+      if (!ok) set_error(p.err, kErrTimeout);
+      // drain: every issued stage load must have landed before shared memory is released
+      const uint32_t issued = it;
+      for (int s = 0; s < C::kStages; ++s) {
+        if ((uint32_t)s >= issued) break;
+        const uint32_t last = issued - 1 - ((issued - 1 - s) % C::kStages);  // last index with it % S == s
+        if (!mbar_wait(&full[s], (last / C::kStages) & 1, kWaitLimitNs)) set_error(p.err, kErrTimeout);
       }
     }
   } else if (warp == 1) {
@@ -493,7 +297,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             break;
           }
           tc_fence_after();
-          if constexpr (kWarpProducer) fence_proxy_async_smem();  // gathered rows came by cp.async
           const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -673,9 +476,6 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
-  if constexpr (KIND == kRouter && NT > 0) {
-    if (p.tail.counter != nullptr) router_tail(p, smem);
-  }
 }
 
 // ------------------------------------------------------------------------------ host side
@@ -720,15 +520,13 @@ int num_sms() {
 }
 
 template <int KIND, int NT>
-cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int* err, cudaStream_t s,
-                          const RouterTail* tail = nullptr) {
+cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int* err, cudaStream_t s) {
   using C = Cfg<KIND, NT>;
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.n_sets = n_sets;
   p.k_splits = k_splits;
   p.err = err;
-  if (KIND == kRouter && NT > 0 && tail != nullptr) p.tail = *tail;
   p.withhold_first_load = (KIND != kRouter && test_withhold_this_launch()) ? 1 : 0;
   const uint32_t a_box = C::kTiled ? kBM : NT;
   const uint32_t w_box = (C::kTiled && KIND != kGateUp) ? 256 : 128;
@@ -745,11 +543,6 @@ cudaError_t launch_kernel(const GemmSetHost* sets, int n_sets, int k_splits, int
     p.row_scale[i] = st.row_scale;
     p.ld_out[i] = st.ld_out > 0 ? st.ld_out : st.n_out;
     p.save_gu[i] = (KIND == kGateUp && NT == 0) ? st.save_gu : nullptr;
-    if (KIND == kGateUp && NT > 0) {
-      p.gather_rows[i] = st.gather_rows;
-      p.gather_src[i] = st.gather_src;
-      if ((st.gather_rows != nullptr) != (st.gather_src != nullptr)) return cudaErrorInvalidValue;
-    }
     p.n_groups[i] = st.n_groups;
     p.m_rows[i] = st.m_rows;
     p.n_out[i] = st.n_out;
@@ -821,28 +614,19 @@ int router_k_splits(int T, int D, int E, int num_sm) {
 
 int router_k_splits(int T, int D, int E) { return router_k_splits(T, D, E, num_sms()); }
 
-bool router_tail_fits(int T, int E, int k_splits) {
-  return T >= 1 && T <= 64 && (long long)T * router_ld(E) * 4 <= kTailTableBytes && k_splits >= 1 &&
-         k_splits <= kMaxSplits;
-}
-
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wg, int T, int D, int E, float* partials, int ld,
-                               int k_splits, int* err, cudaStream_t s, const RouterTail* tail) {
+                               int k_splits, int* err, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   GemmSetHost st;
   memset(&st, 0, sizeof(st));
   st.K = D, st.a = x, st.a_rows = T, st.w = wg, st.n_groups = 1, st.offsets = nullptr, st.m_rows = T;
   st.n_out = E, st.out = partials, st.row_scale = nullptr, st.ld_out = ld;
-  if (T > 64) return tail != nullptr ? cudaErrorInvalidValue : launch_kernel<kRouter, 0>(&st, 1, k_splits, err, s);
-  if (tail != nullptr && !router_tail_fits(T, E, k_splits)) return cudaErrorInvalidValue;
-  if (tail != nullptr && (tail->counter == nullptr || tail->T != T || tail->E != E || tail->k < 1 || tail->k > E ||
-                          tail->k > 32))
-    return cudaErrorInvalidValue;
+  if (T > 64) return launch_kernel<kRouter, 0>(&st, 1, k_splits, err, s);
   switch ((T + 15) / 16 * 16) {
-    case 16: return launch_kernel<kRouter, 16>(&st, 1, k_splits, err, s, tail);
-    case 32: return launch_kernel<kRouter, 32>(&st, 1, k_splits, err, s, tail);
-    case 48: return launch_kernel<kRouter, 48>(&st, 1, k_splits, err, s, tail);
-    default: return launch_kernel<kRouter, 64>(&st, 1, k_splits, err, s, tail);
+    case 16: return launch_kernel<kRouter, 16>(&st, 1, k_splits, err, s);
+    case 32: return launch_kernel<kRouter, 32>(&st, 1, k_splits, err, s);
+    case 48: return launch_kernel<kRouter, 48>(&st, 1, k_splits, err, s);
+    default: return launch_kernel<kRouter, 64>(&st, 1, k_splits, err, s);
   }
 }
 

@@ -13,7 +13,6 @@ namespace moe {
 constexpr int kErrBadIndex = 1;  // an expert id outside [0, E)
 constexpr int kErrTimeout = 2;   // a bounded device-side wait gave up
 constexpr size_t kWsHeader = 256;
-constexpr size_t kRouterTailCounter = 128;  // byte offset in the header: the fused decode router's counter
 
 // Wall-time limit of every spin-wait inside a kernel, measured on %globaltimer.  A context that
 // is descheduled for longer than this while a kernel waits (time-slicing with another process,
@@ -106,42 +105,18 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-// Fused tail of the decode router GEMM (streaming kRouter): top-k selection, weights and the
-// dispatch metadata, computed by the last CTA to finish (grouped_gemm_sm100.cu, router_tail).
-struct RouterTail {
-  int* counter;  // device int, zero when the launch starts (left zero)
-  const float* bias;
-  int T, E, k;
-  int32_t* topk_idx;
-  float* topk_w;
-  int32_t* counts;
-  int32_t* offsets;
-  int32_t* perm_token;
-  int32_t* inv_perm;
-  float* p_perm;
-};
-
 // ---- host launchers (defined in the .cu files) ---------------------------------------------
 // Router: logits on the tensor cores (split-K partial sums, [k_splits][T][ld] fp32, ld = E rounded
 // up to 32), then a warp-level top-k + softmax kernel that reduces the splits in a fixed order.
 int router_k_splits(int T, int D, int E);
-// whether the decode router's fused tail (RouterTail) can run: T <= 64 and its [T][ld] fp32 logit
-// table fits the tail's 64 KB of shared memory
-bool router_tail_fits(int T, int E, int k_splits);
 inline int router_ld(int E) { return (E + 31) / 32 * 32; }
 inline size_t router_scratch_bytes(int T, int D, int E) {
   return align_up((size_t)router_k_splits(T, D, E) * (size_t)T * router_ld(E) * sizeof(float), 256);
 }
 cudaError_t launch_router_gemm(const uint16_t* x, const uint16_t* wg, int T, int D, int E, float* partials, int ld,
-                               int k_splits, int* err, cudaStream_t s, const RouterTail* tail = nullptr);
+                               int k_splits, int* err, cudaStream_t s);
 cudaError_t launch_router_select(const float* partials, int k_splits, int T, int ld, const float* bias, int E, int k,
                                  int32_t* idx, float* w, cudaStream_t s);
-// One-CTA routing for a few tokens when x and W_g fit in shared memory (router_topk.cu): logits on
-// the CUDA cores, top-k and weights, and (counts != NULL) the dispatch metadata.
-bool router_small_fits(int T, int D, int E, int k);
-cudaError_t launch_router_small(const uint16_t* x, const uint16_t* wg, const float* bias, int T, int D, int E, int k,
-                                int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
-                                int32_t* perm_token, int32_t* inv_perm, float* p_perm, int* err, cudaStream_t s);
 
 cudaError_t launch_update_bias(const int32_t* counts, int E, float gamma, float* bias, cudaStream_t s);
 
@@ -169,10 +144,6 @@ struct GemmSetHost {
   const float* row_scale;   // per-row factor (down) or NULL
   int ld_out;               // output row stride in elements (0: n_out)
   uint16_t* save_gu = nullptr;  // tiled gate_up, training: also store g | u [rows, 2 * n_out] bf16
-  // streaming gate_up: gather the token rows from gather_src [*, K] by gather_rows (the
-  // permutation) instead of reading a (NULL: read a)
-  const int32_t* gather_rows = nullptr;
-  const uint16_t* gather_src = nullptr;
 };
 
 enum GemmKind { kGateUp = 0, kDown = 1, kRouter = 2 };

@@ -3,6 +3,9 @@
 // router_topk.cu, permute.cu, grouped_gemm_sm100.cu and combine.cu.
 #include <cstdint>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "grouped_gemm_wide.cuh"
 #include "router_aux.cuh"
@@ -175,15 +178,10 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
                      // optional shared expert over x[T, D]
                      const uint16_t* x, int T, int Fs, const uint16_t* sgu, const uint16_t* sdn, uint16_t* h_sh,
                      float* out_sh, int decode_nt, Tiling tiling, int* err, cudaStream_t s, cudaEvent_t ev_mid,
-                     unsigned ev_flags, uint16_t* save_gu = nullptr, uint16_t* save_gu_sh = nullptr,
-                     const int32_t* perm_token = nullptr) {
-  // perm_token (streaming only): the gate_up launch gathers its token rows from x by the
-  // permutation (x_perm is not read)
+                     unsigned ev_flags, uint16_t* save_gu = nullptr, uint16_t* save_gu_sh = nullptr) {
   GemmSetHost g[2] = {};
-  const bool gather = decode_nt > 0 && perm_token != nullptr;
-  g[0].K = D, g[0].a = gather ? x : x_perm, g[0].a_rows = gather ? T : M, g[0].w = gate_up, g[0].n_groups = E;
-  g[0].offsets = offsets, g[0].n_out = F, g[0].out = h, g[0].save_gu = save_gu;
-  if (gather) g[0].gather_rows = perm_token, g[0].gather_src = x;
+  g[0].K = D, g[0].a = x_perm, g[0].a_rows = M, g[0].w = gate_up, g[0].n_groups = E, g[0].offsets = offsets;
+  g[0].n_out = F, g[0].out = h, g[0].save_gu = save_gu;
   int n_sets = 1;
   if (Fs > 0) {
     g[1].K = D, g[1].a = x, g[1].a_rows = T, g[1].w = sgu, g[1].n_groups = 1, g[1].m_rows = T;
@@ -206,6 +204,59 @@ moe_status_t run_ffn(const uint16_t* x_perm, const int32_t* offsets, const float
     MOE_CUDA_TRY(launch_tiled((TileKind)tiling.dn, kDown, dn, n_sets, err, s));
   else
     MOE_CUDA_TRY(launch_grouped_gemm(kDown, dn, n_sets, decode_nt, err, s));
+  return MOE_OK;
+}
+
+// The shared expert of a prefill forward depends only on x, so it runs on a side stream while the
+// caller's stream routes and dispatches: a fork after the router GEMM and a join before the
+// combine (captured into a CUDA graph as two parallel branches like any cross-stream dependency).
+// One side stream and its two events per (device, caller stream), created on first use and kept
+// until the process exits.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+moe_status_t side_stream_for(cudaStream_t main, SideStream* out) {
+  static std::mutex mu;
+  static std::map<std::pair<int, cudaStream_t>, SideStream> table;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = table.find({dev, main});
+  if (it == table.end()) {
+    SideStream ss;
+    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    it = table.emplace(std::make_pair(dev, main), ss).first;
+  }
+  *out = it->second;
+  return MOE_OK;
+}
+
+// prefill forwards with a shared expert fork it onto the side stream (bf16 weights)
+bool fork_shared_expert(const moe_layer_desc_t& d) {
+  return d.Fs > 0 && !use_decode(d) && d.weight_format == MOE_WEIGHTS_BF16;
+}
+
+// The shared expert alone: gate_up (+ SwiGLU) then down over the T rows of x, one group each.
+moe_status_t run_shared_ffn(const uint16_t* x, int T, int D, int Fs, const uint16_t* sgu, const uint16_t* sdn,
+                            uint16_t* h_sh, float* out_sh, Tiling tiling, uint16_t* save_gu_sh, int* err,
+                            cudaStream_t s) {
+  GemmSetHost g = {};
+  g.K = D, g.a = x, g.a_rows = T, g.w = sgu, g.n_groups = 1, g.m_rows = T, g.n_out = Fs, g.out = h_sh;
+  g.save_gu = save_gu_sh;
+  MOE_CUDA_TRY(launch_tiled((TileKind)tiling.gu, kGateUp, &g, 1, err, s));
+  GemmSetHost dn = {};
+  dn.K = Fs, dn.a = h_sh, dn.a_rows = T, dn.w = sdn, dn.n_groups = 1, dn.m_rows = T, dn.n_out = D, dn.out = out_sh;
+  MOE_CUDA_TRY(launch_tiled((TileKind)tiling.dn, kDown, &dn, 1, err, s));
   return MOE_OK;
 }
 
@@ -243,44 +294,55 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
   const int splits = router_k_splits(T, D, E);
   const bool fp8 = d->weight_format == MOE_WEIGHTS_FP8_E4M3;
   const int nt = use_decode(*d) ? decode_tile(T) : 0;
-  // bf16 decode: the router GEMM's last CTA also selects and dispatches (no top-k or dispatch
-  // launch), and the gate_up launch gathers token rows from x itself (no x_perm)
-  // a few decode tokens whose x and W_g fit in shared memory: one CTA routes (and, for bf16,
-  // dispatches) on the CUDA cores
-  const bool small_router = nt > 0 && router_small_fits(T, D, E, k);
-  const bool fused_decode = nt > 0 && !fp8 && (small_router || router_tail_fits(T, E, splits));
-  if (fused_decode && small_router) {
-    MOE_CUDA_TRY(launch_router_small(x, d->w_gate, d->bias, T, D, E, k, I(w.topk_idx), Fp(w.topk_w), I(w.counts),
-                                     I(w.offsets), I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), err, s));
-    if (ev) MOE_CUDA_TRY(record(ev[1]));
-    if (ev) MOE_CUDA_TRY(record(ev[2]));
-  } else if (fused_decode) {
-    RouterTail tail = {};
-    tail.counter = reinterpret_cast<int*>(b + kRouterTailCounter);
-    tail.bias = d->bias, tail.T = T, tail.E = E, tail.k = k;
-    tail.topk_idx = I(w.topk_idx), tail.topk_w = Fp(w.topk_w), tail.counts = I(w.counts);
-    tail.offsets = I(w.offsets), tail.perm_token = I(w.perm_token), tail.inv_perm = I(w.inv_perm);
-    tail.p_perm = Fp(w.p_perm);
-    MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s, &tail));
-    if (ev) MOE_CUDA_TRY(record(ev[1]));
-    if (ev) MOE_CUDA_TRY(record(ev[2]));
-  } else {
-    if (small_router) {
-      MOE_CUDA_TRY(launch_router_small(x, d->w_gate, d->bias, T, D, E, k, I(w.topk_idx), Fp(w.topk_w), nullptr,
-                                       nullptr, nullptr, nullptr, nullptr, err, s));
-    } else {
-      MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s));
-      MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
-                                        Fp(w.topk_w), s));
+  // prefill with a shared expert: it runs on a side stream (forked after the router GEMM) and the
+  // routed GEMMs below leave it out
+  const bool fork = fork_shared_expert(*d);
+  SideStream side;
+  if (fork && (st = side_stream_for(s, &side)) != MOE_OK) return st;
+  // joins the side stream's branch back into `s` when armed: before the combine, or on an early
+  // error return (a capture of `s` must not end with an unjoined branch)
+  struct Join {
+    cudaStream_t s;
+    cudaEvent_t e;
+    bool armed = false;
+    bool wait() {
+      armed = false;
+      if (cudaStreamWaitEvent(s, e, 0) == cudaSuccess) return true;
+      cudaGetLastError();
+      return false;
     }
-    if (ev) MOE_CUDA_TRY(record(ev[1]));
-    // dispatch + gather (one kernel for T <= 256); the FP8 path gathers f16 rows and, for the
-    // shared expert, an f16 copy of x
-    MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), x, T, D, E, k, I(w.counts), I(w.offsets),
-                                I(w.perm_token), I(w.inv_perm), Fp(w.p_perm), H(w.x_perm), fp8,
-                                (fp8 && Fs > 0) ? H(w.x16) : nullptr, I(w.scratch), err, s, nullptr));
-    if (ev) MOE_CUDA_TRY(record(ev[2]));
+    ~Join() {
+      if (armed) wait();
+    }
+  } join{s, side.join};
+  MOE_CUDA_TRY(launch_router_gemm(x, d->w_gate, T, D, E, Fp(w.router), router_ld(E), splits, err, s));
+  if (fork) {
+    // the shared expert's branch: it needs only x, and the GEMMs it runs take the SMs the
+    // latency-bound top-k and dispatch kernels leave idle
+    if (cudaEventRecord(side.fork, s) != cudaSuccess || cudaStreamWaitEvent(side.stream, side.fork, 0) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    const moe_status_t sst =
+        run_shared_ffn(x, T, D, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh),
+                       prefill_tiling(d->flags), (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) ? H(w.gu_saved_sh) : nullptr,
+                       err, side.stream);
+    if (cudaEventRecord(side.join, side.stream) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    join.armed = true;  // `s` waits for the branch before the combine, or on any early return
+    if (sst != MOE_OK) return sst;
   }
+  MOE_CUDA_TRY(launch_router_select(Fp(w.router), splits, T, router_ld(E), d->bias, E, k, I(w.topk_idx),
+                                    Fp(w.topk_w), s));
+  if (ev) MOE_CUDA_TRY(record(ev[1]));
+  // dispatch + gather (one kernel for T <= 256); the FP8 path gathers f16 rows and, for the
+  // shared expert, an f16 copy of x
+  MOE_CUDA_TRY(launch_permute(I(w.topk_idx), Fp(w.topk_w), x, T, D, E, k, I(w.counts), I(w.offsets), I(w.perm_token),
+                              I(w.inv_perm), Fp(w.p_perm), H(w.x_perm), fp8, (fp8 && Fs > 0) ? H(w.x16) : nullptr,
+                              I(w.scratch), err, s, nullptr));
+  if (ev) MOE_CUDA_TRY(record(ev[2]));
   SplitBuf split;  // split-K buffers of the FP8 weight-streaming GEMMs
   if (w.split_partial_bytes > 0) {
     split.partial = Fp(w.split_partial);
@@ -312,14 +374,14 @@ moe_status_t layer_forward(const moe_layer_desc_t* d, const uint16_t* x, uint16_
     MOE_CUDA_TRY(launch_stream_fp8w(kDown, dn, ds, Fs > 0 ? 2 : 1, nt, split, err, s));
   } else {
   st = run_ffn(H(w.x_perm), I(w.offsets), Fp(w.p_perm), M, E, D, F, d->gate_up, d->down, H(w.h), Fp(w.out_perm), x,
-               T, Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, prefill_tiling(d->flags), err,
+               T, fork ? 0 : Fs, d->shared_gate_up, d->shared_down, H(w.h_sh), Fp(w.out_sh), nt, prefill_tiling(d->flags), err,
                s, ev ? ev[3] : nullptr,
                rec_flags, (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) ? H(w.gu_saved) : nullptr,
-               (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && Fs > 0 ? H(w.gu_saved_sh) : nullptr,
-               fused_decode ? I(w.perm_token) : nullptr);
+               (d->flags & MOE_FLAG_SAVE_FOR_BACKWARD) && Fs > 0 ? H(w.gu_saved_sh) : nullptr);
   if (st != MOE_OK) return st;
   }
   if (ev) MOE_CUDA_TRY(record(ev[4]));
+  if (join.armed && !join.wait()) return MOE_ERR_CUDA;
   MOE_CUDA_TRY(launch_combine(Fp(w.out_perm), I(w.inv_perm), Fs > 0 ? Fp(w.out_sh) : nullptr, T, D, k, y, s));
   if (ev) MOE_CUDA_TRY(record(ev[5]));
   return MOE_OK;
@@ -405,11 +467,6 @@ moe_status_t moe_router_topk(const moe_bf16_t* x, const moe_bf16_t* w_gate, cons
   float* part = reinterpret_cast<float*>(b + kWsHeader);
   const int splits = router_k_splits(T, D, E);
   cudaStream_t s = (cudaStream_t)stream;
-  if (router_small_fits(T, D, E, k)) {  // the layer's decode router, so both give the same bits
-    MOE_CUDA_TRY(launch_router_small(x, w_gate, bias, T, D, E, k, topk_idx, topk_w, nullptr, nullptr, nullptr,
-                                     nullptr, nullptr, reinterpret_cast<int*>(b), s));
-    return MOE_OK;
-  }
   MOE_CUDA_TRY(launch_router_gemm(x, w_gate, T, D, E, part, router_ld(E), splits, reinterpret_cast<int*>(b), s));
   MOE_CUDA_TRY(launch_router_select(part, splits, T, router_ld(E), bias, E, k, topk_idx, topk_w, s));
   return MOE_OK;
@@ -597,17 +654,11 @@ moe_status_t moe_layer_forward_host(const moe_layer_desc_t* desc, const moe_bf16
 
 int moe_layer_kernel_count(const moe_layer_desc_t* desc) {
   if (validate_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  const bool decode = use_decode(*desc);
-  const bool small = decode && router_small_fits(desc->T, desc->D, desc->E, desc->k);
-  // bf16 decode: one router kernel also selects and dispatches, gate_up gathers its rows itself
-  if (decode && desc->weight_format == MOE_WEIGHTS_BF16 &&
-      (small || router_tail_fits(desc->T, desc->E, router_k_splits(desc->T, desc->D, desc->E))))
-    return 1 /*router*/ + 2 /*GEMMs*/ + 1;
-  if (small) return 1 /*router*/ + 1 /*dispatch*/ + 2 + 1;  // E4M3 decode
   // T <= 256: one kernel sorts and gathers (and casts x for the FP8 path's shared expert, T <= 64);
   // above: hist, scan, scatter, gather
   const int dispatch = desc->T <= 256 ? 1 : 4;
-  return 2 /*router GEMM, top-k*/ + dispatch + 2 /*grouped GEMMs*/ + 1 /*combine*/;
+  const int gemms = fork_shared_expert(*desc) ? 4 : 2;  // the shared expert's own two on the side stream
+  return 2 /*router GEMM, top-k*/ + dispatch + gemms + 1 /*combine*/;
 }
 
 int moe_layer_gemm_path(const moe_layer_desc_t* desc) {

@@ -99,22 +99,6 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// ------------------------------------------------------------------------------ LSU copies
-// 16-byte global -> shared copy (L2 only, not L1); src_bytes < 16 zero-fills the rest (0: no read).
-__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes) : "memory");
-}
-// Arrive on `bar` once every cp.async this thread issued so far has landed; the arrival is one of
-// those the barrier was initialised to expect (noinc).
-__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// Order this thread's view of shared memory written by the generic proxy (plain or cp.async
-// stores) before later async-proxy reads (tcgen05.mma operands).
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // ------------------------------------------------------------------------------ tcgen05
 // TMEM allocation (whole warp).  The allocated base address is written to shared memory.
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

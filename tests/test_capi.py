@@ -88,10 +88,13 @@ def test_layer_workspace_size_and_small_workspace(L):
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100000, need - 1, None) == 4
     assert L.moe_layer_forward(ctypes.byref(d), 0x4000, 0x5000, 0x100010, need, None) == 3  # ws not 256-aligned
     assert L.moe_layer_forward(ctypes.byref(d), 0x4008, 0x5000, 0x100000, need, None) == 3
-    # T=16 (bf16 decode): the router GEMM also selects and dispatches; gate_up gathers its rows
-    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 4
-    # forced prefill at T=16: router GEMM, top-k, one kernel that sorts and gathers, 2 GEMMs, combine
-    assert L.moe_layer_kernel_count(ctypes.byref(_desc(flags=1))) == 6
+    # T=16: router GEMM, top-k, one kernel that sorts and gathers, 2 GEMMs, combine
+    assert L.moe_layer_kernel_count(ctypes.byref(d)) == 6
+    assert L.moe_layer_kernel_count(ctypes.byref(_desc(flags=1))) == 6  # forced prefill
+    # prefill with a shared expert: its own gate_up and down on the side stream
+    sh = dict(Fs=64, shared_gate_up=0x6000, shared_down=0x7000)
+    assert L.moe_layer_kernel_count(ctypes.byref(_desc(T=300, **sh))) == 11
+    assert L.moe_layer_kernel_count(ctypes.byref(_desc(T=16, **sh))) == 6  # decode: one launch for both sets
     # T=300 prefill: router GEMM, top-k, hist, scan, scatter, gather, 2 GEMMs, combine
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(T=300))) == 9
     assert L.moe_layer_kernel_count(ctypes.byref(_desc(k=9))) == 0
@@ -216,8 +219,9 @@ def test_backward_entry_validates_on_host(L):
     need_b = L.moe_layer_backward_workspace_size(ctypes.byref(d))
     need_f = L.moe_layer_workspace_size(ctypes.byref(d))
     assert need_b > 256 and need_b % 256 == 0
-    # the training forward keeps g | u: its workspace grows by T*k*2F bf16
-    assert need_f >= L.moe_layer_workspace_size(ctypes.byref(plain)) + 16 * 2 * 2 * 128 * 2
+    # the training forward keeps g | u: its workspace grows by T*k*2F bf16 over a (prefill) forward
+    prefill = _desc(flags=moe.MOE_FLAG_FORCE_PREFILL)
+    assert need_f >= L.moe_layer_workspace_size(ctypes.byref(prefill)) + 16 * 2 * 2 * 128 * 2
     assert L.moe_layer_kernel_count(ctypes.byref(d)) == 6  # tiled kernels at T = 16, separate combine
     g = moe.LayerGrads(0x10000, 0x20000, 0x30000, None, None)
     args = (0x4000, 0x5000, 0x6000, ctypes.byref(g), 0x100000, need_f, 0x200000, need_b, None)
