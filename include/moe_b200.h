@@ -256,7 +256,13 @@ moe_status_t moe_quantize_rows_fp8(const moe_bf16_t* w, int64_t rows, int K, uin
 size_t moe_layer_workspace_size(const moe_layer_desc_t* desc);
 
 /* x [T, D] bf16 (device) -> y [T, D] bf16 (device).  Clears the workspace's error word (and the
- * split-K counters that follow it) first, with one memset on `stream`. */
+ * split-K counters that follow it) first, with one memset on `stream`.
+ * Prefill (T > 64, bf16 weights) with a shared expert runs the shared expert's two GEMMs on a side
+ * stream owned by the library -- one per (device, caller stream), with two events, created on the
+ * first such call and kept until the process exits -- forked from `stream` after the router GEMM
+ * and joined back before the combine.  All work still completes in `stream` order; under stream
+ * capture the graph gets two parallel branches.  Make the first such call on each stream before
+ * capturing it. */
 moe_status_t moe_layer_forward(const moe_layer_desc_t* desc, const moe_bf16_t* x, moe_bf16_t* y,
                                void* ws, size_t ws_bytes, moe_stream_t stream);
 

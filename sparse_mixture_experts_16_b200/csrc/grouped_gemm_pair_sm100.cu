@@ -67,6 +67,7 @@ struct alignas(64) PairParams {
   CUtensorMap t_map128[2];  // the same tensor, box 64 K x 128 rows (a full token half in one copy)
   CUtensorMap w_map[2];     // weights per set: down [rows, K], box 64 K x 128 rows; gate_up viewed as
                             // [groups][2 halves][F rows][K], box 64 K x 64 rows x 2 halves
+  CUtensorMap o_map[2];     // down: fp32 output [rows, D], box 32 columns x 32 rows (TMA stores)
   const int32_t* offsets[2];
   void* out[2];             // gate_up: bf16 h [rows, F]; down: fp32 [rows, D]
   const float* row_scale[2];
@@ -151,6 +152,19 @@ __device__ __forceinline__ bool p_epi_any(bool pred) {
 __device__ __forceinline__ void p_st_shared_f32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+// TMA bulk store of a box from shared memory, tracked in this thread's bulk group
+__device__ __forceinline__ void p_tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void p_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void p_bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void p_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ float4 p_ld_shared_f4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -348,48 +362,74 @@ __global__ void __launch_bounds__(kPThreads, 1) grouped_gemm_pair_kernel(const _
       const int n_out = p.n_out[ti.set];
       const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + buf * kPT;
       const size_t trow = (size_t)ti.row0 + (size_t)ti.m * kPT;
+      if constexpr (KIND == kDown) {
+        // Each warp owns 32 output columns (its TMEM lanes) x 32 tokens per chunk: it scales them by
+        // the tokens' router weights, stages them densely ([token][column], conflict-free) in its
+        // own 4 KB of shared memory and writes them with one TMA bulk store.  A chunk that runs past
+        // the segment (or a column block past the tensor) is stored directly instead: one coalesced
+        // 128-byte row segment per instruction, never a box reaching into another segment's rows.
+        const int c_warp = ti.n * 256 + (int)rank * 128 + q * 32;
+        const float* rs = p.row_scale[ti.set];
+        float* out = static_cast<float*>(p.out[ti.set]);
+        const uint32_t wstg = stage_base + (uint32_t)q * 4096u;
 #pragma unroll 1
-      for (int j0 = 0; j0 < nr; j0 += kPChunk) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tacc + j0, v);
-        tmem_ld_wait();
-        p_epi_sync();  // the previous chunk's readers are done with the stage
+        for (int j0 = 0; j0 < nr; j0 += kPChunk) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tacc + j0, v);
+          tmem_ld_wait();
+          const int nj = min(kPChunk, nr - j0);
+          const float pv = (rs != nullptr && lane < nj) ? rs[trow + j0 + lane] : 1.0f;
+          if (c_warp >= n_out) continue;  // this warp's columns lie past the tensor (D % 256 != 0)
+          if (nj == kPChunk && c_warp + 32 <= n_out) {
+            if (lane == 0) p_bulk_wait_read_all();  // the previous chunk's store has read the staging
+            __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) p_st_shared_f32(st_col + (uint32_t)(j * kPPitch) * 4, v[j]);
-        p_epi_sync();
-        if (j0 + j_in < nr) {
-          const size_t grow = trow + j0 + j_in;
-          if constexpr (KIND == kGateUp) {
-            const int c_base = ti.n * 128 + (int)rank * 64;
-            if (c_base < n_out) {
-              uint16_t* hrow = static_cast<uint16_t*>(p.out[ti.set]) + grow * n_out + c_base;
-              uint16_t* srow =
-                  p.save_gu[ti.set] != nullptr ? p.save_gu[ti.set] + grow * 2 * n_out + c_base : nullptr;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int c = part * 4 + i * 16;
-                const float4 g = p_ld_shared_f4(ld_row + c * 4);
-                const float4 u = p_ld_shared_f4(ld_row + (64 + c) * 4);
-                *reinterpret_cast<uint2*>(hrow + c) =
-                    make_uint2(pack_bf16x2(p_silu_mul(g.x, u.x), p_silu_mul(g.y, u.y)),
-                               pack_bf16x2(p_silu_mul(g.z, u.z), p_silu_mul(g.w, u.w)));
-                if (srow != nullptr) {  // the backward pass's SwiGLU inputs
-                  *reinterpret_cast<uint2*>(srow + c) = make_uint2(pack_bf16x2(g.x, g.y), pack_bf16x2(g.z, g.w));
-                  *reinterpret_cast<uint2*>(srow + n_out + c) =
-                      make_uint2(pack_bf16x2(u.x, u.y), pack_bf16x2(u.z, u.w));
-                }
-              }
+            for (int j = 0; j < 32; ++j)
+              p_st_shared_f32(wstg + (uint32_t)(j * 128 + lane * 4),
+                              __float_as_uint(__uint_as_float(v[j]) * __shfl_sync(0xffffffffu, pv, j)));
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic stores -> the TMA's reads
+            __syncwarp();
+            if (lane == 0) {
+              p_tma_store_2d(&p.o_map[ti.set], wstg, c_warp, (int32_t)(trow + j0));
+              p_bulk_commit();
             }
           } else {
-            const int c_base = ti.n * 256 + (int)rank * 128;
-            float* orow = static_cast<float*>(p.out[ti.set]) + grow * n_out + c_base;
-            const float sc = p.row_scale[ti.set] != nullptr ? p.row_scale[ti.set][grow] : 1.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int j = 0; j < 32; ++j) {
+              const float sc = __shfl_sync(0xffffffffu, pv, j);
+              if (j < nj && c_warp + lane < n_out)
+                out[(trow + j0 + j) * n_out + c_warp + lane] = __uint_as_float(v[j]) * sc;
+            }
+          }
+        }
+      } else {
+        // gate_up: the pair's 64 g and 64 u columns of each 32-token chunk go through a padded
+        // [token][column] staging area so that each thread writes 4 h values of one token row
+#pragma unroll 1
+        for (int j0 = 0; j0 < nr; j0 += kPChunk) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tacc + j0, v);
+          tmem_ld_wait();
+          p_epi_sync();  // the previous chunk's readers are done with the stage
+#pragma unroll
+          for (int j = 0; j < 32; ++j) p_st_shared_f32(st_col + (uint32_t)(j * kPPitch) * 4, v[j]);
+          p_epi_sync();
+          const int c_base = ti.n * 128 + (int)rank * 64;
+          if (j0 + j_in < nr && c_base < n_out) {
+            const size_t grow = trow + j0 + j_in;
+            uint16_t* hrow = static_cast<uint16_t*>(p.out[ti.set]) + grow * n_out + c_base;
+            uint16_t* srow = p.save_gu[ti.set] != nullptr ? p.save_gu[ti.set] + grow * 2 * n_out + c_base : nullptr;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
               const int c = part * 4 + i * 16;
-              if (c_base + c < n_out) {
-                const float4 a = p_ld_shared_f4(ld_row + c * 4);
-                *reinterpret_cast<float4*>(orow + c) = make_float4(a.x * sc, a.y * sc, a.z * sc, a.w * sc);
+              const float4 g = p_ld_shared_f4(ld_row + c * 4);
+              const float4 u = p_ld_shared_f4(ld_row + (64 + c) * 4);
+              *reinterpret_cast<uint2*>(hrow + c) =
+                  make_uint2(pack_bf16x2(p_silu_mul(g.x, u.x), p_silu_mul(g.y, u.y)),
+                             pack_bf16x2(p_silu_mul(g.z, u.z), p_silu_mul(g.w, u.w)));
+              if (srow != nullptr) {  // the backward pass's SwiGLU inputs
+                *reinterpret_cast<uint2*>(srow + c) = make_uint2(pack_bf16x2(g.x, g.y), pack_bf16x2(g.z, g.w));
+                *reinterpret_cast<uint2*>(srow + n_out + c) = make_uint2(pack_bf16x2(u.x, u.y), pack_bf16x2(u.z, u.w));
               }
             }
           }
@@ -398,6 +438,9 @@ __global__ void __launch_bounds__(kPThreads, 1) grouped_gemm_pair_kernel(const _
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));  // release to the MMA issuer
+    }
+    if constexpr (KIND == kDown) {
+      if (lane == 0) p_bulk_wait_all();  // every output store of this warp has been performed
     }
   }
 
@@ -459,6 +502,19 @@ bool p_make_gate_up_map(CUtensorMap* m, const void* base, int groups, int F, int
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 row-major [rows, cols] output map for the down's TMA stores: box 32 columns x 32 rows
+bool p_make_out_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols) {
+  PEncodeFn enc = p_encode_fn();
+  if (enc == nullptr || rows == 0 || cols == 0) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // clusters of two that fit on the device at once (the persistent grid is twice this)
 template <int KIND>
 int pair_clusters() {
@@ -505,6 +561,10 @@ cudaError_t launch_pair(const GemmSetHost* sets, int n_sets, int* err, cudaStrea
     if (KIND == kGateUp ? !p_make_gate_up_map(&p.w_map[i], st.w, st.n_groups, st.n_out, st.K)
                         : !p_make_map(&p.w_map[i], st.w, (uint64_t)st.n_groups * p.w_rows[i], (uint64_t)st.K, 128))
       return cudaErrorInvalidValue;
+    if (KIND == kDown) {
+      const uint64_t out_rows = st.offsets != nullptr ? (uint64_t)st.a_rows : (uint64_t)st.m_rows;
+      if (!p_make_out_map(&p.o_map[i], st.out, out_rows, (uint64_t)st.n_out)) return cudaErrorInvalidValue;
+    }
     p.offsets[i] = st.offsets;
     p.out[i] = st.out;
     p.row_scale[i] = KIND == kDown ? st.row_scale : nullptr;
