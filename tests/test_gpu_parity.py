@@ -318,6 +318,39 @@ def test_decode_layer_equals_the_step_by_step_path_bit_for_bit(w):
     assert rel_rms_err(bf16_np_to_f64(y_layer), y_ref) <= REL_RMS_TOL
 
 
+PREFILL_STEP_CASES = [
+    W(300, 256, 8, 2, 128, bias="zipf:1.1"),               # ragged last tiles, one segment > 128 rows
+    W(520, 512, 32, 4, 256, Fs=128, bias="normal:0.5"),    # with the shared expert (side stream)
+    W(257, 128, 64, 8, 64, bias="zipf:1.1"),               # empty experts, multi-block dispatch
+]
+
+
+@pytest.mark.parametrize("w", PREFILL_STEP_CASES, ids=lambda w: w.name)
+def test_prefill_layer_equals_the_step_by_step_path_bit_for_bit(w):
+    """The prefill layer forward (the shared expert on its side stream) and the step-by-step entry
+    points (router, permute, grouped FFN on x_perm with the same default tiling, the shared expert
+    as a one-segment grouped FFN, combine) are the same computation and must give the same bits."""
+    import torch
+
+    inp, _ = host_case(w)
+    d = device_from_host(inp)
+    L = layer_from(d, w.k)
+    assert L.kernel_count(w.T) == 2 + 4 + (4 if w.Fs else 2) + 1  # hist, scan, scatter, gather
+    y_layer = to_np_bf16(L(d["x"]))
+    assert L.device_error() == 0
+    idx, p = moe.moe_router_topk(d["x"], d["wg"], d["bias"], w.k)
+    pm = moe.moe_permute(idx, p, d["x"], w.E)
+    out_perm, _ = moe.moe_grouped_swiglu_ffn(pm["x_perm"], pm["offsets"], pm["p_perm"], d["gate_up"], d["down"])
+    shared = None
+    if w.Fs:
+        off = torch.tensor([0, w.T], dtype=torch.int32, device="cuda")
+        shared, _ = moe.moe_grouped_swiglu_ffn(d["x"], off, None, d["shared_gate_up"][None], d["shared_down"][None])
+    y_steps = to_np_bf16(moe.moe_combine(out_perm, pm["inv_perm"], shared, w.T, w.k))
+    assert (y_layer == y_steps).all()
+    y_ref, _, _ = oracle_layer(inp, w.k)
+    assert rel_rms_err(bf16_np_to_f64(y_layer), y_ref) <= REL_RMS_TOL
+
+
 def test_layer_host_buffers_match_device_buffers():
     import torch
 
