@@ -86,25 +86,52 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ block_
   pdl_trigger();
 }
 
-// One warp per block of 256 tokens; order-preserving ranks.
-__global__ void __launch_bounds__(32) scatter_kernel(const int32_t* __restrict__ idx, const float* __restrict__ w,
-                                                     int T, int E, int k, const int32_t* __restrict__ block_off,
-                                                     const int32_t* __restrict__ offsets,
-                                                     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm,
-                                                     float* __restrict__ p_perm) {
-  extern __shared__ int run[];  // next free row per expert
-  const int lane = threadIdx.x;
+// One block of 8 warps per 256 tokens; warp w ranks the slots of tokens [32w, 32w + 32) of the
+// block.  Order-preserving: a first pass counts each warp's slots per expert, the warps' counts
+// are prefix-summed in warp order on top of the block's offset, and a second pass hands out rows
+// in slot order (lanes in order within a 32-slot group via __match_any_sync, groups in order).
+constexpr int kScatterWarps = kTokPerBlock / 32;
+
+__global__ void __launch_bounds__(kScatterWarps * 32) scatter_kernel(const int32_t* __restrict__ idx,
+                                                                     const float* __restrict__ w, int T, int E, int k,
+                                                                     const int32_t* __restrict__ block_off,
+                                                                     const int32_t* __restrict__ offsets,
+                                                                     int32_t* __restrict__ perm_token,
+                                                                     int32_t* __restrict__ inv_perm,
+                                                                     float* __restrict__ p_perm) {
+  extern __shared__ int run_all[];  // [warp][E]: the warp's count, then its next free row per expert
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int* run = run_all + warp * E;
+  for (int e = lane; e < E; e += 32) run[e] = 0;
   pdl_wait();
-  for (int e = lane; e < E; e += 32) run[e] = offsets[e] + block_off[(size_t)blockIdx.x * E + e];
   __syncwarp();
   const int t0 = blockIdx.x * kTokPerBlock;
-  const int n_items = min(T - t0, kTokPerBlock) * k;
+  const int n_tok = min(T - t0, kTokPerBlock);
+  const int i_lo = min(warp * 32, n_tok) * k, i_hi = min(warp * 32 + 32, n_tok) * k;
   const size_t base = (size_t)t0 * k;
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int i0 = 0; i0 < n_items; i0 += 32) {
+  for (int i0 = i_lo; i0 < i_hi; i0 += 32) {  // pass 1: this warp's slots per expert
+    const int i = i0 + lane;
+    int e = i < i_hi ? idx[base + i] : -1;
+    if ((unsigned)e >= (unsigned)E) e = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == 31 - __clz(peers)) run[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {  // warp-order prefix on the block's offset
+    int r = offsets[e] + block_off[(size_t)blockIdx.x * E + e];
+    for (int v = 0; v < kScatterWarps; ++v) {
+      const int c = run_all[v * E + e];
+      run_all[v * E + e] = r;
+      r += c;
+    }
+  }
+  __syncthreads();
+  for (int i0 = i_lo; i0 < i_hi; i0 += 32) {  // pass 2: rows in slot order
     const int i = i0 + lane;
     int e = -1;
-    if (i < n_items) {
+    if (i < i_hi) {
       e = idx[base + i];
       if ((unsigned)e >= (unsigned)E) {
         inv_perm[base + i] = -1;  // dropped slot (error already recorded by hist_kernel)
@@ -344,7 +371,8 @@ cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16
   if (e != cudaSuccess) return e;
   ++launches;
   if (nb > 0) {
-    e = launch_pdl(scatter_kernel, dim3(nb), dim3(32), E * sizeof(int), s, idx, topk_w, T, E, k,
+    e = launch_pdl(scatter_kernel, dim3(nb), dim3(kScatterWarps * 32), kScatterWarps * E * sizeof(int), s, idx,
+                   topk_w, T, E, k,
                    (const int32_t*)scratch, (const int32_t*)offsets, perm_token, inv_perm, p_perm);
     if (e != cudaSuccess) return e;
     ++launches;
