@@ -339,7 +339,11 @@ moe_status_t moe_layer_expert_counts(const moe_layer_desc_t* desc, void* ws, siz
                                      const int32_t** counts);
 
 /* Synchronises `stream`, returns the status held in the workspace's error word (MOE_OK,
- * MOE_ERR_DEVICE_INDEX or MOE_ERR_TIMEOUT) and clears it. */
+ * MOE_ERR_DEVICE_INDEX or MOE_ERR_TIMEOUT) and clears it.  MOE_ERR_TIMEOUT: a pipeline wait
+ * inside a GEMM kernel gave up after 1 s of wall-clock time (the GPU's global timer); the kernel
+ * then drained its own copies, freed its tensor memory and returned, and that launch's outputs
+ * are invalid.  A context kept off the GPU for longer than that (time slicing, preemption) can
+ * report it spuriously. */
 moe_status_t moe_get_device_error(void* ws, moe_stream_t stream);
 
 /* Static, human-readable name of a status. */
