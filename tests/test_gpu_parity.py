@@ -121,7 +121,8 @@ def _check_permute(idx, w_np, x_np, E, got):
 
 
 @pytest.mark.parametrize("T,E,k,D", [(1, 4, 2, 64), (255, 8, 2, 128), (256, 8, 2, 128), (1000, 33, 3, 64),
-                                     (777, 256, 8, 192), (300, 1024, 4, 64)])
+                                     (777, 256, 8, 192), (300, 1024, 4, 64), (513, 64, 32, 64),
+                                     (8192, 256, 8, 64)])
 def test_permute_parity_random_routing(T, E, k, D):
     import torch
 
@@ -147,6 +148,35 @@ def test_permute_edge_cases_empty_and_overfull_experts():
     # metadata only (x = None)
     got2 = moe.moe_permute(torch.from_numpy(idx).cuda(), torch.from_numpy(wts).cuda(), None, E)
     assert (got2["perm_token"].cpu().numpy() == got["perm_token"].cpu().numpy()).all()
+
+
+def test_multi_block_permute_drops_out_of_range_ids_and_keeps_the_rest_in_order():
+    """Above 256 tokens the dispatch runs as histogram, scan and scatter kernels.  Slots whose
+    expert id is outside [0, E) get inv_perm -1 and no row; every other slot keeps the order the
+    oracle gives it, counted over the valid slots only."""
+    import torch
+
+    T, E, k = 600, 12, 3
+    rng = np.random.default_rng(5)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    bad = rng.random((T, k)) < 0.05
+    idx_bad = np.where(bad, np.where(rng.random((T, k)) < 0.5, -1, E + 3), idx).astype(np.int32)
+    wts = rng.random((T, k)).astype(np.float32)
+    got = moe.moe_permute(torch.from_numpy(idx_bad).cuda(), torch.from_numpy(wts).cuda(), None, E)
+    assert moe.moe_get_device_error(got["ws"]) == 6  # MOE_ERR_DEVICE_INDEX
+    inv = got["inv_perm"].cpu().numpy().reshape(T, k)
+    assert (inv[bad] == -1).all()
+    # the valid slots in (token, slot) order, stably sorted by expert, are the permutation
+    slots = np.flatnonzero(~bad.reshape(-1))
+    e_valid = idx.reshape(-1)[slots]
+    order = slots[np.argsort(e_valid, kind="stable")]
+    counts = np.bincount(e_valid, minlength=E)
+    assert (got["counts"].cpu().numpy() == counts).all()
+    assert (got["offsets"].cpu().numpy() == np.concatenate([[0], np.cumsum(counts)])).all()
+    n = len(order)
+    assert (got["perm_token"].cpu().numpy()[:n] == order // k).all()
+    assert (inv.reshape(-1)[order] == np.arange(n)).all()
+    assert (got["p_perm"].cpu().numpy()[:n] == wts.reshape(-1)[order]).all()
 
 
 def test_permute_reports_out_of_range_ids_without_faulting():
