@@ -334,6 +334,17 @@ class MoELayer:
             self._ws = torch.zeros(need, dtype=torch.uint8, device=self.w_gate.device)
         return self._ws
 
+    def new_workspace(self, T: int):
+        """A workspace of its own for T tokens: forwards that may overlap (on different streams)
+        each need one."""
+        import torch
+
+        d = self.desc(T)
+        need = lib().moe_layer_workspace_size(ctypes.byref(d))
+        if need == 0:
+            raise MoeError(1, "moe_layer_workspace_size")
+        return torch.zeros(need, dtype=torch.uint8, device=self.w_gate.device)
+
     def kernel_count(self, T: int) -> int:
         d = self.desc(T)
         return lib().moe_layer_kernel_count(ctypes.byref(d))
@@ -363,10 +374,11 @@ class MoELayer:
 
     __call__ = forward
 
-    def forward_host(self, x_host, y_host, stream=None):
-        """x_host / y_host: pinned CPU bf16 tensors [T, D]; asynchronous on the stream."""
+    def forward_host(self, x_host, y_host, stream=None, ws=None):
+        """x_host / y_host: pinned CPU bf16 tensors [T, D]; asynchronous on the stream.  ``ws``:
+        a workspace from new_workspace() (default: the layer's own)."""
         T = x_host.shape[0]
-        ws = self.workspace(T)
+        ws = self.workspace(T) if ws is None else ws
         d = self.desc(T)
         _check(lib().moe_layer_forward_host(ctypes.byref(d), x_host.data_ptr(), y_host.data_ptr(), ws.data_ptr(),
                                             ws.numel(), _stream(stream)), "moe_layer_forward_host")

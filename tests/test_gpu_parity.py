@@ -396,6 +396,31 @@ def test_layer_host_buffers_match_device_buffers():
     assert (yh.view(torch.int16).numpy().view(np.uint16) == y_dev).all()
 
 
+def test_overlapping_host_forwards_on_two_streams_give_the_same_bits():
+    """Double-buffered use of the public API: forwards alternate between two streams, each with
+    its own workspace and output buffer, so they overlap on the GPU (copies against compute, and
+    compute against compute).  The library keeps no state shared between them: every output
+    equals the single-stream forward bit for bit, including the shared expert's side streams."""
+    import torch
+
+    w = W(700, 256, 16, 4, 256, Fs=128, bias="normal:0.5")
+    inp, _ = host_case(w)
+    d = device_from_host(inp)
+    L = layer_from(d, w.k)
+    y_ref = to_np_bf16(L(d["x"]))
+    xh = d["x"].cpu().pin_memory()
+    streams = (torch.cuda.Stream(), torch.cuda.Stream())
+    wss = (L.new_workspace(w.T), L.new_workspace(w.T))
+    outs = [torch.empty_like(xh).pin_memory() for _ in range(6)]
+    for i, yh in enumerate(outs):
+        L.forward_host(xh, yh, stream=streams[i % 2], ws=wss[i % 2])
+    torch.cuda.synchronize()
+    for yh in outs:
+        assert (yh.view(torch.int16).numpy().view(np.uint16) == y_ref).all()
+    for ws in wss:
+        assert moe.moe_get_device_error(ws) == 0
+
+
 def test_layer_timed_records_six_events():
     import torch
 
