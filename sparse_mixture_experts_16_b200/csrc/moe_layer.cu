@@ -20,19 +20,19 @@ constexpr int kDecodeTMax = 64;  // T <= this runs the weight-streaming kernels
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 moe_status_t check_device() {
-  static int verdict[64];  // 0 unknown, 1 ok, 2 bad
+  static int arch_state[64];  // per device: 0 unchecked, 1 sm_100, 2 other
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
     cudaGetLastError();
     return MOE_ERR_NO_DEVICE;
   }
-  if (dev < 64 && verdict[dev] == 1) return MOE_OK;
+  if (dev < 64 && arch_state[dev] == 1) return MOE_OK;
   int major = 0;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_NO_DEVICE;
   }
-  if (dev < 64) verdict[dev] = major == 10 ? 1 : 2;
+  if (dev < 64) arch_state[dev] = major == 10 ? 1 : 2;
   return major == 10 ? MOE_OK : MOE_ERR_NO_DEVICE;
 }
 
