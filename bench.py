@@ -42,15 +42,19 @@ _CSRC = "sparse_mixture_experts_16_b200/csrc/"
 _TRAFFIC = {
     # kernel variant -> (its sources, their sha256, {workload: dram__bytes_read.sum + dram__bytes_write.sum})
     "bf16": ((_CSRC + "grouped_gemm_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
-             "524599bd67b9b6b8deba6af1a7841ddec43f7e8250f30be76b353018d5a9bdf3",
-             {"mixtral": 1.947595e9 + 0.226813e9, "deepseek_decode": 5.876610e9 + 0.003743e9}),
+             "2e3ae53b44d3235d0095eefe97ed358d6e2a12d467004f17987109881b1ff788",
+             {"deepseek": 16.356915e9 + 0.266861e9, "mixtral": 1.946758e9 + 0.226422e9,
+              "gptoss": 1.250717e9 + 0.177929e9, "gptoss_decode_T1": 0.135693e9 + 0.003688e9,
+              "gptoss_decode_T8": 0.707940e9 + 0.003672e9, "gptoss_decode_T32": 1.076501e9 + 0.004444e9,
+              "gptoss_decode_T64": 1.078004e9 + 0.004551e9, "deepseek_decode": 5.876497e9 + 0.004061e9}),
     "bf16_wide": ((_CSRC + "grouped_gemm_wide_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
                   "", {}),
     "bf16_pair": ((_CSRC + "grouped_gemm_pair_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
                   "", {}),
     "fp8": ((_CSRC + "stream_fp8w_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
-            "90184c605698454c7e2560af3fdb691544ae668cddf7910ea71752c9dc8e3252",
-            {"deepseek_decode": 2.942079e9 + 0.003725e9, "gptoss_decode_T64": 0.556999e9 + 0.004705e9}),
+            "fc2cfda7d3d5a31b0b7b6b8abce333afa5af1632c38be3817c2e48fc4ea5a7c3",
+            {"deepseek_decode": 2.942542e9 + 0.003802e9, "gptoss_decode_T1": 0.067338e9 + 0.001457e9,
+             "gptoss_decode_T8": 0.364154e9 + 0.003587e9, "gptoss_decode_T64": 0.556272e9 + 0.004443e9}),
 }
 
 
