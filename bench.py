@@ -465,13 +465,6 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
                                 f"{clocks.get('samples_power_capped', 0)} capped samples)"),
                 "frac_of_burst_peak": round(achieved / pk["bf16_tflops"], 4),
                 "frac_of_sustained_peak": round(achieved / pk["bf16_tflops_sustained"], 4)}
-        if clocks.get("sm_mhz") and clocks.get("sm_max_mhz") and clocks.get("samples_under_load", 0) >= 5:
-            # the burst figure scaled to the median SM clock sampled under load (tensor throughput
-            # is proportional to the clock); a coarse figure from 200 ms samples, so only given
-            # when at least five of them fell under load
-            at_clk = pk["bf16_tflops"] * clocks["sm_mhz"] / clocks["sm_max_mhz"]
-            roof["peak_at_sampled_clock"] = round(at_clk, 1)
-            roof["frac_at_sampled_clock"] = round(achieved / at_clk, 4)
     layer_tflops = w.flops / (ms_per_step / 1e3) / 1e12 * world
     layer_gbs = active_weight_bytes(w, n_active, "all", args.weights) / (ms_per_step / 1e3) / 1e9
 
