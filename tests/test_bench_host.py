@@ -56,6 +56,16 @@ def test_traffic_is_reported_only_for_captured_workloads(bench):
     assert bench.measured_traffic("deepseek", "bf16_wide") is None
 
 
+def test_headline_traffic_is_current_and_near_the_algorithmic_bytes(bench):
+    """The default workload's gate_up capture matches the kernel sources as they are (else the
+    line reports null), and its DRAM bytes sit within 5% above the algorithmic ones: the weights
+    256 x 4096 x 7168 bf16 plus x_perm 65536 x 7168 bf16 read, h 65536 x 2048 bf16 written."""
+    v = bench.measured_traffic("deepseek")
+    assert v is not None
+    algorithmic = (256 * 4096 * 7168 + 65536 * 7168) * 2 + 65536 * 2048 * 2
+    assert algorithmic <= v <= 1.05 * algorithmic
+
+
 def test_tiling_option_maps_to_the_layer_flags(bench):
     import sparse_mixture_experts_16_b200 as moe
 
