@@ -180,6 +180,26 @@ class ClockSampler:
                 "samples_power_capped": capped, "power_w_max": max(r["power"] for r in rows)}
 
 
+def max_over_ranks(vals, dev, world: int):
+    """Each value's maximum over the ranks, from one all-reduce (every rank calls this at the same
+    point, with the same number of values).  One rank: the values unchanged."""
+    vals = [float(v) for v in vals]
+    if world <= 1:
+        return vals
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(vals, device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Tokens per second of the whole job: every rank ran `steps` steps of `tokens_per_step`
+    tokens, and the job took as long as its slowest rank (`max_ms`, summed over the steps)."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
 def tensor_peak(pk: dict, clocks: dict, timed_s: float):
     """The bf16 peak that matches the clocks of the timed region: the sustained figure (a
     seconds-long loop at the 1 kW power cap) only for a region of >= 1 s in which the sampler saw
@@ -379,14 +399,11 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - t_begin
     staged_ms_per_step = sum(step_ms) / len(step_ms)
-    total_ms = sum(plain_ms)
+    (total_ms,) = max_over_ranks([sum(plain_ms)], dev, world)
     if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
     ms_per_step = total_ms / len(plain_ms)
-    value = world * w.T * len(plain_ms) / (total_ms / 1e3)
+    value = whole_job_rate(world, w.T, len(plain_ms), total_ms)
 
     # ---- end to end through the public API with pinned host buffers
     x_h = x.cpu().pin_memory()
@@ -429,13 +446,10 @@ def run_ours(args, w: mi.Workload, rank: int, world: int, local_rank: int):
         stream.synchronize()
         e2e_pipe_ms = e0.elapsed_time(e1)
         del wss, y_hs
-    if world > 1:
-        t = torch.tensor([e2e_ms, e2e_pipe_ms or 0.0], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0].item())
-        e2e_pipe_ms = float(t[1].item()) if e2e_pipe_ms is not None else None
-    e2e_serial_value = world * w.T * e2e_steps / (e2e_ms / 1e3)
-    e2e_value = world * w.T * e2e_steps / (e2e_pipe_ms / 1e3) if e2e_pipe_ms else e2e_serial_value
+    e2e_ms, pipe_max = max_over_ranks([e2e_ms, e2e_pipe_ms or 0.0], dev, world)
+    e2e_pipe_ms = pipe_max if e2e_pipe_ms is not None else None
+    e2e_serial_value = whole_job_rate(world, w.T, e2e_steps, e2e_ms)
+    e2e_value = whole_job_rate(world, w.T, e2e_steps, e2e_pipe_ms) if e2e_pipe_ms else e2e_serial_value
 
     # ---- roofline of the dominant kernel (gate_up grouped GEMM: ~2/3 of the FLOPs / weight bytes)
     clocks = clk.summary()
@@ -554,6 +568,11 @@ def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     except Exception:
         pass
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize(dev)
     with ClockSampler(gpu_id) as clk, torch.cuda.stream(stream):
         t_begin = time.perf_counter()
         for s in range(args.steps):
@@ -567,6 +586,7 @@ def run_train(args, w: mi.Workload, rank: int, world: int, local_rank: int):
     clocks = clk.summary()
     f_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in evs)
     b_ms = statistics.mean(b.elapsed_time(c) for _, b, c in evs)
+    f_ms, b_ms = max_over_ranks([f_ms, b_ms], dev, world)  # the slowest rank's forward and backward
     step_ms = f_ms + b_ms
     gemm_fwd = w.T * (6.0 * w.k * w.D * w.F + 6.0 * w.D * w.Fs)
     bwd_tflops = 2 * gemm_fwd / (b_ms / 1e3) / 1e12
