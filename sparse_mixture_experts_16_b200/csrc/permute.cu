@@ -10,7 +10,8 @@
 //   3. scatter : per block, one warp walks the block's slots in (token, slot) order; ranks of
 //                equal experts inside each 32-slot step come from __match_any_sync + popc, and
 //                a shared running counter per expert carries them across steps
-//   4. gather  : x_perm[r] = x[perm_token[r]], one warp per row, 16-byte vector moves
+//   4. gather  : x_perm[inv_perm[t*k + j]] = x[t], one warp per token: its row is read once and
+//                written to each of its k rows, 16-byte vector moves
 // For T <= 256 steps 1-4 run as one kernel (dispatch_small_kernel: every CTA sorts, all gather).
 // Within an expert, rows are therefore ordered by token id (a token picks an expert at most once).
 #include <cuda_fp16.h>
@@ -281,21 +282,28 @@ __global__ void __launch_bounds__(256) dispatch_small_kernel(const int32_t* __re
   pdl_trigger();
 }
 
-// x_perm[r] = x[perm_token[r]] for r < offsets[E]; one warp per row, 16-byte moves.
+// x_perm[inv_perm[t*k + j]] = x[t] for every kept slot; one warp per token, 16-byte moves.  Each x
+// row is read once and written to its k rows: read by permuted row instead, a token's row would
+// come from DRAM up to k times, since x (T*D*2 bytes) does not stay in L2 between its k slots.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
-                                                          const int32_t* __restrict__ perm_token,
-                                                          const int32_t* __restrict__ offsets, int E, int T,
-                                                          int D, uint16_t* __restrict__ x_perm) {
+                                                          const int32_t* __restrict__ inv_perm, int T, int k,
+                                                          int D, int M, uint16_t* __restrict__ x_perm) {
   pdl_wait();
-  const int n_rows = offsets[E];
   const int lane = threadIdx.x & 31;
   const int nv = D / 8;
-  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n_rows; r += (gridDim.x * blockDim.x) >> 5) {
-    const int t = perm_token[r];
-    if ((unsigned)t >= (unsigned)T) continue;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += (gridDim.x * blockDim.x) >> 5) {
+    int my_r = lane < k ? inv_perm[(size_t)t * k + lane] : -1;
+    if ((unsigned)my_r >= (unsigned)M) my_r = -1;  // a dropped slot (expert id out of range)
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
-    uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * D);
-    for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+    for (int v0 = 0; v0 < nv; v0 += 32) {  // every lane runs every pass: the shuffles stay warp-uniform
+      const int v = v0 + lane;
+      uint4 a = make_uint4(0u, 0u, 0u, 0u);
+      if (v < nv) a = __ldg(src + v);
+      for (int j = 0; j < k; ++j) {
+        const int r = __shfl_sync(0xffffffffu, my_r, j);
+        if (v < nv && (unsigned)r < (unsigned)M) reinterpret_cast<uint4*>(x_perm + (size_t)r * D)[v] = a;
+      }
+    }
   }
   pdl_trigger();
 }
@@ -384,9 +392,9 @@ cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16
     if (x_perm_f16)
       e = launch_pdl(gather_rows_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, (const int32_t*)perm_token,
                      (const int32_t*)offsets, E, T, D, x_perm);
-    else
-      e = launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, (const int32_t*)perm_token,
-                     (const int32_t*)offsets, E, T, D, x_perm);
+    else  // one warp per token
+      e = launch_pdl(gather_rows_kernel, dim3((unsigned)std::min<long long>(148LL * 16, ((long long)T + 7) / 8)),
+                     dim3(256), 0, s, x, (const int32_t*)inv_perm, T, k, D, T * k, x_perm);
     if (e != cudaSuccess) return e;
     ++launches;
   }
