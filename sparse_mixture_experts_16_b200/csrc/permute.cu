@@ -7,9 +7,10 @@
 // A deterministic, stable counting sort of the T*k (token, slot) pairs by expert id:
 //   1. hist    : per block of 256 tokens, per-expert counts with shared-memory atomics
 //   2. scan    : per expert, exclusive scan over blocks; then exclusive scan over experts
-//   3. scatter : per block, one warp walks the block's slots in (token, slot) order; ranks of
-//                equal experts inside each 32-slot step come from __match_any_sync + popc, and
-//                a shared running counter per expert carries them across steps
+//   3. scatter : per block, eight warps each walk 32 tokens' slots in (token, slot) order: a
+//                first pass counts each warp's slots per expert, a warp-order prefix on the
+//                block's offset gives each warp its start rows, and a second pass hands out rows
+//                (ranks of equal experts inside each 32-slot step from __match_any_sync + popc)
 //   4. gather  : x_perm[inv_perm[t*k + j]] = x[t], one warp per token: its row is read once and
 //                written to each of its k rows, 16-byte vector moves
 // For T <= 256 steps 1-4 run as one kernel (dispatch_small_kernel: every CTA sorts, all gather).
@@ -308,25 +309,6 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   pdl_trigger();
 }
 
-// x_perm16[r] = f16(x[perm_token[r]]) for r < offsets[E]; one warp per row.
-__global__ void __launch_bounds__(256) gather_rows_f16_kernel(const uint16_t* __restrict__ x,
-                                                              const int32_t* __restrict__ perm_token,
-                                                              const int32_t* __restrict__ offsets, int E, int T,
-                                                              int D, uint16_t* __restrict__ x_perm16) {
-  pdl_wait();
-  const int n_rows = offsets[E];
-  const int lane = threadIdx.x & 31;
-  const int nv = D / 8;
-  for (int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < n_rows; r += (gridDim.x * blockDim.x) >> 5) {
-    const int t = perm_token[r];
-    if ((unsigned)t >= (unsigned)T) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * D);
-    uint4* dst = reinterpret_cast<uint4*>(x_perm16 + (size_t)r * D);
-    for (int v = lane; v < nv; v += 32) dst[v] = bf16x8_to_f16x8(__ldg(src + v));
-  }
-  pdl_trigger();
-}
-
 __global__ void __launch_bounds__(256) cast_bf16_to_f16_kernel(const uint16_t* __restrict__ src, long long n8,
                                                                uint16_t* __restrict__ dst) {
   pdl_wait();
@@ -349,6 +331,8 @@ cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16
   const int nb = (T + kTokPerBlock - 1) / kTokPerBlock;
   const bool gather = x != nullptr && x_perm != nullptr && T > 0;
   if (!x_perm_f16) x_cast = nullptr;  // the cast copy exists for the f16 (FP8-weight) path only
+  // f16 rows are for the E4M3-weight decode path (T <= 64), which the one-kernel dispatch serves
+  if (x_perm_f16 && nb > 1) return cudaErrorInvalidValue;
   int launches = 0;
   cudaError_t e = cudaSuccess;
   if (nb == 1) {
@@ -385,21 +369,9 @@ cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16
     if (e != cudaSuccess) return e;
     ++launches;
   }
-  if (gather) {
-    const long long rows = (long long)T * k;
-    long long blocks = (rows + 7) / 8;
-    if (blocks > 148LL * 16) blocks = 148LL * 16;
-    if (x_perm_f16)
-      e = launch_pdl(gather_rows_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, x, (const int32_t*)perm_token,
-                     (const int32_t*)offsets, E, T, D, x_perm);
-    else  // one warp per token
-      e = launch_pdl(gather_rows_kernel, dim3((unsigned)std::min<long long>(148LL * 16, ((long long)T + 7) / 8)),
-                     dim3(256), 0, s, x, (const int32_t*)inv_perm, T, k, D, T * k, x_perm);
-    if (e != cudaSuccess) return e;
-    ++launches;
-  }
-  if (gather && x_cast != nullptr) {
-    e = launch_cast_bf16_to_f16(x, (long long)T * D, x_cast, s);
+  if (gather) {  // one warp per token
+    e = launch_pdl(gather_rows_kernel, dim3((unsigned)std::min<long long>(148LL * 16, ((long long)T + 7) / 8)),
+                   dim3(256), 0, s, x, (const int32_t*)inv_perm, T, k, D, T * k, x_perm);
     if (e != cudaSuccess) return e;
     ++launches;
   }
