@@ -82,3 +82,30 @@ def test_layer_matches_the_oracle_on_every_path(cuda_device, w):
             assert np.sqrt(np.mean((y - y_ref) ** 2)) <= 5e-3 * rms, flags
     idx, _ = moe.moe_router_topk(d["x"], d["wg"], d["bias"], w.k)
     assert (idx.cpu().numpy() == idx_ref).all()
+
+
+def _draw_backward_cases(n=8, seed=20261204):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        T = int(rng.choice([1, 7, 64, 65, 130, 257, 400]))
+        E = int(rng.choice([1, 3, 8, 16, 33, 64]))
+        k = int(rng.integers(1, min(E, 6) + 1))
+        D = 64 * int(rng.integers(1, 6))
+        F = 64 * int(rng.integers(1, 6))
+        Fs = int(rng.choice([0, 64, 128]))
+        bias = str(rng.choice(["none", "normal:0.5"]))
+        cases.append(mi.Workload(f"bwdsweep{i}_T{T}D{D}E{E}k{k}F{F}Fs{Fs}", T=T, D=D, E=E, k=k, F=F, Fs=Fs,
+                                 bias=bias, seed=100 + i))
+    return cases
+
+
+@pytest.mark.parametrize("w", _draw_backward_cases(), ids=lambda w: w.name)
+def test_backward_matches_the_oracle_on_irregular_shapes(cuda_device, w):
+    """The training forward (default tiling) and moe_layer_backward on seeded irregular shapes,
+    every gradient within the backward's normwise bound (RMS(err) <= 1e-2 x RMS, max|err| <=
+    2e-2 x max|oracle|) of the oracle's chain rule."""
+    from test_gpu_backward import _check, _run
+
+    h, d, dy_h, L, y, dx, g = _run(w)
+    _check(w, h, dy_h, dx, g)
