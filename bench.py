@@ -42,19 +42,19 @@ _CSRC = "sparse_mixture_experts_16_b200/csrc/"
 _TRAFFIC = {
     # kernel variant -> (its sources, their sha256, {workload: dram__bytes_read.sum + dram__bytes_write.sum})
     "bf16": ((_CSRC + "grouped_gemm_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
-             "2e3ae53b44d3235d0095eefe97ed358d6e2a12d467004f17987109881b1ff788",
-             {"deepseek": 16.356915e9 + 0.266861e9, "mixtral": 1.946758e9 + 0.226422e9,
-              "gptoss": 1.250717e9 + 0.177929e9, "gptoss_decode_T1": 0.135693e9 + 0.003688e9,
-              "gptoss_decode_T8": 0.707940e9 + 0.003672e9, "gptoss_decode_T32": 1.076501e9 + 0.004444e9,
-              "gptoss_decode_T64": 1.078004e9 + 0.004551e9, "deepseek_decode": 5.876497e9 + 0.004061e9}),
+             "499dcc3232d606bb964c25506e639710b704dc2792467aa0d428d086454b0888",
+             {"deepseek": 16.357346e9 + 0.267214e9, "mixtral": 1.946551e9 + 0.226511e9,
+              "gptoss": 1.250823e9 + 0.179702e9, "gptoss_decode_T1": 0.135693e9 + 0.003212e9,
+              "gptoss_decode_T8": 0.707973e9 + 0.003855e9, "gptoss_decode_T32": 1.076509e9 + 0.003957e9,
+              "gptoss_decode_T64": 1.077995e9 + 0.004742e9, "deepseek_decode": 5.876478e9 + 0.004464e9}),
     "bf16_wide": ((_CSRC + "grouped_gemm_wide_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
                   "", {}),
     "bf16_pair": ((_CSRC + "grouped_gemm_pair_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
                   "", {}),
     "fp8": ((_CSRC + "stream_fp8w_sm100.cu", _CSRC + "sm100_ptx.cuh", _CSRC + "moe_common.cuh"),
-            "fc2cfda7d3d5a31b0b7b6b8abce333afa5af1632c38be3817c2e48fc4ea5a7c3",
-            {"deepseek_decode": 2.942542e9 + 0.003802e9, "gptoss_decode_T1": 0.067338e9 + 0.001457e9,
-             "gptoss_decode_T8": 0.364154e9 + 0.003587e9, "gptoss_decode_T64": 0.556272e9 + 0.004443e9}),
+            "bc15fd3599b4d7d25cc3852951449f0a47e6a1ae2b5adb086609c2d1f4a02174",
+            {"deepseek_decode": 2.942161e9 + 0.004544e9, "gptoss_decode_T1": 0.067342e9 + 0.000812e9,
+             "gptoss_decode_T8": 0.364131e9 + 0.004026e9, "gptoss_decode_T64": 0.556408e9 + 0.004305e9}),
 }
 
 

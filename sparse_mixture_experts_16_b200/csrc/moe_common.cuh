@@ -197,7 +197,5 @@ cudaError_t launch_stream_fp8w(GemmKind kind, const GemmSetHost* sets, const flo
 cudaError_t launch_quantize_rows_fp8(const uint16_t* w, long long rows, int K, uint8_t* q, float* scales,
                                      cudaStream_t s);
 
-// x_perm rows as f16 (x_perm16[r] = f16(x[perm_token[r]])) and a plain bf16 -> f16 cast.
-cudaError_t launch_cast_bf16_to_f16(const uint16_t* src, long long n, uint16_t* dst, cudaStream_t s);
 
 }  // namespace moe

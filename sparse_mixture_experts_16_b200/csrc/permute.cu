@@ -309,14 +309,6 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
   pdl_trigger();
 }
 
-__global__ void __launch_bounds__(256) cast_bf16_to_f16_kernel(const uint16_t* __restrict__ src, long long n8,
-                                                               uint16_t* __restrict__ dst) {
-  pdl_wait();
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x)
-    reinterpret_cast<uint4*>(dst)[i] = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(src) + i));
-  pdl_trigger();
-}
-
 }  // namespace
 
 size_t permute_scratch_bytes(int T, int E) {
@@ -377,14 +369,6 @@ cudaError_t launch_permute(const int32_t* idx, const float* topk_w, const uint16
   }
   if (n_launches) *n_launches = launches;
   return cudaGetLastError();
-}
-
-cudaError_t launch_cast_bf16_to_f16(const uint16_t* src, long long n, uint16_t* dst, cudaStream_t s) {
-  if (n == 0) return cudaSuccess;
-  const long long n8 = n / 8;
-  long long blocks = (n8 + 255) / 256;
-  if (blocks > 148LL * 8) blocks = 148LL * 8;
-  return launch_pdl(cast_bf16_to_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, src, n8, dst);
 }
 
 }  // namespace moe
